@@ -1,0 +1,205 @@
+/*
+ * tq.h -- C ABI of the B200 TurboQuant packed-KV library (libtq.so).
+ *
+ * Two operations make up the hot path:
+ *
+ *   tq_quantize_append  rotate each K/V row with a randomized Hadamard transform,
+ *                       store its fp32 L2 norm, Lloyd-Max-encode every rotated unit
+ *                       coordinate and bit-pack the codes into the row's page slot;
+ *   tq_paged_decode     one attention decode step straight over the packed pages:
+ *                       rotate q once, score each key on its codes, online softmax,
+ *                       accumulate V in the rotated domain, inverse-rotate the output.
+ *
+ * Sources (page title, section):
+ *   TorbuQuant (ginkgoq.github.io/TurboQuant), "TQ4 page tensor" diagram -- page
+ *     tensor [num_blocks, block_size, num_kv_heads, slot_bytes], slot -> (block, row),
+ *     slot = [K: packed indices, fp32 norm][V: packed indices, fp32 norm],
+ *     K bytes ceil(D*k_bits/8)+4, V bytes ceil(D*v_bits/8)+4, optional padding;
+ *     the stages "Quantize: rotate, normalize, codebook-encode, pack" and "Store".
+ *   tq-kv (shadowgraph.io), "How It Works" step 3 (randomized Hadamard transform)
+ *     and "Library API" (generate_signs(dim, seed), pre_rotate_query_with_signs,
+ *     fused_attention_scores on compressed keys); "Custom CUDA Kernel Stack"
+ *     (flash decode with split-KV and online softmax; attention score without
+ *     decompression).
+ *   turboquant_serve 0.1.2, "Architecture" (update(): rotate, normalize,
+ *     Lloyd-Max encode, bit-pack; _decode(): unpack, decode, restore magnitude,
+ *     rotate back; one rotation per head_dim; codebooks fitted once and shared).
+ *   turboquant_pro 1.4.2, "How It Works" (norm preserved alongside the bits;
+ *     8 x 3-bit = 3 bytes) and "Fused CUDA decode" (split-K decode on the codes).
+ *
+ * Conventions where the pages are silent (the library and its tests agree on them):
+ *   - signs: s_j = -1 if bit 63 of the j-th SplitMix64 output seeded with
+ *     sign_seed is set, else +1 (j = 0..D-1); the same signs serve K, V, q and
+ *     every head; rotation y = (1/sqrt(D)) H (s * x), H the natural-order
+ *     (Sylvester) Hadamard matrix;
+ *   - norm: L2 norm of the input row, stored as fp32; unit coordinates u = y / n;
+ *   - code: idx = number of boundaries b_i with b_i < u (ties to the lower cell);
+ *     a zero row stores norm 0 and codes idx(0); a row holding a non-finite value
+ *     stores codes 0 and a quiet-NaN norm (0x7FC00000) and raises
+ *     TQ_DEVERR_NONFINITE;
+ *   - packing: code j fills bits [j*bits, (j+1)*bits) of a little-endian bit
+ *     stream (bit p = bit p%8 of byte p/8); the fp32 norm follows, little endian;
+ *   - GQA: query head h reads KV head h / (H_q / H_kv).
+ *
+ * Memory: every pointer below is a DEVICE pointer unless stated otherwise.  The
+ * caller owns all buffers.  Calls are asynchronous on `stream` (a cudaStream_t
+ * passed as void*, NULL = legacy default stream); host-side validation errors are
+ * returned synchronously and nothing is enqueued.  Errors found by a kernel (an
+ * out-of-range slot or block id, a non-finite input row) are OR-ed into a
+ * per-device error word read by tq_get_device_error(); the offending row or
+ * block is skipped, nothing faults.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,  /* bad pointer, shape, stride, dtype or parameter   */
+  TQ_ERR_UNSUPPORTED = 2,  /* valid but not built: head_dim, bits or GQA group */
+  TQ_ERR_CUDA = 3,         /* a CUDA runtime call failed (launch, memcpy, ...)  */
+  TQ_ERR_DEVICE = 4,       /* a kernel reported an error (see the error word)  */
+  TQ_ERR_WORKSPACE = 5     /* workspace missing or too small                    */
+} tq_status;
+
+typedef enum {
+  TQ_U8 = 0,
+  TQ_I32 = 1,
+  TQ_I64 = 2,
+  TQ_F32 = 3,
+  TQ_BF16 = 4,
+  TQ_F16 = 5
+} tq_dtype;
+
+/* Device error word bits (tq_get_device_error). */
+#define TQ_DEVERR_SLOT_RANGE 0x1    /* slot_mapping entry >= num_blocks*block_size */
+#define TQ_DEVERR_BLOCK_RANGE 0x2   /* block_table entry outside [0, num_blocks)   */
+#define TQ_DEVERR_NONFINITE 0x4     /* a K/V input row held a NaN or an infinity   */
+#define TQ_DEVERR_SEQLEN_RANGE 0x8  /* seq_len < 0 or > max_blocks*block_size      */
+
+/* A strided view of a device array.  Strides are in ELEMENTS; shape[i] and
+ * stride[i] for i >= ndim are ignored.  data must be aligned to the element size. */
+typedef struct {
+  void* data;
+  int32_t dtype;      /* tq_dtype */
+  int32_t ndim;
+  int64_t shape[4];
+  int64_t stride[4];
+} tq_tensor;
+
+/* One fp32 Lloyd-Max table (Beta-sphere density for `dim`): `centroids` holds
+ * 2^bits ascending values, `boundaries` the 2^bits - 1 ascending cell edges.
+ * Both are device pointers, 4-byte aligned, owned by the caller and read by
+ * every launch ("fitted once ... and shared", turboquant_serve, "Codebook sharing"). */
+typedef struct {
+  int32_t dim;
+  int32_t bits;
+  const float* centroids;
+  const float* boundaries;
+} tq_codebook;
+
+typedef struct {
+  tq_codebook k;
+  tq_codebook v;
+} tq_codebooks;
+
+/* Bytes of one slot before padding: (ceil(D*k_bits/8)+4) + (ceil(D*v_bits/8)+4)
+ * (TorbuQuant, "TQ4 page tensor").  Host only; *out receives the value.
+ * Errors: TQ_ERR_INVALID_ARG for dim < 1, bits outside 1..8 or out == NULL. */
+TQ_API tq_status tq_slot_bytes(int32_t dim, int32_t k_bits, int32_t v_bits, int32_t* out);
+
+/* Quantize-append (TorbuQuant "Quantize" and "Store"; turboquant_serve update()).
+ *
+ *   pages        u8  [num_blocks, block_size, H_kv, slot_stride]; the last dim is
+ *                contiguous, slot_stride >= tq_slot_bytes(D, k_bits, v_bits) and a
+ *                multiple of 8; bytes beyond slot_bytes are never written.
+ *   slot_mapping i64 [T]: token t goes to slot s = slot_mapping[t], i.e.
+ *                page[s / block_size, s % block_size, h, :] for every KV head h;
+ *                s < 0 skips the token; s >= num_blocks*block_size skips it and
+ *                raises TQ_DEVERR_SLOT_RANGE.
+ *   k, v         [T, H_kv, D] in bf16, f16 or f32 (same dtype); the last dim is
+ *                contiguous; rows are read exactly (converted to fp32).
+ *   cb           host pointer to the K and V tables (device arrays inside);
+ *                cb->k.dim == cb->v.dim == D, cb->k.bits == k_bits, cb->v.bits == v_bits.
+ *   sign_seed    SplitMix64 seed of the rotation signs.
+ *   k_bits, v_bits  1..8.  D must be 64, 128 or 256.
+ * Two tokens mapped to the same slot race (either row may win).
+ * Errors: TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED (nothing enqueued), TQ_ERR_CUDA. */
+TQ_API tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_tensor k,
+                             tq_tensor v, const tq_codebooks* cb, uint64_t sign_seed,
+                             int32_t k_bits, int32_t v_bits, void* stream);
+
+/* Paged decode (tq-kv "Library API" fused scores on compressed keys; "Custom CUDA
+ * Kernel Stack" flash decode v2 split-KV with online softmax; turboquant_pro
+ * "Fused CUDA decode").
+ *
+ *   out          [B, H_q, D], f32 or the dtype of q; last dim contiguous.
+ *                out[b, h] = sum_t softmax_t(scale * <q[b,h], k_hat_t>) v_hat_t over
+ *                t < seq_lens[b], where k_hat/v_hat are the dequantized rows
+ *                norm * R^T c[idx] of KV head h / (H_q/H_kv).  seq_lens[b] == 0 gives 0.
+ *   q            [B, H_q, D] in bf16, f16 or f32; last dim contiguous.
+ *   pages        as in tq_quantize_append (k_bits/v_bits taken from cb).
+ *   block_table  i32 [B, max_blocks]: token t of sequence b lives in block
+ *                block_table[b, t / block_size], row t % block_size.  Entries past
+ *                the sequence are not read.  An entry outside [0, num_blocks) raises
+ *                TQ_DEVERR_BLOCK_RANGE and its block is skipped.
+ *   seq_lens     i32 [B]; 0 <= seq_lens[b] <= max_blocks * block_size, otherwise
+ *                TQ_DEVERR_SEQLEN_RANGE and the sequence gives 0.
+ *   scale        softmax scale (typically 1/sqrt(D)).
+ * H_q must be a multiple of H_kv with H_q / H_kv <= 16; block_size must be 16.
+ * Uses the per-device workspace (tq_set_workspace, or allocated by the library on
+ * the first call that needs more, and kept until process exit).
+ * Errors: TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED / TQ_ERR_WORKSPACE (nothing
+ * enqueued), TQ_ERR_CUDA. */
+TQ_API tq_status tq_paged_decode(tq_tensor out, tq_tensor q, tq_tensor pages,
+                          tq_tensor block_table, tq_tensor seq_lens,
+                          const tq_codebooks* cb, uint64_t sign_seed, float scale,
+                          void* stream);
+
+/* Workspace bytes tq_paged_decode needs for this geometry (host only).  The
+ * workspace holds the split-KV partial results (m, l, O') in fp32. */
+TQ_API tq_status tq_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                   int32_t head_dim, int32_t max_blocks, int32_t block_size,
+                                   size_t* bytes);
+
+/* Give the library a caller-owned device workspace for the CURRENT device
+ * (ptr 256-byte aligned; NULL releases the association).  The library never frees
+ * it.  Calls that use one device's workspace must be ordered on the GPU (one stream,
+ * or events); concurrent decodes on one device race on it. */
+TQ_API tq_status tq_set_workspace(void* ptr, size_t bytes);
+
+/* Read and clear the current device's error word (TQ_DEVERR_* bits).  Host
+ * pointer `out`; synchronises `stream` first. */
+TQ_API tq_status tq_get_device_error(int32_t* out, void* stream);
+
+/* Test export of the rotation used by tq_quantize_append: for each row x of
+ * `x` [N, D] (bf16/f16/f32), writes u = y / n with y = (1/sqrt(D)) H (s*x), n = ||x||,
+ * in fp32 to `u` [N, D] and fp32(n) to `norm` [N], computed with exactly the
+ * device arithmetic the append kernel uses (so encoding these u on the host
+ * reproduces the kernel's codes bit for bit). */
+TQ_API tq_status tq_rotate_unit(tq_tensor u, tq_tensor norm, tq_tensor x, uint64_t sign_seed,
+                         void* stream);
+
+/* Static description of a status code (never NULL). */
+TQ_API const char* tq_status_string(tq_status status);
+
+/* Library version, e.g. "0.1.0". */
+TQ_API const char* tq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */

@@ -1,0 +1,36 @@
+"""B200-native TurboQuant packed-KV quantize-append and paged decode.
+
+Thin Python binding over the C ABI of ``libtq.so`` (declared in
+``include/tq.h``).  Every step of the hot path runs in the library's CUDA
+kernels; this module only marshals torch tensors into ``tq_tensor`` views and
+checks status codes.  There is no CPU fallback: if the library is missing or a
+call fails, an exception is raised.
+
+Public API (names follow the C entry points):
+    slot_bytes(D, k_bits, v_bits) -> int
+    load_codebooks(D, k_bits, v_bits, device) -> Codebooks
+    quantize_append(pages, slot_mapping, k, v, codebooks, sign_seed, stream=None)
+    paged_decode(out, q, pages, block_table, seq_lens, codebooks, sign_seed, scale, stream=None)
+    rotate_unit(u, norm, x, sign_seed, stream=None)       # test export of the rotation
+    decode_workspace_size(...), set_workspace(tensor), get_device_error(stream=None)
+"""
+
+from ._binding import (  # noqa: F401
+    Codebooks,
+    TQError,
+    DEVERR_BLOCK_RANGE,
+    DEVERR_NONFINITE,
+    DEVERR_SEQLEN_RANGE,
+    DEVERR_SLOT_RANGE,
+    decode_workspace_size,
+    get_device_error,
+    library_path,
+    load_codebook_table,
+    load_codebooks,
+    paged_decode,
+    quantize_append,
+    rotate_unit,
+    set_workspace,
+    slot_bytes,
+    version,
+)

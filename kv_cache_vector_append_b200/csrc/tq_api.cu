@@ -1,0 +1,413 @@
+// tq_api.cu -- the extern "C" boundary of libtq.so (declared in include/tq.h):
+// argument validation, kernel dispatch, per-device workspace and error word.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "tq.h"
+#include "tq_launch.cuh"
+
+namespace tq {
+
+__device__ unsigned int g_tq_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  unsigned int* err = nullptr;   // device address of g_tq_error_word
+  void* user_ws = nullptr;
+  size_t user_ws_bytes = 0;
+  void* lib_ws = nullptr;
+  size_t lib_ws_bytes = 0;
+  DeviceInfo info;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+tq_status device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TQ_ERR_CUDA;
+  DeviceState& s = g_dev[dev];
+  if (s.err == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_tq_error_word) != cudaSuccess) return TQ_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&s.info.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return TQ_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&s.info.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+        cudaSuccess)
+      return TQ_ERR_CUDA;
+    s.err = (unsigned int*)p;
+  }
+  *out = &s;
+  return TQ_OK;
+}
+
+int dtype_size(int32_t dt) {
+  switch (dt) {
+    case TQ_U8: return 1;
+    case TQ_I32: return 4;
+    case TQ_I64: return 8;
+    case TQ_F32: return 4;
+    case TQ_BF16: return 2;
+    case TQ_F16: return 2;
+    default: return 0;
+  }
+}
+
+bool is_float_dtype(int32_t dt) { return dt == TQ_F32 || dt == TQ_BF16 || dt == TQ_F16; }
+
+int region_bytes(int dim, int bits) { return (dim * bits + 7) / 8 + 4; }
+
+bool valid_tensor(const tq_tensor& t, int ndim) {
+  if (t.ndim != ndim || t.data == nullptr || dtype_size(t.dtype) == 0) return false;
+  for (int i = 0; i < ndim; ++i)
+    if (t.shape[i] < 0) return false;
+  if ((uintptr_t)t.data % (uintptr_t)dtype_size(t.dtype) != 0) return false;
+  return true;
+}
+
+bool valid_codebook(const tq_codebook& c, int dim) {
+  return c.dim == dim && c.bits >= 1 && c.bits <= 8 && c.centroids != nullptr &&
+         c.boundaries != nullptr && (uintptr_t)c.centroids % 4 == 0 &&
+         (uintptr_t)c.boundaries % 4 == 0;
+}
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int align_mode_of(const void* data, int esize, std::initializer_list<int64_t> strides) {
+  auto ok = [&](int a) {
+    if ((uintptr_t)data % a) return false;
+    for (int64_t s : strides)
+      if ((s * esize) % a) return false;
+    return true;
+  };
+  if (ok(16)) return 16;
+  if (ok(4)) return 4;
+  return 0;
+}
+
+size_t decode_smem_bytes(int dim, int kb, int vb, int h_q, int h_kv, int slot_stride, int wph,
+                         int nstage) {
+  auto lut_words = [](int b) { return b <= 4 ? (1 << (2 * b)) : (1 << b) / 2; };
+  size_t lut = ((size_t)(lut_words(kb) + lut_words(vb)) * 4 + 127) / 128 * 128;
+  size_t q = (size_t)h_q * dim * 4;
+  size_t stage = (size_t)kBlockSize * h_kv * slot_stride * wph;
+  return lut + q + 128 + nstage * stage;
+}
+
+tq_status plan_decode(int batch, int h_q, int h_kv, int dim, int kb, int vb, int slot_stride,
+                      int max_blocks, const DeviceInfo& di, DecodePlan* plan) {
+  if (h_kv < 1 || h_kv > kDecodeWarps) return TQ_ERR_UNSUPPORTED;
+  plan->wph = kDecodeWarps / h_kv;
+  plan->nstage = 4;
+  plan->smem = decode_smem_bytes(dim, kb, vb, h_q, h_kv, slot_stride, plan->wph, 4);
+  while ((int)plan->smem > di.max_smem_optin && plan->wph > 1) {
+    plan->wph /= 2;
+    plan->smem = decode_smem_bytes(dim, kb, vb, h_q, h_kv, slot_stride, plan->wph, 4);
+  }
+  if ((int)plan->smem > di.max_smem_optin) {
+    plan->nstage = 2;
+    plan->smem = decode_smem_bytes(dim, kb, vb, h_q, h_kv, slot_stride, plan->wph, 2);
+    if ((int)plan->smem > di.max_smem_optin) return TQ_ERR_UNSUPPORTED;
+  }
+  const int resident = std::max(1, std::min(4, (int)(228 * 1024 / (plan->smem + 1024))));
+  const int target = di.num_sms * resident * 2;
+  const int steps_max = std::max(1, (max_blocks + plan->wph - 1) / plan->wph);
+  int nsplit = std::max(1, std::min(steps_max, (target + batch - 1) / std::max(batch, 1)));
+  int spb = ((max_blocks + nsplit - 1) / nsplit + plan->wph - 1) / plan->wph * plan->wph;
+  spb = std::max(spb, plan->wph);
+  nsplit = std::max(1, (max_blocks + spb - 1) / spb);
+  plan->nsplit = nsplit;
+  plan->spb = spb;
+  plan->ws_bytes = (size_t)batch * nsplit * plan->wph * h_q * (dim + 2) * sizeof(float);
+  return TQ_OK;
+}
+
+}  // namespace
+}  // namespace tq
+
+using namespace tq;
+
+extern "C" {
+
+const char* tq_version(void) { return "0.1.0"; }
+
+const char* tq_status_string(tq_status s) {
+  switch (s) {
+    case TQ_OK: return "ok";
+    case TQ_ERR_INVALID_ARG: return "invalid argument";
+    case TQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TQ_ERR_CUDA: return "CUDA runtime error";
+    case TQ_ERR_DEVICE: return "device-side error reported";
+    case TQ_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+tq_status tq_slot_bytes(int32_t dim, int32_t k_bits, int32_t v_bits, int32_t* out) {
+  if (out == nullptr || dim < 1 || k_bits < 1 || k_bits > 8 || v_bits < 1 || v_bits > 8)
+    return TQ_ERR_INVALID_ARG;
+  *out = region_bytes(dim, k_bits) + region_bytes(dim, v_bits);
+  return TQ_OK;
+}
+
+tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_tensor k, tq_tensor v,
+                             const tq_codebooks* cb, uint64_t sign_seed, int32_t k_bits,
+                             int32_t v_bits, void* stream) {
+  if (cb == nullptr) return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(pages, 4) || pages.dtype != TQ_U8 || pages.stride[3] != 1)
+    return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(slot_mapping, 1) || slot_mapping.dtype != TQ_I64) return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(k, 3) || !valid_tensor(v, 3) || !is_float_dtype(k.dtype) ||
+      k.dtype != v.dtype || k.stride[2] != 1 || v.stride[2] != 1)
+    return TQ_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (k.shape[i] != v.shape[i]) return TQ_ERR_INVALID_ARG;
+  const int64_t T = k.shape[0];
+  const int h_kv = (int)k.shape[1];
+  const int D = (int)k.shape[2];
+  if (slot_mapping.shape[0] != T || pages.shape[2] != h_kv) return TQ_ERR_INVALID_ARG;
+  if (k_bits < 1 || k_bits > 8 || v_bits < 1 || v_bits > 8) return TQ_ERR_INVALID_ARG;
+  if (!valid_codebook(cb->k, D) || !valid_codebook(cb->v, D) || cb->k.bits != k_bits ||
+      cb->v.bits != v_bits)
+    return TQ_ERR_INVALID_ARG;
+  if (D != 64 && D != 128 && D != 256) return TQ_ERR_UNSUPPORTED;
+  const int kb = region_bytes(D, k_bits), vb = region_bytes(D, v_bits);
+  if (pages.shape[3] < kb + vb || pages.shape[3] % 8 != 0) return TQ_ERR_INVALID_ARG;
+  if (pages.stride[0] % 4 || pages.stride[1] % 4 || pages.stride[2] % 4 ||
+      (uintptr_t)pages.data % 4)
+    return TQ_ERR_INVALID_ARG;
+  if (T == 0 || h_kv == 0) return TQ_OK;
+  DeviceState* ds = nullptr;
+  tq_status s = device_state(&ds);
+  if (s != TQ_OK) return s;
+
+  AppendParams p{};
+  p.pages = (uint8_t*)pages.data;
+  p.num_slots = pages.shape[0] * pages.shape[1];
+  p.block_size = (int32_t)pages.shape[1];
+  p.h_kv = h_kv;
+  p.blk_stride = pages.stride[0];
+  p.row_stride = pages.stride[1];
+  p.head_stride = pages.stride[2];
+  p.slot_mapping = (const int64_t*)slot_mapping.data;
+  p.slot_map_stride = slot_mapping.stride[0];
+  p.num_tokens = T;
+  p.src[0] = k.data;
+  p.src[1] = v.data;
+  p.tok_stride[0] = k.stride[0];
+  p.tok_stride[1] = v.stride[0];
+  p.head_stride_in[0] = k.stride[1];
+  p.head_stride_in[1] = v.stride[1];
+  p.boundaries[0] = cb->k.boundaries;
+  p.boundaries[1] = cb->v.boundaries;
+  p.bits[0] = k_bits;
+  p.bits[1] = v_bits;
+  p.region_off[0] = 0;
+  p.region_off[1] = kb;
+  p.sign_seed = sign_seed;
+  p.err = ds->err;
+  const int es = dtype_size(k.dtype);
+  p.align_mode = std::min(align_mode_of(k.data, es, {k.stride[0], k.stride[1]}),
+                          align_mode_of(v.data, es, {v.stride[0], v.stride[1]}));
+  if (p.align_mode == 16 &&
+      (align_mode_of(k.data, es, {k.stride[0], k.stride[1]}) != 16 ||
+       align_mode_of(v.data, es, {v.stride[0], v.stride[1]}) != 16))
+    p.align_mode = 4;
+  if (k.dtype == TQ_F32 && p.align_mode == 0) return TQ_ERR_INVALID_ARG;
+  return launch_append_any(D, k.dtype, p, ds->info, as_stream(stream));
+}
+
+tq_status tq_rotate_unit(tq_tensor u, tq_tensor norm, tq_tensor x, uint64_t sign_seed,
+                         void* stream) {
+  if (!valid_tensor(x, 2) || !valid_tensor(u, 2) || !valid_tensor(norm, 1)) return TQ_ERR_INVALID_ARG;
+  if (!is_float_dtype(x.dtype) || u.dtype != TQ_F32 || norm.dtype != TQ_F32) return TQ_ERR_INVALID_ARG;
+  if (x.stride[1] != 1 || u.stride[1] != 1 || u.shape[0] != x.shape[0] ||
+      u.shape[1] != x.shape[1] || norm.shape[0] != x.shape[0])
+    return TQ_ERR_INVALID_ARG;
+  const int D = (int)x.shape[1];
+  if (D != 64 && D != 128 && D != 256) return TQ_ERR_UNSUPPORTED;
+  if (x.shape[0] == 0) return TQ_OK;
+  DeviceState* ds = nullptr;
+  tq_status s = device_state(&ds);
+  if (s != TQ_OK) return s;
+  RotateParams p{};
+  p.x = x.data;
+  p.x_row_stride = x.stride[0];
+  p.rows = x.shape[0];
+  p.u = (float*)u.data;
+  p.u_row_stride = u.stride[0];
+  p.norm = (float*)norm.data;
+  p.norm_stride = norm.stride[0];
+  p.sign_seed = sign_seed;
+  p.align_mode = align_mode_of(x.data, dtype_size(x.dtype), {x.stride[0]});
+  if (x.dtype == TQ_F32 && p.align_mode == 0) return TQ_ERR_INVALID_ARG;
+  return launch_rotate_any(D, x.dtype, p, ds->info, as_stream(stream));
+}
+
+tq_status tq_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                   int32_t head_dim, int32_t max_blocks, int32_t block_size,
+                                   size_t* bytes) {
+  if (bytes == nullptr || batch < 0 || num_q_heads < 1 || num_kv_heads < 1 || max_blocks < 0 ||
+      block_size != kBlockSize || num_q_heads % num_kv_heads)
+    return TQ_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  tq_status s = device_state(&ds);
+  if (s != TQ_OK) return s;
+  // the worst case over supported bit widths: 8-bit K and V (largest slots)
+  DecodePlan plan;
+  const int slot = region_bytes(head_dim, 8) * 2;
+  s = plan_decode(std::max(batch, 1), num_q_heads, num_kv_heads, head_dim, 8, 8, slot,
+                  std::max(max_blocks, 1), ds->info, &plan);
+  if (s != TQ_OK) return s;
+  // smaller slots can only give more stages of the same split plan, never a larger one
+  DecodePlan small;
+  plan_decode(std::max(batch, 1), num_q_heads, num_kv_heads, head_dim, 1, 1,
+              region_bytes(head_dim, 1) * 2, std::max(max_blocks, 1), ds->info, &small);
+  *bytes = std::max(plan.ws_bytes, small.ws_bytes);
+  return TQ_OK;
+}
+
+tq_status tq_set_workspace(void* ptr, size_t bytes) {
+  DeviceState* ds = nullptr;
+  tq_status s = device_state(&ds);
+  if (s != TQ_OK) return s;
+  if (ptr != nullptr && (uintptr_t)ptr % 256) return TQ_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  ds->user_ws = ptr;
+  ds->user_ws_bytes = ptr ? bytes : 0;
+  return TQ_OK;
+}
+
+tq_status tq_get_device_error(int32_t* out, void* stream) {
+  if (out == nullptr) return TQ_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  tq_status s = device_state(&ds);
+  if (s != TQ_OK) return s;
+  cudaStream_t st = as_stream(stream);
+  unsigned int h = 0;
+  if (cudaMemcpyAsync(&h, ds->err, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  if (cudaMemsetAsync(ds->err, 0, sizeof(unsigned int), st) != cudaSuccess) return TQ_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return TQ_ERR_CUDA;
+  *out = (int32_t)h;
+  return TQ_OK;
+}
+
+tq_status tq_paged_decode(tq_tensor out, tq_tensor q, tq_tensor pages, tq_tensor block_table,
+                          tq_tensor seq_lens, const tq_codebooks* cb, uint64_t sign_seed,
+                          float scale, void* stream) {
+  if (cb == nullptr || !std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(q, 3) || !is_float_dtype(q.dtype) || q.stride[2] != 1) return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(out, 3) || !is_float_dtype(out.dtype) || out.stride[2] != 1 ||
+      (out.dtype != TQ_F32 && out.dtype != q.dtype))
+    return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(pages, 4) || pages.dtype != TQ_U8) return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(block_table, 2) || block_table.dtype != TQ_I32 || block_table.stride[1] != 1)
+    return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(seq_lens, 1) || seq_lens.dtype != TQ_I32 || seq_lens.stride[0] != 1)
+    return TQ_ERR_INVALID_ARG;
+  const int B = (int)q.shape[0], h_q = (int)q.shape[1], D = (int)q.shape[2];
+  const int h_kv = (int)pages.shape[2];
+  for (int i = 0; i < 3; ++i)
+    if (out.shape[i] != q.shape[i]) return TQ_ERR_INVALID_ARG;
+  if (block_table.shape[0] != B || seq_lens.shape[0] != B) return TQ_ERR_INVALID_ARG;
+  if (h_kv < 1 || h_q % h_kv) return TQ_ERR_INVALID_ARG;
+  if (!valid_codebook(cb->k, D) || !valid_codebook(cb->v, D)) return TQ_ERR_INVALID_ARG;
+  const int kbits = cb->k.bits, vbits = cb->v.bits;
+  const int kb = region_bytes(D, kbits), vb = region_bytes(D, vbits);
+  const int64_t stride = pages.shape[3];
+  if (stride < kb + vb || stride % 8) return TQ_ERR_INVALID_ARG;
+  // contiguous page tensor: whole blocks are staged with 16-byte copies
+  if (pages.stride[3] != 1 || pages.stride[2] != stride || pages.stride[1] != h_kv * stride ||
+      pages.stride[0] != pages.shape[1] * h_kv * stride || (uintptr_t)pages.data % 16)
+    return TQ_ERR_INVALID_ARG;
+  if (pages.shape[1] != kBlockSize) return TQ_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128 && D != 256) return TQ_ERR_UNSUPPORTED;
+  if (h_q / h_kv > 16 || h_kv > kDecodeWarps) return TQ_ERR_UNSUPPORTED;
+  if (!decode_bits_supported(kbits, vbits)) return TQ_ERR_UNSUPPORTED;
+  if (B == 0) return TQ_OK;
+  DeviceState* ds = nullptr;
+  tq_status s = device_state(&ds);
+  if (s != TQ_OK) return s;
+  const int max_blocks = std::max<int>(1, (int)block_table.shape[1]);
+  DecodePlan plan;
+  s = plan_decode(B, h_q, h_kv, D, kbits, vbits, (int)stride, max_blocks, ds->info, &plan);
+  if (s != TQ_OK) return s;
+
+  float* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (ds->user_ws != nullptr) {
+      if (ds->user_ws_bytes < plan.ws_bytes) return TQ_ERR_WORKSPACE;
+      ws = (float*)ds->user_ws;
+    } else {
+      if (ds->lib_ws_bytes < plan.ws_bytes) {
+        if (ds->lib_ws) cudaFree(ds->lib_ws);
+        ds->lib_ws = nullptr;
+        ds->lib_ws_bytes = 0;
+        size_t want = std::max<size_t>(plan.ws_bytes, 1 << 20);
+        if (cudaMalloc(&ds->lib_ws, want) != cudaSuccess) return TQ_ERR_WORKSPACE;
+        ds->lib_ws_bytes = want;
+      }
+      ws = (float*)ds->lib_ws;
+    }
+  }
+
+  DecodeParams p{};
+  p.pages = (const uint8_t*)pages.data;
+  p.num_blocks = (int32_t)pages.shape[0];
+  p.h_kv = h_kv;
+  p.slot_stride = (int32_t)stride;
+  p.blk_stride = pages.stride[0];
+  p.block_table = (const int32_t*)block_table.data;
+  p.bt_stride = block_table.stride[0];
+  p.max_blocks = (int32_t)block_table.shape[1];
+  p.seq_lens = (const int32_t*)seq_lens.data;
+  p.batch = B;
+  p.q = q.data;
+  p.q_bstride = q.stride[0];
+  p.q_hstride = q.stride[1];
+  p.q_dtype = q.dtype;
+  p.h_q = h_q;
+  p.group = h_q / h_kv;
+  p.kc = cb->k.centroids;
+  p.vc = cb->v.centroids;
+  p.k_region = kb;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.sign_seed = sign_seed;
+  p.wph = plan.wph;
+  p.spb = plan.spb;
+  p.nsplit = plan.nsplit;
+  p.ws = ws;
+  p.err = ds->err;
+
+  MergeParams m{};
+  m.ws = ws;
+  m.out = out.data;
+  m.o_bstride = out.stride[0];
+  m.o_hstride = out.stride[1];
+  m.out_dtype = out.dtype;
+  m.h_q = h_q;
+  m.nsplit = plan.nsplit;
+  m.wph = plan.wph;
+  m.spb = plan.spb;
+  m.max_blocks = p.max_blocks;
+  m.seq_lens = p.seq_lens;
+  m.sign_seed = sign_seed;
+
+  cudaStream_t st = as_stream(stream);
+  switch (D) {
+    case 64: return launch_decode_d64(kbits, vbits, p, m, plan, st);
+    case 128: return launch_decode_d128(kbits, vbits, p, m, plan, st);
+    default: return launch_decode_d256(kbits, vbits, p, m, plan, st);
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,6 @@
+// Quantize-append kernels for head_dim 128, f32 input.
+#include "tq_append_launch.cuh"
+
+namespace tq {
+TQ_DEFINE_APPEND(128, f32, float)
+}  // namespace tq

@@ -1,0 +1,6 @@
+// Quantize-append kernels for head_dim 256, f16 input.
+#include "tq_append_launch.cuh"
+
+namespace tq {
+TQ_DEFINE_APPEND(256, f16, __half)
+}  // namespace tq

@@ -1,0 +1,74 @@
+// tq_append_launch.cuh -- host launchers of the append and rotation-export
+// kernels, instantiated once per (head_dim, input dtype) translation unit.
+#pragma once
+
+#include "tq_launch.cuh"
+
+namespace tq {
+
+template <int D, typename Tin>
+tq_status launch_append_t(const AppendParams& p, const DeviceInfo& di, cudaStream_t st) {
+  const size_t smem = append_smem_bytes<D>(InType<Tin>::kBytes);
+  if ((int)smem > di.max_smem_optin) return TQ_ERR_UNSUPPORTED;
+  auto kern = append_kernel<D, Tin>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return TQ_ERR_CUDA;
+  using G = AppendGeom<D>;
+  const int64_t tiles = 2 * ((p.num_tokens * p.h_kv + G::ROWS - 1) / G::ROWS);
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kAppendWarps * 32, smem) !=
+      cudaSuccess)
+    per_sm = 1;
+  per_sm = std::max(per_sm, 1);
+  const int64_t max_ctas = (int64_t)di.num_sms * per_sm;
+  const int64_t want = (tiles + kAppendWarps - 1) / kAppendWarps;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, max_ctas));
+  kern<<<grid, kAppendWarps * 32, smem, st>>>(p);
+  return launch_status();
+}
+
+template <int D, typename Tin>
+tq_status launch_rotate_t(const RotateParams& p, const DeviceInfo& di, cudaStream_t st) {
+  using G = AppendGeom<D>;
+  const size_t smem = 4 * D + kAppendWarps * G::ROWS * (D * InType<Tin>::kBytes + 16);
+  auto kern = rotate_unit_kernel<D, Tin>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return TQ_ERR_CUDA;
+  const int64_t tiles = (p.rows + G::ROWS - 1) / G::ROWS;
+  const int64_t want = (tiles + kAppendWarps - 1) / kAppendWarps;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)di.num_sms * 4));
+  kern<<<grid, kAppendWarps * 32, smem, st>>>(p);
+  return launch_status();
+}
+
+#define TQ_DECLARE_APPEND(D_, NAME_, T_)                                                  \
+  tq_status launch_append_d##D_##_##NAME_(const AppendParams& p, const DeviceInfo& di,   \
+                                          cudaStream_t st);                              \
+  tq_status launch_rotate_d##D_##_##NAME_(const RotateParams& p, const DeviceInfo& di,   \
+                                          cudaStream_t st);
+#define TQ_DEFINE_APPEND(D_, NAME_, T_)                                                   \
+  tq_status launch_append_d##D_##_##NAME_(const AppendParams& p, const DeviceInfo& di,   \
+                                          cudaStream_t st) {                             \
+    return launch_append_t<D_, T_>(p, di, st);                                          \
+  }                                                                                      \
+  tq_status launch_rotate_d##D_##_##NAME_(const RotateParams& p, const DeviceInfo& di,   \
+                                          cudaStream_t st) {                             \
+    return launch_rotate_t<D_, T_>(p, di, st);                                          \
+  }
+
+#define TQ_FOR_EACH_APPEND(X) \
+  X(64, bf16, __nv_bfloat16)  \
+  X(64, f16, __half)          \
+  X(64, f32, float)           \
+  X(128, bf16, __nv_bfloat16) \
+  X(128, f16, __half)         \
+  X(128, f32, float)          \
+  X(256, bf16, __nv_bfloat16) \
+  X(256, f16, __half)         \
+  X(256, f32, float)
+
+TQ_FOR_EACH_APPEND(TQ_DECLARE_APPEND)
+
+}  // namespace tq

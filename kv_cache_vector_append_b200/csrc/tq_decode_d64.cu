@@ -1,0 +1,9 @@
+// Decode kernels for head_dim 64 (one translation unit per head dimension).
+#include "tq_launch.cuh"
+
+namespace tq {
+tq_status launch_decode_d64(int kb, int vb, const DecodeParams& p, const MergeParams& m,
+                             const DecodePlan& plan, cudaStream_t st) {
+  return launch_decode_dim<64>(kb, vb, p, m, plan, st);
+}
+}  // namespace tq

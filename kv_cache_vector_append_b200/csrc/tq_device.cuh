@@ -1,0 +1,85 @@
+// tq_device.cuh -- device helpers shared by the append and decode kernels:
+// the sign generator, cp.async staging, bounded waits and the error word.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include <type_traits>
+
+#include "tq.h"
+
+namespace tq {
+
+__host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// Compile-time loop: f(std::integral_constant<int, I>{}) for I = 0 .. N-1.
+template <int N, int I = 0, typename F>
+__device__ __forceinline__ void static_for(F&& f) {
+  if constexpr (I < N) {
+    f(std::integral_constant<int, I>{});
+    static_for<N, I + 1>(f);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Rotation signs.  tq-kv ("Library API") draws the Hadamard signs from a seeded
+// generator; the pages leave it open.  This library uses SplitMix64 (Steele,
+// Lea and Flood, 2014): output j of the generator seeded with `seed` is the
+// state seed + (j+1)*gamma passed through two xor-shift-multiply rounds, and the
+// sign of coordinate j is negative when bit 63 of that output is set.
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t j) {
+  uint64_t z = seed + (j + 1ull) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Sign-bit mask of coordinate j: 0x80000000 when s_j = -1, else 0.
+__device__ __forceinline__ uint32_t sign_mask_at(uint64_t seed, int j) {
+  return (uint32_t)(splitmix64_at(seed, (uint64_t)j) >> 63) << 31;
+}
+
+// ---------------------------------------------------------------------------
+// fp32 <-> storage types
+// ---------------------------------------------------------------------------
+template <typename T> struct InType;
+template <> struct InType<float> { static constexpr int kBytes = 4; };
+template <> struct InType<__nv_bfloat16> { static constexpr int kBytes = 2; };
+template <> struct InType<__half> { static constexpr int kBytes = 2; };
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
+
+// ---------------------------------------------------------------------------
+// Async global->shared copies (cp.async, Ampere-style, still the lightest way to
+// stage arbitrarily strided 16-byte pieces on sm_100a).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
+  uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(s), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
+  uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(s), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+
+__device__ __forceinline__ void report_error(unsigned int* err, unsigned int bits) {
+  if (err) atomicOr(err, bits);
+}
+
+__device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
+
+}  // namespace tq
