@@ -88,6 +88,7 @@ typedef enum {
 #define TQ_DEVERR_BLOCK_RANGE 0x2   /* block_table entry outside [0, num_blocks)   */
 #define TQ_DEVERR_NONFINITE 0x4     /* a K/V input row held a NaN or an infinity   */
 #define TQ_DEVERR_SEQLEN_RANGE 0x8  /* seq_len < 0 or > max_blocks*block_size      */
+#define TQ_DEVERR_TIMEOUT 0x10      /* a bounded wait inside a kernel gave up        */
 
 /* A strided view of a device array.  Strides are in ELEMENTS; shape[i] and
  * stride[i] for i >= ndim are ignored.  data must be aligned to the element size. */

@@ -92,40 +92,41 @@ int align_mode_of(const void* data, int esize, std::initializer_list<int64_t> st
   return 0;
 }
 
-size_t decode_smem_bytes(int dim, int kb, int vb, int h_q, int h_kv, int slot_stride, int wph,
-                         int nstage) {
-  auto lut_words = [](int b) { return b <= 4 ? (1 << (2 * b)) : (1 << b) / 2; };
-  size_t lut = ((size_t)(lut_words(kb) + lut_words(vb)) * 4 + 127) / 128 * 128;
-  size_t q = (size_t)h_q * dim * 4;
-  size_t stage = (size_t)kBlockSize * h_kv * slot_stride * wph;
-  return lut + q + 128 + nstage * stage;
-}
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+// Geometry of the decode kernels for one call (see tq_decode.cuh).
 tq_status plan_decode(int batch, int h_q, int h_kv, int dim, int kb, int vb, int slot_stride,
-                      int max_blocks, const DeviceInfo& di, DecodePlan* plan) {
+                      int max_blocks, bool shared_lut, const DeviceInfo& di, DecodePlan* plan) {
   if (h_kv < 1 || h_kv > kDecodeWarps) return TQ_ERR_UNSUPPORTED;
-  plan->wph = kDecodeWarps / h_kv;
-  plan->nstage = 4;
-  plan->smem = decode_smem_bytes(dim, kb, vb, h_q, h_kv, slot_stride, plan->wph, 4);
-  while ((int)plan->smem > di.max_smem_optin && plan->wph > 1) {
+  // whole page blocks are staged with one bulk copy each (unpadded rows): on B200 one
+  // 17 KB copy per block streams far better than one ~1 KB copy per row
+  plan->row_copies = 0;
+  plan->row_pitch = h_kv * slot_stride;
+  plan->shared_lut = shared_lut && kb == vb;
+  const size_t lut = decode_lut_bytes(kb, vb, plan->shared_lut);
+  // at most 4 blocks per step, so that one warp issues a step's row copies in two rounds
+  plan->wph = std::min(kDecodeWarps / h_kv, 4);
+  for (;;) {
+    plan->stage_bytes = plan->wph * kBlockSize * plan->row_pitch;
+    // block ids a CTA preloads: its whole step range when the grid is full
+    const int64_t steps_upper = (int64_t)batch * ((max_blocks + plan->wph - 1) / plan->wph);
+    const int64_t per_cta = (steps_upper + 2 * di.num_sms - 1) / (2 * di.num_sms) + 1;
+    plan->ids_cap = (int)std::min<int64_t>(per_cta * plan->wph, 4096);
+    plan->smem = lut + (size_t)kDecodeStages * plan->stage_bytes + kDecodeStages * 16 +
+                 4 * ((size_t)batch + 1) + 4 * ((1 << kb) + (1 << vb)) + 4 * plan->ids_cap + 16;
+    if ((int)plan->smem <= di.max_smem_optin || plan->wph == 1) break;
     plan->wph /= 2;
-    plan->smem = decode_smem_bytes(dim, kb, vb, h_q, h_kv, slot_stride, plan->wph, 4);
   }
-  if ((int)plan->smem > di.max_smem_optin) {
-    plan->nstage = 2;
-    plan->smem = decode_smem_bytes(dim, kb, vb, h_q, h_kv, slot_stride, plan->wph, 2);
-    if ((int)plan->smem > di.max_smem_optin) return TQ_ERR_UNSUPPORTED;
-  }
-  const int resident = std::max(1, std::min(4, (int)(228 * 1024 / (plan->smem + 1024))));
-  const int target = di.num_sms * resident * 2;
-  const int steps_max = std::max(1, (max_blocks + plan->wph - 1) / plan->wph);
-  int nsplit = std::max(1, std::min(steps_max, (target + batch - 1) / std::max(batch, 1)));
-  int spb = ((max_blocks + nsplit - 1) / nsplit + plan->wph - 1) / plan->wph * plan->wph;
-  spb = std::max(spb, plan->wph);
-  nsplit = std::max(1, (max_blocks + spb - 1) / spb);
-  plan->nsplit = nsplit;
-  plan->spb = spb;
-  plan->ws_bytes = (size_t)batch * nsplit * plan->wph * h_q * (dim + 2) * sizeof(float);
+  if ((int)plan->smem > di.max_smem_optin) return TQ_ERR_UNSUPPORTED;
+  plan->max_ctas = 2 * di.num_sms;
+  // workspace: rotated queries, their scales, step prefix sums, partial records
+  plan->qfrag_off = 0;
+  plan->qscale_off = align256((size_t)batch * h_q * dim * 2);
+  plan->prefix_off = plan->qscale_off + align256((size_t)batch * h_q * 4);
+  plan->part_off = plan->prefix_off + align256(((size_t)batch + 1) * 4);
+  plan->ws_bytes = plan->part_off + (size_t)(plan->max_ctas + batch) *
+                                        std::min(kDecodeWarps / h_kv, 4) * h_q * (dim + 2) *
+                                        sizeof(float);
   return TQ_OK;
 }
 
@@ -260,17 +261,13 @@ tq_status tq_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t n
   DeviceState* ds = nullptr;
   tq_status s = device_state(&ds);
   if (s != TQ_OK) return s;
-  // the worst case over supported bit widths: 8-bit K and V (largest slots)
+  // the record area is sized for the largest warps-per-head count, so any bit widths fit
   DecodePlan plan;
-  const int slot = region_bytes(head_dim, 8) * 2;
-  s = plan_decode(std::max(batch, 1), num_q_heads, num_kv_heads, head_dim, 8, 8, slot,
-                  std::max(max_blocks, 1), ds->info, &plan);
+  s = plan_decode(std::max(batch, 1), num_q_heads, num_kv_heads, head_dim, 1, 1,
+                  region_bytes(head_dim, 1) * 2 + 8, std::max(max_blocks, 1), false, ds->info,
+                  &plan);
   if (s != TQ_OK) return s;
-  // smaller slots can only give more stages of the same split plan, never a larger one
-  DecodePlan small;
-  plan_decode(std::max(batch, 1), num_q_heads, num_kv_heads, head_dim, 1, 1,
-              region_bytes(head_dim, 1) * 2, std::max(max_blocks, 1), ds->info, &small);
-  *bytes = std::max(plan.ws_bytes, small.ws_bytes);
+  *bytes = plan.ws_bytes;
   return TQ_OK;
 }
 
@@ -336,17 +333,20 @@ tq_status tq_paged_decode(tq_tensor out, tq_tensor q, tq_tensor pages, tq_tensor
   DeviceState* ds = nullptr;
   tq_status s = device_state(&ds);
   if (s != TQ_OK) return s;
-  const int max_blocks = std::max<int>(1, (int)block_table.shape[1]);
+  const int max_blocks = (int)block_table.shape[1];
+  const bool shared_lut = cb->k.bits == cb->v.bits && cb->k.centroids == cb->v.centroids;
   DecodePlan plan;
-  s = plan_decode(B, h_q, h_kv, D, kbits, vbits, (int)stride, max_blocks, ds->info, &plan);
+  s = plan_decode(B, h_q, h_kv, D, kbits, vbits, (int)stride, std::max(max_blocks, 1), shared_lut,
+                  ds->info, &plan);
   if (s != TQ_OK) return s;
+  if ((h_kv * stride) % 8) return TQ_ERR_INVALID_ARG;
 
-  float* ws = nullptr;
+  uint8_t* ws = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);
     if (ds->user_ws != nullptr) {
       if (ds->user_ws_bytes < plan.ws_bytes) return TQ_ERR_WORKSPACE;
-      ws = (float*)ds->user_ws;
+      ws = (uint8_t*)ds->user_ws;
     } else {
       if (ds->lib_ws_bytes < plan.ws_bytes) {
         if (ds->lib_ws) cudaFree(ds->lib_ws);
@@ -356,57 +356,67 @@ tq_status tq_paged_decode(tq_tensor out, tq_tensor q, tq_tensor pages, tq_tensor
         if (cudaMalloc(&ds->lib_ws, want) != cudaSuccess) return TQ_ERR_WORKSPACE;
         ds->lib_ws_bytes = want;
       }
-      ws = (float*)ds->lib_ws;
+      ws = (uint8_t*)ds->lib_ws;
     }
   }
+
+  QPrepParams qp{};
+  qp.q = q.data;
+  qp.q_bstride = q.stride[0];
+  qp.q_hstride = q.stride[1];
+  qp.q_dtype = q.dtype;
+  qp.h_q = h_q;
+  qp.scale_log2 = scale * 1.4426950408889634f;
+  qp.sign_seed = sign_seed;
+  qp.qfrag = (uint32_t*)(ws + plan.qfrag_off);
+  qp.qscale = (float*)(ws + plan.qscale_off);
 
   DecodeParams p{};
   p.pages = (const uint8_t*)pages.data;
   p.num_blocks = (int32_t)pages.shape[0];
   p.h_kv = h_kv;
   p.slot_stride = (int32_t)stride;
+  p.row_pitch = plan.row_pitch;
   p.blk_stride = pages.stride[0];
   p.block_table = (const int32_t*)block_table.data;
   p.bt_stride = block_table.stride[0];
-  p.max_blocks = (int32_t)block_table.shape[1];
+  p.max_blocks = max_blocks;
   p.seq_lens = (const int32_t*)seq_lens.data;
   p.batch = B;
-  p.q = q.data;
-  p.q_bstride = q.stride[0];
-  p.q_hstride = q.stride[1];
-  p.q_dtype = q.dtype;
   p.h_q = h_q;
   p.group = h_q / h_kv;
   p.kc = cb->k.centroids;
   p.vc = cb->v.centroids;
+  p.shared_lut = plan.shared_lut;
   p.k_region = kb;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.sign_seed = sign_seed;
   p.wph = plan.wph;
-  p.spb = plan.spb;
-  p.nsplit = plan.nsplit;
-  p.ws = ws;
+  p.stage_bytes = plan.stage_bytes;
+  p.ids_cap = plan.ids_cap;
+  p.row_copies = plan.row_copies;
+  p.qfrag = qp.qfrag;
+  p.qscale = qp.qscale;
+  p.prefix = (int32_t*)(ws + plan.prefix_off);
+  p.part = (float*)(ws + plan.part_off);
   p.err = ds->err;
 
   MergeParams m{};
-  m.ws = ws;
+  m.part = p.part;
+  m.prefix = p.prefix;
   m.out = out.data;
   m.o_bstride = out.stride[0];
   m.o_hstride = out.stride[1];
   m.out_dtype = out.dtype;
   m.h_q = h_q;
-  m.nsplit = plan.nsplit;
   m.wph = plan.wph;
-  m.spb = plan.spb;
-  m.max_blocks = p.max_blocks;
-  m.seq_lens = p.seq_lens;
   m.sign_seed = sign_seed;
 
+  const int64_t per_step = plan.wph;
+  const int64_t steps_upper = (int64_t)B * ((max_blocks + per_step - 1) / per_step);
   cudaStream_t st = as_stream(stream);
   switch (D) {
-    case 64: return launch_decode_d64(kbits, vbits, p, m, plan, st);
-    case 128: return launch_decode_d128(kbits, vbits, p, m, plan, st);
-    default: return launch_decode_d256(kbits, vbits, p, m, plan, st);
+    case 64: return launch_decode_d64(kbits, vbits, p, qp, m, plan, steps_upper, st);
+    case 128: return launch_decode_d128(kbits, vbits, p, qp, m, plan, steps_upper, st);
+    default: return launch_decode_d256(kbits, vbits, p, qp, m, plan, steps_upper, st);
   }
 }
 

@@ -6,13 +6,20 @@
 // (randomized Hadamard transform); turboquant_serve 0.1.2, "Architecture" (update():
 // rotate, normalize, Lloyd-Max encode, bit-pack, store uint8).
 //
-// Work layout.  A row is one (token, KV head) vector of K or of V.  A warp owns a
-// tile of 32 rows of one kind (K or V); for D <= 128 each lane holds a whole row in
-// registers (no shuffles in the transform), for D = 256 two lanes share a row
-// (one cross-lane butterfly stage).  Input tiles are staged in shared memory with
-// cp.async (double-buffered per warp) so that global reads are fully coalesced;
-// packed regions are staged in shared memory and written back one contiguous
-// region per store instruction.
+// Work layout.  A row is one (token, KV head) vector of K or of V.  Every lane holds
+// 64 consecutive coordinates of a row in registers (D/64 lanes per row), so the FWHT
+// is six register stages plus log2(D/64) shuffle stages.  A warp owns a tile of
+// 32*64/D rows of one kind (K or V); lane l serves row l % ROWS, part l / ROWS, so
+// that each 8-lane phase of a 16-byte shared load touches 8 different rows (padded
+// pitch, no bank conflicts).  Input tiles are staged in shared memory by cp.async
+// (double-buffered per warp); packed regions are staged in shared memory and
+// written back one contiguous region per store instruction.
+//
+// Encode.  idx = #{i : b_i < u} over the fp32 boundaries.  For bits <= 4 (and when no
+// two boundaries share a bucket) the top 12 bits of u's float encoding (sign,
+// exponent, 3 mantissa bits) index a byte table k0 = #{b_i < lowest float of the
+// bucket}; one compare against b[k0] then gives idx exactly.  Otherwise a
+// branch-free binary search over the boundaries in Eytzinger order.
 #pragma once
 
 #include "tq_device.cuh"
@@ -53,81 +60,116 @@ struct RotateParams {      // test export of the rotation (tq_rotate_unit)
   int32_t align_mode;
 };
 
-constexpr int kAppendWarps = 4;
+constexpr int kAppendWarps = 8;
+constexpr int kBucketShift = 20;                 // 12-bit buckets: sign, exponent, 3 bits
+constexpr int kBuckets = 1 << (32 - kBucketShift);
 
 template <int D>
 struct AppendGeom {
-  static constexpr int TPR = D > 128 ? D / 128 : 1;   // lanes per row
-  static constexpr int E = D / TPR;                   // elements per lane
+  static constexpr int E = 64;                        // elements per lane
+  static constexpr int TPR = D / E;                   // lanes per row
   static constexpr int ROWS = 32 / TPR;               // rows per warp tile
   static constexpr int MAXW = D * 8 / 32 + 1;         // packed words + norm, 8-bit
   static constexpr int OUTPITCH = MAXW | 1;           // odd pitch: conflict-free
 };
 
-// Builds the Eytzinger (breadth-first) image of the sorted boundary array so
-// that a binary search walks i -> 2i + (u > t[i]).  t[0] is unused.
-__device__ __forceinline__ void build_eytzinger(float* t, const float* b, int bits, int tid,
-                                                int nthreads) {
+// Shared tables of one kind (K or V).
+struct alignas(16) EncodeTables {
+  uint8_t k0[kBuckets];     // #{b_i < lowest float of the bucket}
+  float bnd[257];           // boundaries b_0..b_{L-2}, then +inf
+  float eytz[256];          // Eytzinger image (t[0] unused)
+  int fast;                 // bucket encode valid for this table
+};
+
+__device__ __forceinline__ void build_tables(EncodeTables* t, const float* b, int bits, int tid,
+                                             int nthreads) {
   const int n = (1 << bits) - 1;
+  for (int i = tid; i <= n; i += nthreads) t->bnd[i] = i < n ? b[i] : INFINITY;
   for (int i = 1 + tid; i <= n; i += nthreads) {
-    int d = 31 - __clz(i);
-    int k = i - (1 << d);
-    int src = ((2 * k + 1) << (bits - 1 - d)) - 1;
-    t[i] = b[src];
+    const int d = 31 - __clz(i);
+    const int k = i - (1 << d);
+    t->eytz[i] = b[((2 * k + 1) << (bits - 1 - d)) - 1];
+  }
+  if (tid == 0) {
+    int ok = bits <= 4;
+    for (int i = 0; i + 1 < n; ++i)
+      if ((__float_as_uint(b[i]) >> kBucketShift) == (__float_as_uint(b[i + 1]) >> kBucketShift))
+        ok = 0;
+    t->fast = ok;
+  }
+  // k0 of each bucket: the lowest float of bucket g is g << 20 for a positive bucket
+  // and -((g & 0x7ff) << 20 | 0xfffff) for a negative one.  (Only used for bits <= 4.)
+  if (bits > 4) return;
+  for (int g = tid; g < kBuckets; g += nthreads) {
+    const uint32_t lowbits = (g & 0x800) ? ((uint32_t)g << kBucketShift) | 0xFFFFFu
+                                         : (uint32_t)g << kBucketShift;
+    const float lo = __uint_as_float(lowbits);
+    int c = 0;
+    for (int i = 0; i < n; ++i) c += (b[i] < lo) ? 1 : 0;
+    t->k0[g] = (uint8_t)c;
   }
 }
 
-// Stage `nrows` rows of `rowbytes` bytes into shared memory (pitch `pitch`).
-// Row r starts at row_ptr(r).  Issued by one warp.
-template <int D, typename Tin, typename RowPtr>
+// Stage `nrows` rows of RB bytes into shared memory (pitch `pitch`); row r starts at
+// row_ptr(r).  Issued by one warp.
+template <int RB, typename RowPtr>
 __device__ __forceinline__ void stage_rows(uint8_t* dst, int pitch, int nrows, RowPtr row_ptr,
                                            int align_mode, int lane) {
-  constexpr int RB = D * InType<Tin>::kBytes;
   if (align_mode == 16) {
     constexpr int NC = RB / 16;
     for (int f = lane; f < nrows * NC; f += 32) {
-      int r = f / NC, c = f % NC;
+      const int r = f / NC, c = f % NC;
       cp_async16(dst + r * pitch + c * 16, (const uint8_t*)row_ptr(r) + c * 16);
     }
   } else if (align_mode == 4) {
     constexpr int NC = RB / 4;
     for (int f = lane; f < nrows * NC; f += 32) {
-      int r = f / NC, c = f % NC;
+      const int r = f / NC, c = f % NC;
       cp_async4(dst + r * pitch + c * 4, (const uint8_t*)row_ptr(r) + c * 4);
     }
   } else {
     constexpr int NC = RB / 2;
     for (int f = lane; f < nrows * NC; f += 32) {
-      int r = f / NC, c = f % NC;
+      const int r = f / NC, c = f % NC;
       *(uint16_t*)(dst + r * pitch + c * 2) = *((const uint16_t*)row_ptr(r) + c);
     }
   }
 }
 
-// Load this lane's E elements of its row from shared memory as fp32.
-template <int E, typename Tin>
-__device__ __forceinline__ void load_row(float (&x)[E], const uint8_t* p) {
+// Load this lane's 64 input elements from shared memory as fp32 with the rotation
+// signs applied (the sign flip is an xor of the sign bit; for bf16 it rides along
+// with the widening: bits << 16 plus the mask, or the high half masked and xor-ed).
+template <typename Tin>
+__device__ __forceinline__ void load_signed(float (&x)[64], const uint8_t* p,
+                                            const uint32_t* m) {
   if constexpr (sizeof(Tin) == 4) {
 #pragma unroll
-    for (int c = 0; c < E / 4; ++c) {
-      float4 q = *(const float4*)(p + 16 * c);
-      x[4 * c + 0] = q.x; x[4 * c + 1] = q.y; x[4 * c + 2] = q.z; x[4 * c + 3] = q.w;
+    for (int c = 0; c < 16; ++c) {
+      const uint4 q = *(const uint4*)(p + 16 * c);
+      const uint4 s = *(const uint4*)(m + 4 * c);
+      x[4 * c + 0] = __uint_as_float(q.x ^ s.x);
+      x[4 * c + 1] = __uint_as_float(q.y ^ s.y);
+      x[4 * c + 2] = __uint_as_float(q.z ^ s.z);
+      x[4 * c + 3] = __uint_as_float(q.w ^ s.w);
     }
   } else {
 #pragma unroll
-    for (int c = 0; c < E / 8; ++c) {
-      uint4 q = *(const uint4*)(p + 16 * c);
-      uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    for (int c = 0; c < 8; ++c) {
+      const uint4 q = *(const uint4*)(p + 16 * c);
+      const uint4 s0 = *(const uint4*)(m + 8 * c);
+      const uint4 s1 = *(const uint4*)(m + 8 * c + 4);
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+      const uint32_t s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
-          x[8 * c + 2 * k + 0] = __uint_as_float(w[k] << 16);
-          x[8 * c + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+          x[8 * c + 2 * k + 0] = __uint_as_float((w[k] << 16) ^ s[2 * k]);
+          x[8 * c + 2 * k + 1] = __uint_as_float((w[k] & 0xFFFF0000u) ^ s[2 * k + 1]);
         } else {
-          __half2 h = *reinterpret_cast<__half2*>(&w[k]);
-          float2 f = __half22float2(h);
-          x[8 * c + 2 * k + 0] = f.x;
-          x[8 * c + 2 * k + 1] = f.y;
+          __half2 h = *reinterpret_cast<const __half2*>(&w[k]);
+          const float2 f = __half22float2(h);
+          x[8 * c + 2 * k + 0] = __uint_as_float(__float_as_uint(f.x) ^ s[2 * k]);
+          x[8 * c + 2 * k + 1] = __uint_as_float(__float_as_uint(f.y) ^ s[2 * k + 1]);
         }
       }
     }
@@ -135,48 +177,41 @@ __device__ __forceinline__ void load_row(float (&x)[E], const uint8_t* p) {
 }
 
 // The rotation shared by quantize-append and its test export.  On entry x holds
-// this lane's E input elements (coordinates half*E .. half*E+E-1 of the row); on
-// exit x holds the unnormalised transform H (s * x) of those coordinates, and the
-// function returns the scale r with u = x * r; *norm_out = ||x||_2 (fp32).
+// this lane's 64 sign-flipped input elements (coordinates 64*part .. 64*part+63 of
+// the row); on exit x holds the unnormalised transform H (s * x) of those
+// coordinates, and the function returns r with u = x * r; *norm_out = ||x||_2.
 // Order of operations (fixed, so the export reproduces the kernel exactly):
-//   ss = sum of x_j^2 by fused multiply-add in coordinate order (lane pairs then
-//   add their halves), n = sqrt(ss) (IEEE), sign flips, FWHT butterflies in
-//   stages h = 1, 2, 4, ..., D/2, r = 1 / (n * sqrt(D)) (IEEE reciprocal), or 0
-//   when n == 0.
+//   ss = sum of x_j^2 by fused multiply-add in coordinate order within a lane, then
+//   the lanes of a row add their sums pairwise (xor butterfly over the part bits);
+//   n = sqrt(ss) (IEEE); FWHT butterflies in stages h = 1, 2, 4, ..., D/2;
+//   r = 1 / (n * sqrt(D)) (IEEE reciprocal), or 0 when n == 0.
 template <int D>
-__device__ __forceinline__ float rotate_row(float (&x)[AppendGeom<D>::E], const uint32_t* smask,
-                                            int half, float* norm_out) {
-  constexpr int E = AppendGeom<D>::E;
-  constexpr int TPR = AppendGeom<D>::TPR;
+__device__ __forceinline__ float rotate_row(float (&x)[64], int part, float* norm_out) {
+  using G = AppendGeom<D>;
   float ss = 0.f;
 #pragma unroll
-  for (int j = 0; j < E; ++j) ss = __fmaf_rn(x[j], x[j], ss);
-  if constexpr (TPR == 2) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, 1));
+  for (int j = 0; j < 64; ++j) ss = __fmaf_rn(x[j], x[j], ss);
+#pragma unroll
+  for (int m = 1; m < G::TPR; m <<= 1)
+    ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, G::ROWS * m));
   const float n = sqrtf(ss);
 #pragma unroll
-  for (int c = 0; c < E / 4; ++c) {
-    uint4 m = *(const uint4*)(smask + half * E + 4 * c);
-    x[4 * c + 0] = __uint_as_float(__float_as_uint(x[4 * c + 0]) ^ m.x);
-    x[4 * c + 1] = __uint_as_float(__float_as_uint(x[4 * c + 1]) ^ m.y);
-    x[4 * c + 2] = __uint_as_float(__float_as_uint(x[4 * c + 2]) ^ m.z);
-    x[4 * c + 3] = __uint_as_float(__float_as_uint(x[4 * c + 3]) ^ m.w);
-  }
+  for (int h = 1; h < 64; h <<= 1) {
 #pragma unroll
-  for (int h = 1; h < E; h <<= 1) {
-#pragma unroll
-    for (int i = 0; i < E; ++i) {
+    for (int i = 0; i < 64; ++i) {
       if ((i & h) == 0) {
-        float a = x[i], b = x[i + h];
+        const float a = x[i], b = x[i + h];
         x[i] = __fadd_rn(a, b);
         x[i + h] = __fsub_rn(a, b);
       }
     }
   }
-  if constexpr (TPR == 2) {
 #pragma unroll
-    for (int i = 0; i < E; ++i) {
-      float o = __shfl_xor_sync(0xffffffffu, x[i], 1);
-      x[i] = half == 0 ? __fadd_rn(x[i], o) : __fsub_rn(o, x[i]);
+  for (int m = 1; m < G::TPR; m <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, x[i], G::ROWS * m);
+      x[i] = (part & m) ? __fsub_rn(o, x[i]) : __fadd_rn(x[i], o);
     }
   }
   *norm_out = n;
@@ -184,24 +219,27 @@ __device__ __forceinline__ float rotate_row(float (&x)[AppendGeom<D>::E], const 
   return n > 0.f ? __frcp_rn(__fmul_rn(n, sqrt_d)) : 0.f;
 }
 
-// Encode u = x[j] * r with the Eytzinger table and pack the codes LSB-first into
-// `words` (E*BITS/32 words: this lane's share of the bit stream).
-template <int E, int BITS>
-__device__ __forceinline__ void encode_pack(const float (&x)[E], float r, const float* tab,
+// Encode u = x[j] * r and pack the 64 codes LSB-first into 2*BITS words.
+template <int BITS, bool FAST>
+__device__ __forceinline__ void encode_pack(const float (&x)[64], float r, const EncodeTables* t,
                                             uint32_t* words) {
-  constexpr int W = E * BITS / 32;
+  constexpr int W = 64 * BITS / 32;
   uint32_t acc[W];
 #pragma unroll
   for (int w = 0; w < W; ++w) acc[w] = 0u;
 #pragma unroll
-  for (int j = 0; j < E; ++j) {
+  for (int j = 0; j < 64; ++j) {
     const float u = __fmul_rn(x[j], r);
-    int i = 1;
+    uint32_t code;
+    if constexpr (FAST) {
+      const uint32_t k0 = t->k0[__float_as_uint(u) >> kBucketShift];
+      code = k0 + (u > t->bnd[k0] ? 1u : 0u);
+    } else {
+      int i = 1;
 #pragma unroll
-    for (int s = 0; s < BITS; ++s) i = 2 * i + (u > tab[i] ? 1 : 0);
-    const uint32_t code = (uint32_t)(i - (1 << BITS));
-    constexpr int dummy = 0;
-    (void)dummy;
+      for (int s = 0; s < BITS; ++s) i = 2 * i + (u > t->eytz[i] ? 1 : 0);
+      code = (uint32_t)(i - (1 << BITS));
+    }
     const int bit = j * BITS;
     const int w0 = bit >> 5, o0 = bit & 31;
     acc[w0] |= code << o0;
@@ -211,26 +249,40 @@ __device__ __forceinline__ void encode_pack(const float (&x)[E], float r, const 
   for (int w = 0; w < W; ++w) words[w] = acc[w];
 }
 
+template <int BITS>
+__device__ __forceinline__ void encode_pack_any(const float (&x)[64], float r,
+                                                const EncodeTables* t, uint32_t* words) {
+  if constexpr (BITS <= 4) {
+    if (t->fast) {
+      encode_pack<BITS, true>(x, r, t, words);
+      return;
+    }
+  }
+  encode_pack<BITS, false>(x, r, t, words);
+}
+
 template <int D, typename Tin>
-__global__ void __launch_bounds__(kAppendWarps * 32)
+struct AppendSmem {
+  using G = AppendGeom<D>;
+  static constexpr int RB = D * InType<Tin>::kBytes;
+  static constexpr int INPITCH = RB + 16;
+  static constexpr int PER_WARP = 2 * G::ROWS * INPITCH + G::ROWS * G::OUTPITCH * 4 + G::ROWS * 8;
+  static constexpr int TABLES = ((2 * (int)sizeof(EncodeTables) + 4 * D) + 127) / 128 * 128;
+  static constexpr int BYTES = TABLES + kAppendWarps * PER_WARP;
+};
+
+template <int D, typename Tin>
+__global__ void __launch_bounds__(kAppendWarps * 32, 2)
 append_kernel(AppendParams p) {
   using G = AppendGeom<D>;
-  constexpr int RB = D * InType<Tin>::kBytes;
-  constexpr int INPITCH = RB + 16;
+  using SM = AppendSmem<D, Tin>;
   extern __shared__ __align__(16) uint8_t smem[];
-  float* tab = (float*)smem;                           // 2 x 256 floats (Eytzinger, K and V)
-  uint32_t* smask = (uint32_t*)(smem + 2048);          // D sign masks
-  uint8_t* wbase = smem + 2048 + 4 * D;
+  EncodeTables* tabs = (EncodeTables*)smem;                       // [2]: K, V
+  uint32_t* smask = (uint32_t*)(smem + 2 * sizeof(EncodeTables));  // D sign masks
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int PER_WARP = 2 * G::ROWS * INPITCH + G::ROWS * G::OUTPITCH * 4 + G::ROWS * 8;
-  uint8_t* in_s = wbase + warp * PER_WARP;
-  uint32_t* out_s = (uint32_t*)(in_s + 2 * G::ROWS * INPITCH);
+  uint8_t* in_s = smem + SM::TABLES + warp * SM::PER_WARP;
+  uint32_t* out_s = (uint32_t*)(in_s + 2 * G::ROWS * SM::INPITCH);
   int64_t* dst_s = (int64_t*)(out_s + G::ROWS * G::OUTPITCH);
-
-  build_eytzinger(tab, p.boundaries[0], p.bits[0], threadIdx.x, blockDim.x);
-  build_eytzinger(tab + 256, p.boundaries[1], p.bits[1], threadIdx.x, blockDim.x);
-  for (int j = threadIdx.x; j < D; j += blockDim.x) smask[j] = sign_mask_at(p.sign_seed, j);
-  __syncthreads();
 
   const int64_t rows_per_kind = p.num_tokens * p.h_kv;
   const int64_t tiles_per_kind = (rows_per_kind + G::ROWS - 1) / G::ROWS;
@@ -245,19 +297,26 @@ append_kernel(AppendParams p) {
     const Tin* base = (const Tin*)p.src[kind];
     const int64_t ts = p.tok_stride[kind], hs = p.head_stride_in[kind];
     const int hk = p.h_kv;
-    stage_rows<D, Tin>(in_s + buf * G::ROWS * INPITCH, INPITCH, nr,
+    stage_rows<SM::RB>(in_s + buf * G::ROWS * SM::INPITCH, SM::INPITCH, nr,
                        [&](int r) {
-                         int64_t row = r0 + r;
-                         int64_t t = row / hk;
-                         int h = (int)(row - t * hk);
+                         const int64_t row = r0 + r;
+                         const int64_t t = row / hk;
+                         const int h = (int)(row - t * hk);
                          return (const void*)(base + t * ts + h * hs);
                        },
                        p.align_mode, lane);
   };
-
-  int buf = 0;
+  // the first tile's rows are in flight while the tables are built
   if (gwarp < ntiles) issue(gwarp, 0);
   cp_async_commit();
+  build_tables(&tabs[0], p.boundaries[0], p.bits[0], threadIdx.x, blockDim.x);
+  build_tables(&tabs[1], p.boundaries[1], p.bits[1], threadIdx.x, blockDim.x);
+  for (int j = threadIdx.x; j < D; j += blockDim.x) smask[j] = sign_mask_at(p.sign_seed, j);
+  __syncthreads();
+
+  const int rl = lane % G::ROWS;           // row within the tile
+  const int part = lane / G::ROWS;         // which 64 coordinates of the row
+  int buf = 0;
   for (int64_t tile = gwarp; tile < ntiles; tile += nwarps) {
     const int64_t next = tile + nwarps;
     if (next < ntiles) issue(next, buf ^ 1);
@@ -287,33 +346,32 @@ append_kernel(AppendParams p) {
     cp_async_wait<1>();
     __syncwarp();
     {
-      const int rl = lane / G::TPR;          // row within the tile
-      const int half = lane % G::TPR;
-      float x[G::E];
-      load_row<G::E, Tin>(x, in_s + buf * G::ROWS * INPITCH + rl * INPITCH + half * G::E *
-                                  InType<Tin>::kBytes);
+      float x[64];
+      load_signed<Tin>(x, in_s + buf * G::ROWS * SM::INPITCH + rl * SM::INPITCH +
+                              part * 64 * InType<Tin>::kBytes,
+                       smask + part * 64);
       float n;
-      const float r = rotate_row<D>(x, smask, half, &n);
+      const float r = rotate_row<D>(x, part, &n);
       const bool bad = !(fabsf(n) <= 3.402823466e38f);   // inf or NaN
       uint32_t* orow = out_s + rl * G::OUTPITCH;
-      const float* t = tab + 256 * kind;
+      const EncodeTables* t = &tabs[kind];
       const int wpl = (nw - 1) / G::TPR;                  // words per lane
-      uint32_t* mine = orow + half * wpl;
+      uint32_t* mine = orow + part * wpl;
       switch (bits) {
-        case 1: encode_pack<G::E, 1>(x, r, t, mine); break;
-        case 2: encode_pack<G::E, 2>(x, r, t, mine); break;
-        case 3: encode_pack<G::E, 3>(x, r, t, mine); break;
-        case 4: encode_pack<G::E, 4>(x, r, t, mine); break;
-        case 5: encode_pack<G::E, 5>(x, r, t, mine); break;
-        case 6: encode_pack<G::E, 6>(x, r, t, mine); break;
-        case 7: encode_pack<G::E, 7>(x, r, t, mine); break;
-        default: encode_pack<G::E, 8>(x, r, t, mine); break;
+        case 1: encode_pack_any<1>(x, r, t, mine); break;
+        case 2: encode_pack_any<2>(x, r, t, mine); break;
+        case 3: encode_pack_any<3>(x, r, t, mine); break;
+        case 4: encode_pack_any<4>(x, r, t, mine); break;
+        case 5: encode_pack_any<5>(x, r, t, mine); break;
+        case 6: encode_pack_any<6>(x, r, t, mine); break;
+        case 7: encode_pack_any<7>(x, r, t, mine); break;
+        default: encode_pack_any<8>(x, r, t, mine); break;
       }
       if (bad) {
         for (int w = 0; w < wpl; ++w) mine[w] = 0u;
-        if (half == 0 && rl < nr) report_error(p.err, TQ_DEVERR_NONFINITE);
+        if (part == 0 && rl < nr) report_error(p.err, TQ_DEVERR_NONFINITE);
       }
-      if (half == G::TPR - 1) orow[nw - 1] = bad ? 0x7FC00000u : __float_as_uint(n);
+      if (part == G::TPR - 1) orow[nw - 1] = bad ? 0x7FC00000u : __float_as_uint(n);
     }
     __syncwarp();
     // write back: one row region per pass (contiguous words)
@@ -330,14 +388,6 @@ append_kernel(AppendParams p) {
   cp_async_wait<0>();
 }
 
-template <int D>
-constexpr size_t append_smem_bytes(int in_bytes) {
-  using G = AppendGeom<D>;
-  return 2048 + 4 * D +
-         (size_t)kAppendWarps * (2 * G::ROWS * (D * in_bytes + 16) + G::ROWS * G::OUTPITCH * 4 +
-                                 G::ROWS * 8);
-}
-
 // Test export: the rotation of tq_quantize_append, written out as fp32 u and n.
 template <int D, typename Tin>
 __global__ void __launch_bounds__(kAppendWarps * 32)
@@ -351,28 +401,28 @@ rotate_unit_kernel(RotateParams p) {
   uint8_t* in_s = smem + 4 * D + warp * G::ROWS * INPITCH;
   for (int j = threadIdx.x; j < D; j += blockDim.x) smask[j] = sign_mask_at(p.sign_seed, j);
   __syncthreads();
+  const int rl = lane % G::ROWS, part = lane / G::ROWS;
   const int64_t ntiles = (p.rows + G::ROWS - 1) / G::ROWS;
   for (int64_t tile = (int64_t)blockIdx.x * kAppendWarps + warp; tile < ntiles;
        tile += (int64_t)gridDim.x * kAppendWarps) {
     const int64_t r0 = tile * G::ROWS;
     const int nr = (int)imin64((int64_t)G::ROWS, p.rows - r0);
     const Tin* base = (const Tin*)p.x;
-    stage_rows<D, Tin>(in_s, INPITCH, nr,
-                       [&](int r) { return (const void*)(base + (r0 + r) * p.x_row_stride); },
-                       p.align_mode, lane);
+    stage_rows<RB>(in_s, INPITCH, nr,
+                   [&](int r) { return (const void*)(base + (r0 + r) * p.x_row_stride); },
+                   p.align_mode, lane);
     cp_async_commit();
     cp_async_wait<0>();
     __syncwarp();
-    const int rl = lane / G::TPR, half = lane % G::TPR;
-    float x[G::E];
-    load_row<G::E, Tin>(x, in_s + rl * INPITCH + half * G::E * InType<Tin>::kBytes);
+    float x[64];
+    load_signed<Tin>(x, in_s + rl * INPITCH + part * 64 * InType<Tin>::kBytes, smask + part * 64);
     float n;
-    const float r = rotate_row<D>(x, smask, half, &n);
+    const float r = rotate_row<D>(x, part, &n);
     if (rl < nr) {
-      float* u = p.u + (r0 + rl) * p.u_row_stride + half * G::E;
+      float* u = p.u + (r0 + rl) * p.u_row_stride + part * 64;
 #pragma unroll
-      for (int j = 0; j < G::E; ++j) u[j] = __fmul_rn(x[j], r);
-      if (half == 0) p.norm[(r0 + rl) * p.norm_stride] = n;
+      for (int j = 0; j < 64; ++j) u[j] = __fmul_rn(x[j], r);
+      if (part == 0) p.norm[(r0 + rl) * p.norm_stride] = n;
     }
     __syncwarp();
   }

@@ -8,7 +8,7 @@ namespace tq {
 
 template <int D, typename Tin>
 tq_status launch_append_t(const AppendParams& p, const DeviceInfo& di, cudaStream_t st) {
-  const size_t smem = append_smem_bytes<D>(InType<Tin>::kBytes);
+  const size_t smem = AppendSmem<D, Tin>::BYTES;
   if ((int)smem > di.max_smem_optin) return TQ_ERR_UNSUPPORTED;
   auto kern = append_kernel<D, Tin>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=

@@ -18,11 +18,15 @@ struct DeviceInfo {
 };
 
 struct DecodePlan {
-  int wph = 1;        // warps (sub-streams) per KV head
-  int nsplit = 1;     // splits per sequence
-  int spb = 1;        // blocks per split
-  int nstage = 4;     // pipeline depth
-  size_t smem = 0;    // dynamic shared memory of the decode kernel
+  int wph = 1;            // warps (sub-streams) per KV head
+  int row_pitch = 0;      // padded shared-memory row pitch (bytes)
+  int stage_bytes = 0;    // one pipeline stage: wph blocks
+  int ids_cap = 0;        // block ids a CTA preloads into shared memory
+  int row_copies = 0;     // one bulk copy per page row (padded pitch) or per block
+  int shared_lut = 0;     // K and V share one lookup table
+  size_t smem = 0;        // dynamic shared memory of the decode kernel
+  int max_ctas = 0;       // upper bound of the persistent grid
+  size_t qfrag_off = 0, qscale_off = 0, prefix_off = 0, part_off = 0;
   size_t ws_bytes = 0;
 };
 
@@ -34,12 +38,15 @@ tq_status launch_append_any(int dim, int dtype, const AppendParams& p, const Dev
                             cudaStream_t st);
 tq_status launch_rotate_any(int dim, int dtype, const RotateParams& p, const DeviceInfo& di,
                             cudaStream_t st);
-tq_status launch_decode_d64(int kb, int vb, const DecodeParams& p, const MergeParams& m,
-                            const DecodePlan& plan, cudaStream_t st);
-tq_status launch_decode_d128(int kb, int vb, const DecodeParams& p, const MergeParams& m,
-                             const DecodePlan& plan, cudaStream_t st);
-tq_status launch_decode_d256(int kb, int vb, const DecodeParams& p, const MergeParams& m,
-                             const DecodePlan& plan, cudaStream_t st);
+tq_status launch_decode_d64(int kb, int vb, const DecodeParams& p, const QPrepParams& qp,
+                            const MergeParams& m, const DecodePlan& plan, int64_t steps_upper,
+                            cudaStream_t st);
+tq_status launch_decode_d128(int kb, int vb, const DecodeParams& p, const QPrepParams& qp,
+                             const MergeParams& m, const DecodePlan& plan, int64_t steps_upper,
+                             cudaStream_t st);
+tq_status launch_decode_d256(int kb, int vb, const DecodeParams& p, const QPrepParams& qp,
+                             const MergeParams& m, const DecodePlan& plan, int64_t steps_upper,
+                             cudaStream_t st);
 
 // (K bits, V bits) pairs with a compiled decode kernel.
 inline bool decode_bits_supported(int kb, int vb) {
@@ -49,37 +56,51 @@ inline bool decode_bits_supported(int kb, int vb) {
   return false;
 }
 
-template <int D, int KB, int VB, int NH, int NS>
-tq_status launch_decode_t(const DecodeParams& p, const MergeParams& m, const DecodePlan& plan,
-                          cudaStream_t st) {
-  auto kern = decode_kernel<D, KB, VB, NH, NS>;
+template <int D, int KB, int VB, int NH>
+tq_status launch_decode_t(DecodeParams p, QPrepParams qp, MergeParams m, const DecodePlan& plan,
+                          int64_t steps_upper, cudaStream_t st) {
+  auto kern = decode_kernel<D, KB, VB, NH>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem) !=
       cudaSuccess)
     return TQ_ERR_CUDA;
-  dim3 grid(plan.nsplit, p.batch);
-  kern<<<grid, p.h_kv * plan.wph * 32, plan.smem, st>>>(p);
+  const int threads = p.h_kv * plan.wph * 32;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, plan.smem) !=
+      cudaSuccess)
+    return TQ_ERR_CUDA;
+  per_sm = std::max(1, std::min(per_sm, 2));
+  int num_sms = plan.max_ctas / 2;
+  // persistent grid, but at least two steps per CTA so that tiny batches do not pay
+  // one prologue per step
+  const int64_t ctas = std::max<int64_t>(
+      1, std::min<int64_t>(std::min<int64_t>((int64_t)num_sms * per_sm, plan.max_ctas),
+                           (steps_upper + 1) / 2));
+  m.nctas = (int32_t)ctas;
+  const int qrows = p.batch * p.h_q;
+  qprep_kernel<D, KB><<<(qrows + 7) / 8, 256, 0, st>>>(qp, qrows);
   tq_status s = launch_status();
   if (s != TQ_OK) return s;
-  merge_kernel<D><<<dim3(p.h_q, p.batch), D, 0, st>>>(m);
+  kern<<<(unsigned)ctas, threads, plan.smem, st>>>(p);
+  s = launch_status();
+  if (s != TQ_OK) return s;
+  merge_kernel<D><<<dim3(p.h_q, p.batch), 256, 0, st>>>(m);
   return launch_status();
 }
 
 template <int D, int KB, int VB>
-tq_status launch_decode_bits(const DecodeParams& p, const MergeParams& m, const DecodePlan& plan,
-                             cudaStream_t st) {
-  const bool nh2 = p.group > 8;
-  if (plan.nstage == 4)
-    return nh2 ? launch_decode_t<D, KB, VB, 2, 4>(p, m, plan, st)
-               : launch_decode_t<D, KB, VB, 1, 4>(p, m, plan, st);
-  return nh2 ? launch_decode_t<D, KB, VB, 2, 2>(p, m, plan, st)
-             : launch_decode_t<D, KB, VB, 1, 2>(p, m, plan, st);
+tq_status launch_decode_bits(const DecodeParams& p, const QPrepParams& qp, const MergeParams& m,
+                             const DecodePlan& plan, int64_t steps_upper, cudaStream_t st) {
+  return p.group > 8 ? launch_decode_t<D, KB, VB, 2>(p, qp, m, plan, steps_upper, st)
+                     : launch_decode_t<D, KB, VB, 1>(p, qp, m, plan, steps_upper, st);
 }
 
 template <int D>
-tq_status launch_decode_dim(int kb, int vb, const DecodeParams& p, const MergeParams& m,
-                            const DecodePlan& plan, cudaStream_t st) {
+tq_status launch_decode_dim(int kb, int vb, const DecodeParams& p, const QPrepParams& qp,
+                            const MergeParams& m, const DecodePlan& plan, int64_t steps_upper,
+                            cudaStream_t st) {
 #define TQ_BITS_CASE(KB_, VB_) \
-  if (kb == KB_ && vb == VB_) return launch_decode_bits<D, KB_, VB_>(p, m, plan, st);
+  if (kb == KB_ && vb == VB_)  \
+    return launch_decode_bits<D, KB_, VB_>(p, qp, m, plan, steps_upper, st);
   TQ_BITS_CASE(2, 2)
   TQ_BITS_CASE(3, 3)
   TQ_BITS_CASE(4, 4)
@@ -90,6 +111,12 @@ tq_status launch_decode_dim(int kb, int vb, const DecodeParams& p, const MergePa
   TQ_BITS_CASE(4, 3)
 #undef TQ_BITS_CASE
   return TQ_ERR_UNSUPPORTED;
+}
+
+// Bytes of the replicated lookup table(s) of the decode kernel.
+inline size_t decode_lut_bytes(int kb, int vb, bool shared) {
+  auto one = [](int b) { return (size_t)(b <= 4 ? (1 << (2 * b)) : (1 << b)) * 32 * 4; };
+  return shared ? one(kb) : one(kb) + one(vb);
 }
 
 }  // namespace tq
