@@ -169,6 +169,33 @@ TQ_API tq_status tq_paged_decode(tq_tensor out, tq_tensor q, tq_tensor pages,
                           const tq_codebooks* cb, uint64_t sign_seed, float scale,
                           void* stream);
 
+/* Allocation-free variant of tq_paged_decode (this library's own addition; the
+ * pages describe no counterpart).  Same arguments, semantics and results as
+ * tq_paged_decode, but its scratch is a fixed device array inside the library
+ * (TQ_NOALLOC_SCRATCH_BYTES bytes, held by every device that loads the library
+ * until the process exits) instead of a workspace the caller sets or the library
+ * allocates.  It is meant for callers that must not allocate device memory on
+ * the call path: a serving loop that keeps every allocation out of its steady
+ * state (cudaMalloc/cudaFree can synchronise the device and fragment a pooled
+ * allocator), or an embedding runtime that owns all device memory and forbids
+ * libraries from allocating behind its back.  It calls no cudaMalloc, cudaFree or
+ * allocating library routine.
+ *
+ *   - The first call on each device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress, which may load the library's module there);
+ *     make that first call outside any stream capture.
+ *   - A geometry whose scratch would exceed TQ_NOALLOC_SCRATCH_BYTES (see
+ *     tq_decode_workspace_size for the size) is rejected with TQ_ERR_WORKSPACE and
+ *     nothing is enqueued.
+ *   - Every call on a device shares the one array, and it keeps whatever the last
+ *     call left there (no call needs it zeroed).  Calls whose kernels overlap on the
+ *     GPU (different streams without ordering) race on it: order them. */
+#define TQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+TQ_API tq_status tq_paged_decode_noalloc(tq_tensor out, tq_tensor q, tq_tensor pages,
+                                         tq_tensor block_table, tq_tensor seq_lens,
+                                         const tq_codebooks* cb, uint64_t sign_seed, float scale,
+                                         void* stream);
+
 /* Workspace bytes tq_paged_decode needs for this geometry (host only).  The
  * workspace holds the split-KV partial results (m, l, O') in fp32. */
 TQ_API tq_status tq_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,

@@ -11,6 +11,7 @@ Public API (names follow the C entry points):
     load_codebooks(D, k_bits, v_bits, device) -> Codebooks
     quantize_append(pages, slot_mapping, k, v, codebooks, sign_seed, stream=None)
     paged_decode(out, q, pages, block_table, seq_lens, codebooks, sign_seed, scale, stream=None)
+    paged_decode_noalloc(...)   # same, with the library's fixed scratch (no allocation)
     rotate_unit(u, norm, x, sign_seed, stream=None)       # test export of the rotation
     decode_workspace_size(...), set_workspace(tensor), get_device_error(stream=None)
 """
@@ -28,6 +29,7 @@ from ._binding import (  # noqa: F401
     load_codebook_table,
     load_codebooks,
     paged_decode,
+    paged_decode_noalloc,
     quantize_append,
     rotate_unit,
     set_workspace,

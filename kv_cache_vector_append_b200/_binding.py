@@ -23,7 +23,7 @@ DEVERR_BLOCK_RANGE = 0x2
 DEVERR_NONFINITE = 0x4
 DEVERR_SEQLEN_RANGE = 0x8
 
-EXPORTED = ("tq_slot_bytes", "tq_quantize_append", "tq_paged_decode",
+EXPORTED = ("tq_slot_bytes", "tq_quantize_append", "tq_paged_decode", "tq_paged_decode_noalloc",
             "tq_decode_workspace_size", "tq_set_workspace", "tq_get_device_error",
             "tq_rotate_unit", "tq_status_string", "tq_version")
 
@@ -70,6 +70,8 @@ def _load():
                                        ctypes.c_int32, ctypes.c_void_p]
     lib.tq_paged_decode.argtypes = [T, T, T, T, T, CB, ctypes.c_uint64, ctypes.c_float,
                                     ctypes.c_void_p]
+    lib.tq_paged_decode_noalloc.argtypes = [T, T, T, T, T, CB, ctypes.c_uint64, ctypes.c_float,
+                                            ctypes.c_void_p]
     lib.tq_decode_workspace_size.argtypes = [ctypes.c_int32] * 6 + [ctypes.POINTER(ctypes.c_size_t)]
     lib.tq_set_workspace.argtypes = [ctypes.c_void_p, ctypes.c_size_t]
     lib.tq_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p]
@@ -220,6 +222,21 @@ def paged_decode(out, q, pages, block_table, seq_lens, codebooks: Codebooks, sig
                                    _desc(seq_lens), ctypes.byref(codebooks.desc),
                                    ctypes.c_uint64(sign_seed), ctypes.c_float(scale), st),
            "tq_paged_decode")
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def paged_decode_noalloc(out, q, pages, block_table, seq_lens, codebooks: Codebooks,
+                         sign_seed: int, scale: float, stream=None) -> None:
+    """tq_paged_decode_noalloc: the decode with the library's fixed scratch array
+    (no device allocation on the call path; see include/tq.h)."""
+    _require_cuda(out, q, pages, block_table, seq_lens)
+    st = _stream_handle(stream, q.device)
+    _check(_load().tq_paged_decode_noalloc(_desc(out), _desc(q), _desc(pages), _desc(block_table),
+                                           _desc(seq_lens), ctypes.byref(codebooks.desc),
+                                           ctypes.c_uint64(sign_seed), ctypes.c_float(scale), st),
+           "tq_paged_decode_noalloc")
 
 
 def rotate_unit(u, norm, x, sign_seed: int, stream=None) -> None:

@@ -14,6 +14,12 @@ namespace tq {
 
 __device__ unsigned int g_tq_error_word;
 
+// Scratch of tq_paged_decode_noalloc: a fixed device array that every device which
+// loads the library holds until the process exits.  Host code never dereferences
+// this name (on the host it is only a stand-in); its device address is looked up
+// per device with cudaGetSymbolAddress.
+static __device__ __align__(256) uint8_t g_tq_noalloc_scratch[TQ_NOALLOC_SCRATCH_BYTES];
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -24,6 +30,7 @@ struct DeviceState {
   size_t user_ws_bytes = 0;
   void* lib_ws = nullptr;
   size_t lib_ws_bytes = 0;
+  uint8_t* noalloc_scratch = nullptr;   // device address of g_tq_noalloc_scratch
   DeviceInfo info;
 };
 
@@ -128,6 +135,142 @@ tq_status plan_decode(int batch, int h_q, int h_kv, int dim, int kb, int vb, int
                                         std::min(kDecodeWarps / h_kv, 4) * h_q * (dim + 2) *
                                         sizeof(float);
   return TQ_OK;
+}
+
+struct DecodeCall {
+  int B = 0, h_q = 0, h_kv = 0, D = 0, kbits = 0, vbits = 0, kb = 0, max_blocks = 0;
+  int64_t stride = 0;
+  DeviceState* ds = nullptr;
+  DecodePlan plan;
+};
+
+// Validation and geometry of one decode call (shared by the decode entry points).
+tq_status decode_prepare(const tq_tensor& out, const tq_tensor& q, const tq_tensor& pages,
+                         const tq_tensor& block_table, const tq_tensor& seq_lens,
+                         const tq_codebooks* cb, float scale, DecodeCall* call) {
+  if (cb == nullptr || !std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(q, 3) || !is_float_dtype(q.dtype) || q.stride[2] != 1) return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(out, 3) || !is_float_dtype(out.dtype) || out.stride[2] != 1 ||
+      (out.dtype != TQ_F32 && out.dtype != q.dtype))
+    return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(pages, 4) || pages.dtype != TQ_U8) return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(block_table, 2) || block_table.dtype != TQ_I32 || block_table.stride[1] != 1)
+    return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(seq_lens, 1) || seq_lens.dtype != TQ_I32 || seq_lens.stride[0] != 1)
+    return TQ_ERR_INVALID_ARG;
+  const int B = (int)q.shape[0], h_q = (int)q.shape[1], D = (int)q.shape[2];
+  const int h_kv = (int)pages.shape[2];
+  for (int i = 0; i < 3; ++i)
+    if (out.shape[i] != q.shape[i]) return TQ_ERR_INVALID_ARG;
+  if (block_table.shape[0] != B || seq_lens.shape[0] != B) return TQ_ERR_INVALID_ARG;
+  if (h_kv < 1 || h_q % h_kv) return TQ_ERR_INVALID_ARG;
+  if (!valid_codebook(cb->k, D) || !valid_codebook(cb->v, D)) return TQ_ERR_INVALID_ARG;
+  const int kbits = cb->k.bits, vbits = cb->v.bits;
+  const int kb = region_bytes(D, kbits), vb = region_bytes(D, vbits);
+  const int64_t stride = pages.shape[3];
+  if (stride < kb + vb || stride % 8) return TQ_ERR_INVALID_ARG;
+  // contiguous page tensor: whole blocks are staged with 16-byte copies
+  if (pages.stride[3] != 1 || pages.stride[2] != stride || pages.stride[1] != h_kv * stride ||
+      pages.stride[0] != pages.shape[1] * h_kv * stride || (uintptr_t)pages.data % 16)
+    return TQ_ERR_INVALID_ARG;
+  if (pages.shape[1] != kBlockSize) return TQ_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128 && D != 256) return TQ_ERR_UNSUPPORTED;
+  if (h_q / h_kv > 16 || h_kv > kDecodeWarps) return TQ_ERR_UNSUPPORTED;
+  if (!decode_bits_supported(kbits, vbits)) return TQ_ERR_UNSUPPORTED;
+  call->B = B;
+  if (B == 0) return TQ_OK;
+  DeviceState* ds = nullptr;
+  tq_status s = device_state(&ds);
+  if (s != TQ_OK) return s;
+  const int max_blocks = (int)block_table.shape[1];
+  const bool shared_lut = cb->k.bits == cb->v.bits && cb->k.centroids == cb->v.centroids;
+  DecodePlan plan;
+  s = plan_decode(B, h_q, h_kv, D, kbits, vbits, (int)stride, std::max(max_blocks, 1), shared_lut,
+                  ds->info, &plan);
+  if (s != TQ_OK) return s;
+  if ((h_kv * stride) % 8) return TQ_ERR_INVALID_ARG;
+  call->h_q = h_q;
+  call->h_kv = h_kv;
+  call->D = D;
+  call->kbits = kbits;
+  call->vbits = vbits;
+  call->kb = kb;
+  call->stride = stride;
+  call->max_blocks = max_blocks;
+  call->ds = ds;
+  call->plan = plan;
+  return TQ_OK;
+}
+
+// Launch the decode kernels of a prepared call on workspace `ws` (plan.ws_bytes bytes).
+tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tensor& q,
+                     const tq_tensor& pages, const tq_tensor& block_table,
+                     const tq_tensor& seq_lens, const tq_codebooks* cb, uint64_t sign_seed,
+                     float scale, uint8_t* ws, void* stream) {
+  const int B = call.B, h_q = call.h_q, h_kv = call.h_kv, D = call.D;
+  const int kbits = call.kbits, vbits = call.vbits, kb = call.kb;
+  const int64_t stride = call.stride;
+  const int max_blocks = call.max_blocks;
+  DeviceState* ds = call.ds;
+  const DecodePlan& plan = call.plan;
+  QPrepParams qp{};
+  qp.q = q.data;
+  qp.q_bstride = q.stride[0];
+  qp.q_hstride = q.stride[1];
+  qp.q_dtype = q.dtype;
+  qp.h_q = h_q;
+  qp.scale_log2 = scale * 1.4426950408889634f;
+  qp.sign_seed = sign_seed;
+  qp.qfrag = (uint32_t*)(ws + plan.qfrag_off);
+  qp.qscale = (float*)(ws + plan.qscale_off);
+
+  DecodeParams p{};
+  p.pages = (const uint8_t*)pages.data;
+  p.num_blocks = (int32_t)pages.shape[0];
+  p.h_kv = h_kv;
+  p.slot_stride = (int32_t)stride;
+  p.row_pitch = plan.row_pitch;
+  p.blk_stride = pages.stride[0];
+  p.block_table = (const int32_t*)block_table.data;
+  p.bt_stride = block_table.stride[0];
+  p.max_blocks = max_blocks;
+  p.seq_lens = (const int32_t*)seq_lens.data;
+  p.batch = B;
+  p.h_q = h_q;
+  p.group = h_q / h_kv;
+  p.kc = cb->k.centroids;
+  p.vc = cb->v.centroids;
+  p.shared_lut = plan.shared_lut;
+  p.k_region = kb;
+  p.wph = plan.wph;
+  p.stage_bytes = plan.stage_bytes;
+  p.ids_cap = plan.ids_cap;
+  p.row_copies = plan.row_copies;
+  p.qfrag = qp.qfrag;
+  p.qscale = qp.qscale;
+  p.prefix = (int32_t*)(ws + plan.prefix_off);
+  p.part = (float*)(ws + plan.part_off);
+  p.err = ds->err;
+
+  MergeParams m{};
+  m.part = p.part;
+  m.prefix = p.prefix;
+  m.out = out.data;
+  m.o_bstride = out.stride[0];
+  m.o_hstride = out.stride[1];
+  m.out_dtype = out.dtype;
+  m.h_q = h_q;
+  m.wph = plan.wph;
+  m.sign_seed = sign_seed;
+
+  const int64_t per_step = plan.wph;
+  const int64_t steps_upper = (int64_t)B * ((max_blocks + per_step - 1) / per_step);
+  cudaStream_t st = as_stream(stream);
+  switch (D) {
+    case 64: return launch_decode_d64(kbits, vbits, p, qp, m, plan, steps_upper, st);
+    case 128: return launch_decode_d128(kbits, vbits, p, qp, m, plan, steps_upper, st);
+    default: return launch_decode_d256(kbits, vbits, p, qp, m, plan, steps_upper, st);
+  }
 }
 
 }  // namespace
@@ -300,47 +443,11 @@ tq_status tq_get_device_error(int32_t* out, void* stream) {
 tq_status tq_paged_decode(tq_tensor out, tq_tensor q, tq_tensor pages, tq_tensor block_table,
                           tq_tensor seq_lens, const tq_codebooks* cb, uint64_t sign_seed,
                           float scale, void* stream) {
-  if (cb == nullptr || !std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
-  if (!valid_tensor(q, 3) || !is_float_dtype(q.dtype) || q.stride[2] != 1) return TQ_ERR_INVALID_ARG;
-  if (!valid_tensor(out, 3) || !is_float_dtype(out.dtype) || out.stride[2] != 1 ||
-      (out.dtype != TQ_F32 && out.dtype != q.dtype))
-    return TQ_ERR_INVALID_ARG;
-  if (!valid_tensor(pages, 4) || pages.dtype != TQ_U8) return TQ_ERR_INVALID_ARG;
-  if (!valid_tensor(block_table, 2) || block_table.dtype != TQ_I32 || block_table.stride[1] != 1)
-    return TQ_ERR_INVALID_ARG;
-  if (!valid_tensor(seq_lens, 1) || seq_lens.dtype != TQ_I32 || seq_lens.stride[0] != 1)
-    return TQ_ERR_INVALID_ARG;
-  const int B = (int)q.shape[0], h_q = (int)q.shape[1], D = (int)q.shape[2];
-  const int h_kv = (int)pages.shape[2];
-  for (int i = 0; i < 3; ++i)
-    if (out.shape[i] != q.shape[i]) return TQ_ERR_INVALID_ARG;
-  if (block_table.shape[0] != B || seq_lens.shape[0] != B) return TQ_ERR_INVALID_ARG;
-  if (h_kv < 1 || h_q % h_kv) return TQ_ERR_INVALID_ARG;
-  if (!valid_codebook(cb->k, D) || !valid_codebook(cb->v, D)) return TQ_ERR_INVALID_ARG;
-  const int kbits = cb->k.bits, vbits = cb->v.bits;
-  const int kb = region_bytes(D, kbits), vb = region_bytes(D, vbits);
-  const int64_t stride = pages.shape[3];
-  if (stride < kb + vb || stride % 8) return TQ_ERR_INVALID_ARG;
-  // contiguous page tensor: whole blocks are staged with 16-byte copies
-  if (pages.stride[3] != 1 || pages.stride[2] != stride || pages.stride[1] != h_kv * stride ||
-      pages.stride[0] != pages.shape[1] * h_kv * stride || (uintptr_t)pages.data % 16)
-    return TQ_ERR_INVALID_ARG;
-  if (pages.shape[1] != kBlockSize) return TQ_ERR_UNSUPPORTED;
-  if (D != 64 && D != 128 && D != 256) return TQ_ERR_UNSUPPORTED;
-  if (h_q / h_kv > 16 || h_kv > kDecodeWarps) return TQ_ERR_UNSUPPORTED;
-  if (!decode_bits_supported(kbits, vbits)) return TQ_ERR_UNSUPPORTED;
-  if (B == 0) return TQ_OK;
-  DeviceState* ds = nullptr;
-  tq_status s = device_state(&ds);
-  if (s != TQ_OK) return s;
-  const int max_blocks = (int)block_table.shape[1];
-  const bool shared_lut = cb->k.bits == cb->v.bits && cb->k.centroids == cb->v.centroids;
-  DecodePlan plan;
-  s = plan_decode(B, h_q, h_kv, D, kbits, vbits, (int)stride, std::max(max_blocks, 1), shared_lut,
-                  ds->info, &plan);
-  if (s != TQ_OK) return s;
-  if ((h_kv * stride) % 8) return TQ_ERR_INVALID_ARG;
-
+  DecodeCall call;
+  tq_status s = decode_prepare(out, q, pages, block_table, seq_lens, cb, scale, &call);
+  if (s != TQ_OK || call.B == 0) return s;
+  DeviceState* ds = call.ds;
+  const DecodePlan& plan = call.plan;
   uint8_t* ws = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);
@@ -360,64 +467,34 @@ tq_status tq_paged_decode(tq_tensor out, tq_tensor q, tq_tensor pages, tq_tensor
     }
   }
 
-  QPrepParams qp{};
-  qp.q = q.data;
-  qp.q_bstride = q.stride[0];
-  qp.q_hstride = q.stride[1];
-  qp.q_dtype = q.dtype;
-  qp.h_q = h_q;
-  qp.scale_log2 = scale * 1.4426950408889634f;
-  qp.sign_seed = sign_seed;
-  qp.qfrag = (uint32_t*)(ws + plan.qfrag_off);
-  qp.qscale = (float*)(ws + plan.qscale_off);
+  return decode_run(call, out, q, pages, block_table, seq_lens, cb, sign_seed, scale, ws, stream);
+}
 
-  DecodeParams p{};
-  p.pages = (const uint8_t*)pages.data;
-  p.num_blocks = (int32_t)pages.shape[0];
-  p.h_kv = h_kv;
-  p.slot_stride = (int32_t)stride;
-  p.row_pitch = plan.row_pitch;
-  p.blk_stride = pages.stride[0];
-  p.block_table = (const int32_t*)block_table.data;
-  p.bt_stride = block_table.stride[0];
-  p.max_blocks = max_blocks;
-  p.seq_lens = (const int32_t*)seq_lens.data;
-  p.batch = B;
-  p.h_q = h_q;
-  p.group = h_q / h_kv;
-  p.kc = cb->k.centroids;
-  p.vc = cb->v.centroids;
-  p.shared_lut = plan.shared_lut;
-  p.k_region = kb;
-  p.wph = plan.wph;
-  p.stage_bytes = plan.stage_bytes;
-  p.ids_cap = plan.ids_cap;
-  p.row_copies = plan.row_copies;
-  p.qfrag = qp.qfrag;
-  p.qscale = qp.qscale;
-  p.prefix = (int32_t*)(ws + plan.prefix_off);
-  p.part = (float*)(ws + plan.part_off);
-  p.err = ds->err;
-
-  MergeParams m{};
-  m.part = p.part;
-  m.prefix = p.prefix;
-  m.out = out.data;
-  m.o_bstride = out.stride[0];
-  m.o_hstride = out.stride[1];
-  m.out_dtype = out.dtype;
-  m.h_q = h_q;
-  m.wph = plan.wph;
-  m.sign_seed = sign_seed;
-
-  const int64_t per_step = plan.wph;
-  const int64_t steps_upper = (int64_t)B * ((max_blocks + per_step - 1) / per_step);
-  cudaStream_t st = as_stream(stream);
-  switch (D) {
-    case 64: return launch_decode_d64(kbits, vbits, p, qp, m, plan, steps_upper, st);
-    case 128: return launch_decode_d128(kbits, vbits, p, qp, m, plan, steps_upper, st);
-    default: return launch_decode_d256(kbits, vbits, p, qp, m, plan, steps_upper, st);
+tq_status tq_paged_decode_noalloc(tq_tensor out, tq_tensor q, tq_tensor pages,
+                                  tq_tensor block_table, tq_tensor seq_lens,
+                                  const tq_codebooks* cb, uint64_t sign_seed, float scale,
+                                  void* stream) {
+  DecodeCall call;
+  tq_status s = decode_prepare(out, q, pages, block_table, seq_lens, cb, scale, &call);
+  if (s != TQ_OK || call.B == 0) return s;
+  if (call.plan.ws_bytes > TQ_NOALLOC_SCRATCH_BYTES) return TQ_ERR_WORKSPACE;
+  DeviceState* ds = call.ds;
+  uint8_t* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (ds->noalloc_scratch == nullptr) {
+      // one-time set-up on this device (the current one): the scratch array's address
+      void* addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_tq_noalloc_scratch) != cudaSuccess || addr == nullptr)
+        return TQ_ERR_CUDA;
+      ds->noalloc_scratch = (uint8_t*)addr;
+    }
+    ws = ds->noalloc_scratch;
   }
+  // Nothing in the scratch has to start at zero: every byte a launch reads (rotated
+  // queries, prefix sums, partial records) is written earlier in the same launch
+  // sequence, so the contents left by a previous call do no harm.
+  return decode_run(call, out, q, pages, block_table, seq_lens, cb, sign_seed, scale, ws, stream);
 }
 
 }  // extern "C"
