@@ -1,5 +1,6 @@
 // tq_api.cu -- the extern "C" boundary of libtq.so (declared in include/tq.h):
 // argument validation, kernel dispatch, per-device workspace and error word.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -103,12 +104,19 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 // Geometry of the decode kernels for one call (see tq_decode.cuh).
 tq_status plan_decode(int batch, int h_q, int h_kv, int dim, int kb, int vb, int slot_stride,
-                      int max_blocks, bool shared_lut, const DeviceInfo& di, DecodePlan* plan) {
+                      int max_blocks, bool shared_lut, bool allow_tensor_copy, const DeviceInfo& di,
+                      DecodePlan* plan) {
   if (h_kv < 1 || h_kv > kDecodeWarps) return TQ_ERR_UNSUPPORTED;
-  // whole page blocks are staged with one bulk copy each (unpadded rows): on B200 one
-  // 17 KB copy per block streams far better than one ~1 KB copy per row
-  plan->row_copies = 0;
-  plan->row_pitch = h_kv * slot_stride;
+  // A block is staged by one TMA copy.  When a row is a multiple of 16 bytes and the
+  // padded row fits a tensor box (at most 256 u64 columns), the copy is a 2-D box of
+  // 16 rows x pitch/8 u64 whose columns past the row end are zero-filled, giving rows
+  // padded to a pitch of 20 (mod 32) words; otherwise it is a 1-D bulk copy of the
+  // block with unpadded rows.
+  const int row_bytes = h_kv * slot_stride;
+  int words = row_bytes / 4;
+  words += ((20 - words % 32) + 32) % 32;
+  plan->copy_mode = allow_tensor_copy && row_bytes % 16 == 0 && 4 * words / 8 <= 256;
+  plan->row_pitch = plan->copy_mode ? 4 * words : row_bytes;
   plan->shared_lut = shared_lut && kb == vb;
   const size_t lut = decode_lut_bytes(kb, vb, plan->shared_lut);
   // at most 4 blocks per step, so that one warp issues a step's row copies in two rounds
@@ -119,7 +127,7 @@ tq_status plan_decode(int batch, int h_q, int h_kv, int dim, int kb, int vb, int
     const int64_t steps_upper = (int64_t)batch * ((max_blocks + plan->wph - 1) / plan->wph);
     const int64_t per_cta = (steps_upper + 2 * di.num_sms - 1) / (2 * di.num_sms) + 1;
     plan->ids_cap = (int)std::min<int64_t>(per_cta * plan->wph, 4096);
-    plan->smem = lut + (size_t)kDecodeStages * plan->stage_bytes + kDecodeStages * 16 +
+    plan->smem = lut + 128 + (size_t)kDecodeStages * plan->stage_bytes + kDecodeStages * 16 +
                  4 * ((size_t)batch + 1) + 4 * ((1 << kb) + (1 << vb)) + 4 * plan->ids_cap + 16;
     if ((int)plan->smem <= di.max_smem_optin || plan->wph == 1) break;
     plan->wph /= 2;
@@ -135,6 +143,40 @@ tq_status plan_decode(int batch, int h_q, int h_kv, int dim, int kb, int vb, int
                                         std::min(kDecodeWarps / h_kv, 4) * h_q * (dim + 2) *
                                         sizeof(float);
   return TQ_OK;
+}
+
+// cuTensorMapEncodeTiled, looked up once through the runtime (no link against libcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// Tensor map of the page pool seen as (num_blocks * 16) rows of row_bytes / 8 u64
+// columns, read in boxes of 16 rows x pitch / 8 columns (columns past the row end are
+// out of bounds and zero-filled).  Returns false when the driver rejects the map.
+bool encode_page_map(CUtensorMap* map, const void* pages, int64_t num_blocks, int row_bytes,
+                     int pitch) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (fn == nullptr || num_blocks * kBlockSize > 0xffffffffll) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)(row_bytes / 8), (cuuint64_t)(num_blocks * kBlockSize)};
+  const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  const cuuint32_t box[2] = {(cuuint32_t)(pitch / 8), (cuuint32_t)kBlockSize};
+  const cuuint32_t estride[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void*>(pages), dims, strides, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 struct DecodeCall {
@@ -186,7 +228,7 @@ tq_status decode_prepare(const tq_tensor& out, const tq_tensor& q, const tq_tens
   const bool shared_lut = cb->k.bits == cb->v.bits && cb->k.centroids == cb->v.centroids;
   DecodePlan plan;
   s = plan_decode(B, h_q, h_kv, D, kbits, vbits, (int)stride, std::max(max_blocks, 1), shared_lut,
-                  ds->info, &plan);
+                  true, ds->info, &plan);
   if (s != TQ_OK) return s;
   if ((h_kv * stride) % 8) return TQ_ERR_INVALID_ARG;
   call->h_q = h_q;
@@ -212,7 +254,16 @@ tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tens
   const int64_t stride = call.stride;
   const int max_blocks = call.max_blocks;
   DeviceState* ds = call.ds;
-  const DecodePlan& plan = call.plan;
+  DecodePlan plan = call.plan;
+  CUtensorMap tmap;
+  std::memset(&tmap, 0, sizeof(tmap));
+  if (plan.copy_mode &&
+      !encode_page_map(&tmap, pages.data, pages.shape[0], h_kv * (int)stride, plan.row_pitch)) {
+    // the 1-D bulk layout never needs more shared memory or workspace than the 2-D one
+    const tq_status s = plan_decode(B, h_q, h_kv, D, kbits, vbits, (int)stride,
+                                    std::max(max_blocks, 1), plan.shared_lut, false, ds->info, &plan);
+    if (s != TQ_OK) return s;
+  }
   QPrepParams qp{};
   qp.q = q.data;
   qp.q_bstride = q.stride[0];
@@ -245,7 +296,7 @@ tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tens
   p.wph = plan.wph;
   p.stage_bytes = plan.stage_bytes;
   p.ids_cap = plan.ids_cap;
-  p.row_copies = plan.row_copies;
+  p.copy_mode = plan.copy_mode;
   p.qfrag = qp.qfrag;
   p.qscale = qp.qscale;
   p.prefix = (int32_t*)(ws + plan.prefix_off);
@@ -267,9 +318,9 @@ tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tens
   const int64_t steps_upper = (int64_t)B * ((max_blocks + per_step - 1) / per_step);
   cudaStream_t st = as_stream(stream);
   switch (D) {
-    case 64: return launch_decode_d64(kbits, vbits, p, qp, m, plan, steps_upper, st);
-    case 128: return launch_decode_d128(kbits, vbits, p, qp, m, plan, steps_upper, st);
-    default: return launch_decode_d256(kbits, vbits, p, qp, m, plan, steps_upper, st);
+    case 64: return launch_decode_d64(kbits, vbits, p, qp, m, plan, tmap, steps_upper, st);
+    case 128: return launch_decode_d128(kbits, vbits, p, qp, m, plan, tmap, steps_upper, st);
+    default: return launch_decode_d256(kbits, vbits, p, qp, m, plan, tmap, steps_upper, st);
   }
 }
 
@@ -328,6 +379,7 @@ tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_tensor 
       (uintptr_t)pages.data % 4)
     return TQ_ERR_INVALID_ARG;
   if (T == 0 || h_kv == 0) return TQ_OK;
+  if (T * h_kv >= ((int64_t)1 << 31) - 64) return TQ_ERR_UNSUPPORTED;   // 32-bit row indices
   DeviceState* ds = nullptr;
   tq_status s = device_state(&ds);
   if (s != TQ_OK) return s;
@@ -336,6 +388,9 @@ tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_tensor 
   p.pages = (uint8_t*)pages.data;
   p.num_slots = pages.shape[0] * pages.shape[1];
   p.block_size = (int32_t)pages.shape[1];
+  p.bs_shift = -1;
+  for (int sh = 0; sh < 31; ++sh)
+    if ((int64_t)1 << sh == pages.shape[1]) p.bs_shift = sh;
   p.h_kv = h_kv;
   p.blk_stride = pages.stride[0];
   p.row_stride = pages.stride[1];
@@ -407,8 +462,8 @@ tq_status tq_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t n
   // the record area is sized for the largest warps-per-head count, so any bit widths fit
   DecodePlan plan;
   s = plan_decode(std::max(batch, 1), num_q_heads, num_kv_heads, head_dim, 1, 1,
-                  region_bytes(head_dim, 1) * 2 + 8, std::max(max_blocks, 1), false, ds->info,
-                  &plan);
+                  region_bytes(head_dim, 1) * 2 + 8, std::max(max_blocks, 1), false, false,
+                  ds->info, &plan);
   if (s != TQ_OK) return s;
   *bytes = plan.ws_bytes;
   return TQ_OK;

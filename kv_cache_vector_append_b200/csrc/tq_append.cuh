@@ -46,6 +46,7 @@ struct AppendParams {
   uint64_t sign_seed;
   unsigned int* err;
   int32_t align_mode;       // 16: rows 16-byte aligned; 4: 4-byte aligned; 0: any
+  int32_t bs_shift;         // log2(block_size) when it is a power of two, else -1
 };
 
 struct RotateParams {      // test export of the rotation (tq_rotate_unit)
@@ -81,6 +82,8 @@ struct alignas(16) EncodeTables {
   int fast;                 // bucket encode valid for this table
 };
 
+// Phase 1 (then a CTA barrier, then phase 2): boundaries, Eytzinger image, and the
+// check that no two boundaries share a bucket.
 __device__ __forceinline__ void build_tables(EncodeTables* t, const float* b, int bits, int tid,
                                              int nthreads) {
   const int n = (1 << bits) - 1;
@@ -97,16 +100,26 @@ __device__ __forceinline__ void build_tables(EncodeTables* t, const float* b, in
         ok = 0;
     t->fast = ok;
   }
-  // k0 of each bucket: the lowest float of bucket g is g << 20 for a positive bucket
-  // and -((g & 0x7ff) << 20 | 0xfffff) for a negative one.  (Only used for bits <= 4.)
+}
+
+// Phase 2: k0 of each bucket = #{b_i < lowest float of the bucket}, by binary search
+// over the boundaries already in shared memory.  The lowest float of bucket g is
+// g << 20 for a positive bucket and -((g & 0x7ff) << 20 | 0xfffff) for a negative one.
+// Only used for bits <= 4.
+__device__ __forceinline__ void build_bucket_table(EncodeTables* t, int bits, int tid,
+                                                   int nthreads) {
   if (bits > 4) return;
+  const int n = (1 << bits) - 1;
   for (int g = tid; g < kBuckets; g += nthreads) {
     const uint32_t lowbits = (g & 0x800) ? ((uint32_t)g << kBucketShift) | 0xFFFFFu
                                          : (uint32_t)g << kBucketShift;
     const float lo = __uint_as_float(lowbits);
-    int c = 0;
-    for (int i = 0; i < n; ++i) c += (b[i] < lo) ? 1 : 0;
-    t->k0[g] = (uint8_t)c;
+    int a = 0, c = n;                   // count of boundaries < lo lies in [a, c]
+    while (a < c) {
+      const int m = (a + c) >> 1;
+      if (t->bnd[m] < lo) a = m + 1; else c = m;
+    }
+    t->k0[g] = (uint8_t)a;
   }
 }
 
@@ -266,7 +279,8 @@ struct AppendSmem {
   using G = AppendGeom<D>;
   static constexpr int RB = D * InType<Tin>::kBytes;
   static constexpr int INPITCH = RB + 16;
-  static constexpr int PER_WARP = 2 * G::ROWS * INPITCH + G::ROWS * G::OUTPITCH * 4 + G::ROWS * 8;
+  static constexpr int PER_WARP =
+      2 * G::ROWS * INPITCH + G::ROWS * G::OUTPITCH * 4 + 2 * G::ROWS * 8 + 2 * G::ROWS * 8;
   static constexpr int TABLES = ((2 * (int)sizeof(EncodeTables) + 4 * D) + 127) / 128 * 128;
   static constexpr int BYTES = TABLES + kAppendWarps * PER_WARP;
 };
@@ -282,28 +296,50 @@ append_kernel(AppendParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* in_s = smem + SM::TABLES + warp * SM::PER_WARP;
   uint32_t* out_s = (uint32_t*)(in_s + 2 * G::ROWS * SM::INPITCH);
-  int64_t* dst_s = (int64_t*)(out_s + G::ROWS * G::OUTPITCH);
+  int64_t* dst_s = (int64_t*)(out_s + G::ROWS * G::OUTPITCH);     // [2][ROWS] region offsets
+  const uint8_t** src_s = (const uint8_t**)(dst_s + 2 * G::ROWS);  // [2][ROWS] row addresses
 
-  const int64_t rows_per_kind = p.num_tokens * p.h_kv;
+  const int64_t rows_per_kind = p.num_tokens * p.h_kv;            // < 2^31 (host check)
   const int64_t tiles_per_kind = (rows_per_kind + G::ROWS - 1) / G::ROWS;
   const int64_t ntiles = 2 * tiles_per_kind;
   const int64_t gwarp = (int64_t)blockIdx.x * kAppendWarps + warp;
   const int64_t nwarps = (int64_t)gridDim.x * kAppendWarps;
 
+  // Stage tile `tile` into buffer `buf`: lane r < ROWS resolves row r0 + r once (its
+  // input address and its slot's region offset), then the warp copies the rows.
   auto issue = [&](int64_t tile, int buf) {
     const int kind = tile >= tiles_per_kind;
-    const int64_t r0 = (tile - kind * tiles_per_kind) * G::ROWS;
+    const int r0 = (int)((tile - kind * tiles_per_kind) * G::ROWS);
     const int nr = (int)imin64((int64_t)G::ROWS, rows_per_kind - r0);
-    const Tin* base = (const Tin*)p.src[kind];
-    const int64_t ts = p.tok_stride[kind], hs = p.head_stride_in[kind];
-    const int hk = p.h_kv;
+    if (lane < nr) {
+      const uint32_t row = (uint32_t)(r0 + lane);
+      const uint32_t t = row / (uint32_t)p.h_kv;
+      const uint32_t h = row - t * (uint32_t)p.h_kv;
+      src_s[buf * G::ROWS + lane] =
+          (const uint8_t*)p.src[kind] +
+          ((int64_t)t * p.tok_stride[kind] + (int64_t)h * p.head_stride_in[kind]) * SM::RB / D;
+      const int64_t slot = p.slot_mapping[(int64_t)t * p.slot_map_stride];
+      int64_t off = -1;
+      if (slot >= 0) {
+        if (slot < p.num_slots) {
+          int64_t blk, rr;
+          if (p.bs_shift >= 0) {
+            blk = slot >> p.bs_shift;
+            rr = slot & ((1 << p.bs_shift) - 1);
+          } else {
+            blk = slot / p.block_size;
+            rr = slot - blk * p.block_size;
+          }
+          off = blk * p.blk_stride + rr * p.row_stride + h * p.head_stride + p.region_off[kind];
+        } else {
+          report_error(p.err, TQ_DEVERR_SLOT_RANGE);
+        }
+      }
+      dst_s[buf * G::ROWS + lane] = off;
+    }
+    __syncwarp();
     stage_rows<SM::RB>(in_s + buf * G::ROWS * SM::INPITCH, SM::INPITCH, nr,
-                       [&](int r) {
-                         const int64_t row = r0 + r;
-                         const int64_t t = row / hk;
-                         const int h = (int)(row - t * hk);
-                         return (const void*)(base + t * ts + h * hs);
-                       },
+                       [&](int r) { return (const void*)src_s[buf * G::ROWS + r]; },
                        p.align_mode, lane);
   };
   // the first tile's rows are in flight while the tables are built
@@ -312,6 +348,9 @@ append_kernel(AppendParams p) {
   build_tables(&tabs[0], p.boundaries[0], p.bits[0], threadIdx.x, blockDim.x);
   build_tables(&tabs[1], p.boundaries[1], p.bits[1], threadIdx.x, blockDim.x);
   for (int j = threadIdx.x; j < D; j += blockDim.x) smask[j] = sign_mask_at(p.sign_seed, j);
+  __syncthreads();
+  build_bucket_table(&tabs[0], p.bits[0], threadIdx.x, blockDim.x);
+  build_bucket_table(&tabs[1], p.bits[1], threadIdx.x, blockDim.x);
   __syncthreads();
 
   const int rl = lane % G::ROWS;           // row within the tile
@@ -326,23 +365,6 @@ append_kernel(AppendParams p) {
     const int nr = (int)imin64((int64_t)G::ROWS, rows_per_kind - r0);
     const int bits = p.bits[kind];
     const int nw = D * bits / 32 + 1;   // packed words + norm word
-    // destination byte offset of each row's region (-1: skip)
-    if (lane < nr) {
-      const int64_t row = r0 + lane;
-      const int64_t t = row / p.h_kv;
-      const int h = (int)(row - t * p.h_kv);
-      const int64_t slot = p.slot_mapping[t * p.slot_map_stride];
-      int64_t off = -1;
-      if (slot >= 0) {
-        if (slot < p.num_slots) {
-          const int64_t blk = slot / p.block_size, rr = slot - blk * p.block_size;
-          off = blk * p.blk_stride + rr * p.row_stride + h * p.head_stride + p.region_off[kind];
-        } else {
-          report_error(p.err, TQ_DEVERR_SLOT_RANGE);
-        }
-      }
-      dst_s[lane] = off;
-    }
     cp_async_wait<1>();
     __syncwarp();
     {
@@ -376,7 +398,7 @@ append_kernel(AppendParams p) {
     __syncwarp();
     // write back: one row region per pass (contiguous words)
     for (int rr = 0; rr < nr; ++rr) {
-      const int64_t off = dst_s[rr];
+      const int64_t off = dst_s[buf * G::ROWS + rr];
       if (off < 0) continue;
       uint32_t* dst = (uint32_t*)(p.pages + off);
       const uint32_t* src = out_s + rr * G::OUTPITCH;

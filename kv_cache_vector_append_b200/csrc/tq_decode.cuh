@@ -18,9 +18,11 @@
 // steps (stream-K style), so ragged batches and single long sequences balance
 // alike.  Inside a CTA one warp serves one (KV head, sub-stream):
 //   * page blocks (16 tokens x all KV heads; one per sub-stream and step) are staged
-//     into shared memory by bulk (TMA) copies, one per block, into a 4-deep ring of
-//     stages guarded by mbarriers; the last warp to release a stage refills it, so no
-//     warp ever waits for the whole CTA;
+//     into shared memory by one TMA tensor copy each (a 16-row box one padding wider
+//     than a row, the padding zero-filled out of bounds) into a 4-deep ring of stages
+//     guarded by mbarriers; the last warp to release a stage refills it, so no warp
+//     ever waits for the whole CTA; the padded pitch of 20 (mod 32) words makes the
+//     per-thread code loads below bank-conflict free;
 //   * codes become fp16 through per-lane replicated lookup tables of code PAIRS
 //     (bits <= 4: entry (x | y << bits) = (c[x], c[y])) or single codes, so that
 //     the 32 lanes of a warp always hit 32 different banks;
@@ -49,7 +51,7 @@ namespace tq {
 constexpr int kBlockSize = 16;        // tokens per page block
 constexpr int kDecodeWarps = 8;
 constexpr int kDecodeStages = 4;
-constexpr uint32_t kWaitLimit = 1u << 24;   // polls before a wait gives up (> 1 s)
+constexpr uint32_t kWaitLimit = 2000;      // polls (each <= ~1 ms) before a wait gives up
 constexpr float kLazyRescale = 8.0f;  // log2 units
 
 struct DecodeParams {
@@ -73,7 +75,8 @@ struct DecodeParams {
   int32_t wph;                  // warps (sub-streams) per KV head = blocks per step
   int32_t stage_bytes;
   int32_t ids_cap;              // block ids of its step range a CTA preloads (entries)
-  int32_t row_copies;           // 1: one bulk copy per page row (padded pitch); 0: per block
+  int32_t copy_mode;            // 1: 2-D tensor box per block (rows padded to row_pitch)
+                                // 0: 1-D bulk copy per block (row_pitch = row bytes)
   const uint32_t* qfrag;        // [B][H_q][4 tig][KSTEPS][2] half2, from qprep_kernel
   const float* qscale;          // [B][H_q]: |q'| * scale * log2(e)
   int32_t* prefix;              // [B + 1] step prefix sums (written by CTA 0)
@@ -337,7 +340,7 @@ __device__ __forceinline__ float log2_ceilish(float x) {
 // centroids].
 template <int D, int KB, int VB, int NH>
 __global__ void __launch_bounds__(kDecodeWarps * 32, (NH == 1 && D <= 128) ? 2 : 1)
-decode_kernel(DecodeParams p) {
+decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   using C = DecodeCfg<D, KB, VB>;
   using KS = typename C::KS;
   using VS = typename C::VS;
@@ -349,6 +352,7 @@ decode_kernel(DecodeParams p) {
   const bool one_lut = KB == VB && p.shared_lut;
   uint32_t* lutV = one_lut ? lutK : lutK + LK::kBytes / 4;
   uint8_t* stages = smem + (one_lut ? LK::kBytes : C::kLutBytes);
+  stages += (128u - (smem_u32(stages) & 127u)) & 127u;   // TMA destinations: 128-byte aligned
   uint64_t* full = (uint64_t*)(stages + NST * p.stage_bytes);
   int* released = (int*)(full + NST);
   uint32_t* present = (uint32_t*)(released + NST);     // per stage: bit k = block k staged
@@ -439,50 +443,27 @@ decode_kernel(DecodeParams p) {
     ids[i] = block_id(s0 + i / per_step, (int)(i % per_step));
   __syncthreads();
 
-  // Stage refill for global step s (issued by one whole warp): bulk copies of the
-  // step's page rows (or whole blocks), completing on full[stage]; present[stage]
-  // tells the consumers which blocks arrived.
+  // Stage refill for global step s (issued by one warp): one TMA copy per block of
+  // the step, completing on full[stage]; present[stage] tells the consumers which
+  // blocks were staged.  With copy_mode 1 the block is a 2-D box of 16 rows whose
+  // width is the padded pitch: the columns past the row end lie outside the tensor
+  // and are zero-filled, which pads every row in shared memory.
+  const uint32_t blk_copy_bytes = p.copy_mode ? (uint32_t)blk_smem : (uint32_t)(kBlockSize * row_bytes);
   auto refill = [&](int64_t s) {
     const int x = (int)((s - s0) % NST);
-    const int ncopies = p.row_copies ? per_step * kBlockSize : per_step;
-    const uint32_t cbytes = p.row_copies ? (uint32_t)row_bytes : (uint32_t)(kBlockSize * row_bytes);
     const int64_t i0 = (s - s0) * per_step;
-    uint32_t mine = 0, bits = 0;
-    int32_t myblk[2] = {-1, -1};                       // ncopies <= 64 (wph <= 4 rows)
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int c = lane + 32 * j;
-      if (c < ncopies) {
-        const int k = p.row_copies ? c / kBlockSize : c;
-        const int32_t blk = i0 + k < p.ids_cap ? ids[i0 + k] : block_id(s, k);
-        myblk[j] = blk;
-        if (blk >= 0) {
-          mine += cbytes;
-          bits |= 1u << k;
-        }
-      }
-    }
-    uint32_t total = mine;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      total += __shfl_xor_sync(0xffffffffu, total, o);
-      bits |= __shfl_xor_sync(0xffffffffu, bits, o);
-    }
+    int32_t blk = -1;
+    if (lane < per_step) blk = i0 + lane < p.ids_cap ? ids[i0 + lane] : block_id(s, lane);
+    const uint32_t bits = __ballot_sync(0xffffffffu, blk >= 0);
     if (lane == 0) {
       present[x] = bits;                 // published by the arrive (release) below
-      mbar_arrive_expect_tx(&full[x], total);
+      mbar_arrive_expect_tx(&full[x], __popc(bits) * blk_copy_bytes);
     }
     __syncwarp();
-    uint8_t* dst = stages + x * p.stage_bytes;
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int c = lane + 32 * j;
-      if (c < ncopies && myblk[j] >= 0) {
-        const int k = p.row_copies ? c / kBlockSize : c;
-        const int r = p.row_copies ? c % kBlockSize : 0;
-        const uint8_t* src = p.pages + (int64_t)myblk[j] * p.blk_stride + (int64_t)r * row_bytes;
-        bulk_g2s(dst + k * blk_smem + r * pitch, src, cbytes, &full[x]);
-      }
+    if (blk >= 0) {
+      uint8_t* d = stages + x * p.stage_bytes + lane * blk_smem;
+      if (p.copy_mode) tensor_g2s_2d(d, &tmap, 0, blk * kBlockSize, &full[x]);
+      else bulk_g2s(d, p.pages + (int64_t)blk * p.blk_stride, blk_copy_bytes, &full[x]);
     }
   };
   if (warp == 0)

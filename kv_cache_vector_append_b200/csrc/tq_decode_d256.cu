@@ -3,8 +3,8 @@
 
 namespace tq {
 tq_status launch_decode_d256(int kb, int vb, const DecodeParams& p, const QPrepParams& qp,
-                            const MergeParams& m, const DecodePlan& plan, int64_t steps_upper,
-                            cudaStream_t st) {
-  return launch_decode_dim<256>(kb, vb, p, qp, m, plan, steps_upper, st);
+                            const MergeParams& m, const DecodePlan& plan,
+                            const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st) {
+  return launch_decode_dim<256>(kb, vb, p, qp, m, plan, tmap, steps_upper, st);
 }
 }  // namespace tq

@@ -22,7 +22,7 @@ struct DecodePlan {
   int row_pitch = 0;      // padded shared-memory row pitch (bytes)
   int stage_bytes = 0;    // one pipeline stage: wph blocks
   int ids_cap = 0;        // block ids a CTA preloads into shared memory
-  int row_copies = 0;     // one bulk copy per page row (padded pitch) or per block
+  int copy_mode = 0;      // 1: 2-D tensor box per block (padded rows); 0: 1-D bulk copy
   int shared_lut = 0;     // K and V share one lookup table
   size_t smem = 0;        // dynamic shared memory of the decode kernel
   int max_ctas = 0;       // upper bound of the persistent grid
@@ -39,14 +39,14 @@ tq_status launch_append_any(int dim, int dtype, const AppendParams& p, const Dev
 tq_status launch_rotate_any(int dim, int dtype, const RotateParams& p, const DeviceInfo& di,
                             cudaStream_t st);
 tq_status launch_decode_d64(int kb, int vb, const DecodeParams& p, const QPrepParams& qp,
-                            const MergeParams& m, const DecodePlan& plan, int64_t steps_upper,
-                            cudaStream_t st);
+                            const MergeParams& m, const DecodePlan& plan,
+                            const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st);
 tq_status launch_decode_d128(int kb, int vb, const DecodeParams& p, const QPrepParams& qp,
-                             const MergeParams& m, const DecodePlan& plan, int64_t steps_upper,
-                             cudaStream_t st);
+                             const MergeParams& m, const DecodePlan& plan,
+                             const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st);
 tq_status launch_decode_d256(int kb, int vb, const DecodeParams& p, const QPrepParams& qp,
-                             const MergeParams& m, const DecodePlan& plan, int64_t steps_upper,
-                             cudaStream_t st);
+                             const MergeParams& m, const DecodePlan& plan,
+                             const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st);
 
 // (K bits, V bits) pairs with a compiled decode kernel.
 inline bool decode_bits_supported(int kb, int vb) {
@@ -58,7 +58,7 @@ inline bool decode_bits_supported(int kb, int vb) {
 
 template <int D, int KB, int VB, int NH>
 tq_status launch_decode_t(DecodeParams p, QPrepParams qp, MergeParams m, const DecodePlan& plan,
-                          int64_t steps_upper, cudaStream_t st) {
+                          const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st) {
   auto kern = decode_kernel<D, KB, VB, NH>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem) !=
       cudaSuccess)
@@ -80,7 +80,7 @@ tq_status launch_decode_t(DecodeParams p, QPrepParams qp, MergeParams m, const D
   qprep_kernel<D, KB><<<(qrows + 7) / 8, 256, 0, st>>>(qp, qrows);
   tq_status s = launch_status();
   if (s != TQ_OK) return s;
-  kern<<<(unsigned)ctas, threads, plan.smem, st>>>(p);
+  kern<<<(unsigned)ctas, threads, plan.smem, st>>>(p, tmap);
   s = launch_status();
   if (s != TQ_OK) return s;
   merge_kernel<D><<<dim3(p.h_q, p.batch), 256, 0, st>>>(m);
@@ -89,18 +89,19 @@ tq_status launch_decode_t(DecodeParams p, QPrepParams qp, MergeParams m, const D
 
 template <int D, int KB, int VB>
 tq_status launch_decode_bits(const DecodeParams& p, const QPrepParams& qp, const MergeParams& m,
-                             const DecodePlan& plan, int64_t steps_upper, cudaStream_t st) {
-  return p.group > 8 ? launch_decode_t<D, KB, VB, 2>(p, qp, m, plan, steps_upper, st)
-                     : launch_decode_t<D, KB, VB, 1>(p, qp, m, plan, steps_upper, st);
+                             const DecodePlan& plan, const CUtensorMap& tmap,
+                             int64_t steps_upper, cudaStream_t st) {
+  return p.group > 8 ? launch_decode_t<D, KB, VB, 2>(p, qp, m, plan, tmap, steps_upper, st)
+                     : launch_decode_t<D, KB, VB, 1>(p, qp, m, plan, tmap, steps_upper, st);
 }
 
 template <int D>
 tq_status launch_decode_dim(int kb, int vb, const DecodeParams& p, const QPrepParams& qp,
-                            const MergeParams& m, const DecodePlan& plan, int64_t steps_upper,
-                            cudaStream_t st) {
+                            const MergeParams& m, const DecodePlan& plan,
+                            const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st) {
 #define TQ_BITS_CASE(KB_, VB_) \
   if (kb == KB_ && vb == VB_)  \
-    return launch_decode_bits<D, KB_, VB_>(p, qp, m, plan, steps_upper, st);
+    return launch_decode_bits<D, KB_, VB_>(p, qp, m, plan, tmap, steps_upper, st);
   TQ_BITS_CASE(2, 2)
   TQ_BITS_CASE(3, 3)
   TQ_BITS_CASE(4, 4)
