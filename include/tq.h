@@ -89,6 +89,8 @@ typedef enum {
 #define TQ_DEVERR_NONFINITE 0x4     /* a K/V input row held a NaN or an infinity   */
 #define TQ_DEVERR_SEQLEN_RANGE 0x8  /* seq_len < 0 or > max_blocks*block_size      */
 #define TQ_DEVERR_TIMEOUT 0x10      /* a bounded wait inside a kernel gave up        */
+#define TQ_DEVERR_LAYOUT 0x20       /* the decode kernel's shared-memory layout did not
+                                       match its launch; the launch did nothing      */
 
 /* A strided view of a device array.  Strides are in ELEMENTS; shape[i] and
  * stride[i] for i >= ndim are ignored.  data must be aligned to the element size. */
@@ -160,6 +162,8 @@ TQ_API tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_
  *                TQ_DEVERR_SEQLEN_RANGE and the sequence gives 0.
  *   scale        softmax scale (typically 1/sqrt(D)).
  * H_q must be a multiple of H_kv with H_q / H_kv <= 16; block_size must be 16.
+ * One cooperative kernel launch: the CTAs that share a sequence wait for one another
+ * (bounded; TQ_DEVERR_TIMEOUT) before merging its partial results.
  * Uses the per-device workspace (tq_set_workspace, or allocated by the library on
  * the first call that needs more, and kept until process exit).
  * Errors: TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED / TQ_ERR_WORKSPACE (nothing
@@ -187,9 +191,9 @@ TQ_API tq_status tq_paged_decode(tq_tensor out, tq_tensor q, tq_tensor pages,
  *   - A geometry whose scratch would exceed TQ_NOALLOC_SCRATCH_BYTES (see
  *     tq_decode_workspace_size for the size) is rejected with TQ_ERR_WORKSPACE and
  *     nothing is enqueued.
- *   - Every call on a device shares the one array, and it keeps whatever the last
- *     call left there (no call needs it zeroed).  Calls whose kernels overlap on the
- *     GPU (different streams without ordering) race on it: order them. */
+ *   - Every call on a device shares the one array.  It starts zeroed and every
+ *     call leaves its merge counters at zero again.  Calls whose kernels overlap on
+ *     the GPU (different streams without ordering) race on it: order them. */
 #define TQ_NOALLOC_SCRATCH_BYTES (16u << 20)
 TQ_API tq_status tq_paged_decode_noalloc(tq_tensor out, tq_tensor q, tq_tensor pages,
                                          tq_tensor block_table, tq_tensor seq_lens,
@@ -197,19 +201,24 @@ TQ_API tq_status tq_paged_decode_noalloc(tq_tensor out, tq_tensor q, tq_tensor p
                                          void* stream);
 
 /* Workspace bytes tq_paged_decode needs for this geometry (host only).  The
- * workspace holds the split-KV partial results (m, l, O') in fp32. */
+ * workspace holds 2 * batch u32 merge counters at its start (zero between calls:
+ * each call clears the ones it raised) and the split-KV partial results (m, l, O')
+ * in fp32. */
 TQ_API tq_status tq_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                                    int32_t head_dim, int32_t max_blocks, int32_t block_size,
                                    size_t* bytes);
 
 /* Give the library a caller-owned device workspace for the CURRENT device
- * (ptr 256-byte aligned; NULL releases the association).  The library never frees
- * it.  Calls that use one device's workspace must be ordered on the GPU (one stream,
- * or events); concurrent decodes on one device race on it. */
+ * (ptr 256-byte aligned; NULL releases the association).  The library zeroes it
+ * here (cudaMemset, synchronous) and never frees it; the caller must not write to
+ * it while it is set.  Calls that use one device's workspace must be ordered on the
+ * GPU (one stream, or events); concurrent decodes on one device race on it. */
 TQ_API tq_status tq_set_workspace(void* ptr, size_t bytes);
 
 /* Read and clear the current device's error word (TQ_DEVERR_* bits).  Host
- * pointer `out`; synchronises `stream` first. */
+ * pointer `out`; synchronises `stream` first.  When the word is non-zero it also
+ * clears the merge counters of the device's workspaces, which a failed decode may
+ * have left raised. */
 TQ_API tq_status tq_get_device_error(int32_t* out, void* stream);
 
 /* Test export of the rotation used by tq_quantize_append: for each row x of

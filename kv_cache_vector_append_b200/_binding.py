@@ -22,6 +22,8 @@ DEVERR_SLOT_RANGE = 0x1
 DEVERR_BLOCK_RANGE = 0x2
 DEVERR_NONFINITE = 0x4
 DEVERR_SEQLEN_RANGE = 0x8
+DEVERR_TIMEOUT = 0x10
+DEVERR_LAYOUT = 0x20
 
 EXPORTED = ("tq_slot_bytes", "tq_quantize_append", "tq_paged_decode", "tq_paged_decode_noalloc",
             "tq_decode_workspace_size", "tq_set_workspace", "tq_get_device_error",

@@ -21,6 +21,15 @@ __device__ unsigned int g_tq_error_word;
 // per device with cudaGetSymbolAddress.
 static __device__ __align__(256) uint8_t g_tq_noalloc_scratch[TQ_NOALLOC_SCRATCH_BYTES];
 
+__device__ unsigned int g_tq_dyn_base;
+
+// Records where dynamic shared memory starts in the shared window of a kernel that
+// has no static shared memory (the decode kernel's layout is planned against it).
+__global__ void dyn_smem_base_probe() {
+  extern __shared__ __align__(16) uint8_t smem[];
+  g_tq_dyn_base = (unsigned int)__cvta_generic_to_shared(smem);
+}
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -32,6 +41,7 @@ struct DeviceState {
   void* lib_ws = nullptr;
   size_t lib_ws_bytes = 0;
   uint8_t* noalloc_scratch = nullptr;   // device address of g_tq_noalloc_scratch
+  size_t counter_bytes = 0;             // largest merge-counter area a decode call used
   DeviceInfo info;
 };
 
@@ -50,6 +60,12 @@ tq_status device_state(DeviceState** out) {
     if (cudaDeviceGetAttribute(&s.info.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
         cudaSuccess)
       return TQ_ERR_CUDA;
+    dyn_smem_base_probe<<<1, 1, 16>>>();
+    unsigned int base = 0;
+    if (cudaGetLastError() != cudaSuccess ||
+        cudaMemcpyFromSymbol(&base, g_tq_dyn_base, sizeof(base)) != cudaSuccess)
+      return TQ_ERR_CUDA;
+    s.info.dyn_smem_base = base;
     s.err = (unsigned int*)p;
   }
   *out = &s;
@@ -102,11 +118,18 @@ int align_mode_of(const void* data, int esize, std::initializer_list<int64_t> st
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Geometry of the decode kernels for one call (see tq_decode.cuh).
+int pow2_floor(int x) {
+  int r = 1;
+  while (2 * r <= x) r *= 2;
+  return r;
+}
+
+// Geometry of the decode kernel for one call (see tq_decode.cuh).
 tq_status plan_decode(int batch, int h_q, int h_kv, int dim, int kb, int vb, int slot_stride,
-                      int max_blocks, bool shared_lut, bool allow_tensor_copy, const DeviceInfo& di,
+                      int max_blocks, bool allow_tensor_copy, const DeviceInfo& di,
                       DecodePlan* plan) {
-  if (h_kv < 1 || h_kv > kDecodeWarps) return TQ_ERR_UNSUPPORTED;
+  plan->maxw = decode_maxw(dim, h_q / h_kv);
+  if (h_kv < 1 || h_kv > plan->maxw) return TQ_ERR_UNSUPPORTED;
   // A block is staged by one TMA copy.  When a row is a multiple of 16 bytes and the
   // padded row fits a tensor box (at most 256 u64 columns), the copy is a 2-D box of
   // 16 rows x pitch/8 u64 whose columns past the row end are zero-filled, giving rows
@@ -117,30 +140,76 @@ tq_status plan_decode(int batch, int h_q, int h_kv, int dim, int kb, int vb, int
   words += ((20 - words % 32) + 32) % 32;
   plan->copy_mode = allow_tensor_copy && row_bytes % 16 == 0 && 4 * words / 8 <= 256;
   plan->row_pitch = plan->copy_mode ? 4 * words : row_bytes;
-  plan->shared_lut = shared_lut && kb == vb;
-  const size_t lut = decode_lut_bytes(kb, vb, plan->shared_lut);
-  // at most 4 blocks per step, so that one warp issues a step's row copies in two rounds
-  plan->wph = std::min(kDecodeWarps / h_kv, 4);
-  for (;;) {
-    plan->stage_bytes = plan->wph * kBlockSize * plan->row_pitch;
-    // block ids a CTA preloads: its whole step range when the grid is full
-    const int64_t steps_upper = (int64_t)batch * ((max_blocks + plan->wph - 1) / plan->wph);
-    const int64_t per_cta = (steps_upper + 2 * di.num_sms - 1) / (2 * di.num_sms) + 1;
-    plan->ids_cap = (int)std::min<int64_t>(per_cta * plan->wph, 4096);
-    plan->smem = lut + 128 + (size_t)kDecodeStages * plan->stage_bytes + kDecodeStages * 16 +
-                 4 * ((size_t)batch + 1) + 4 * ((1 << kb) + (1 << vb)) + 4 * plan->ids_cap + 16;
-    if ((int)plan->smem <= di.max_smem_optin || plan->wph == 1) break;
-    plan->wph /= 2;
+  plan->lut_bytes = (int)decode_lut_bytes(kb, vb);
+  plan->max_ctas = di.num_sms;
+  const int wph_max = pow2_floor(plan->maxw / h_kv);
+  // The dynamic shared memory spans shared-window addresses [base, base + budget).  The
+  // tables go to a multiple of 65536 inside it; the stages fill the space below and
+  // above them; the misc area (barriers, q', prefix sums, block ids, merge partials)
+  // goes at the bottom or at the top, whichever leaves more stages.
+  const int64_t base = di.dyn_smem_base;
+  const int64_t budget = (int64_t)di.max_smem_optin;
+  const int64_t lut = plan->lut_bytes;
+  bool found = false;
+  for (int wph = wph_max; wph >= 1 && !found; wph /= 2) {
+    const int64_t stage = (int64_t)wph * kBlockSize * plan->row_pitch;
+    const int64_t steps_upper = (int64_t)batch * ((max_blocks + wph - 1) / wph);
+    const int64_t per_cta = (steps_upper + di.num_sms - 1) / di.num_sms + 1;
+    const int ids_cap = (int)std::min<int64_t>(per_cta * wph, 4096);
+    const int min_st = wph == 1 ? 2 : 4;
+    int best_nst = 0;
+    int64_t best_end = 0;
+    DecodePlan best;
+    for (int64_t L = 65536; L + lut <= base + budget; L += 65536) {
+      if (L < base) continue;
+      const int64_t low = L - base, high = base + budget - (L + lut);
+      for (int nst = kMaxStages; nst >= min_st; --nst) {
+        const int64_t misc = 16 * nst + 2LL * h_q * dim + 4LL * h_q + 4LL * (batch + 1) +
+                             4LL * ids_cap + 4 * 36 + (int64_t)plan->maxw * (dim + 2) * 4 + 16;
+        for (int at_top = 0; at_top < 2; ++at_top) {
+          const int64_t below = at_top ? low : low - misc;   // room for stages below
+          if (below < 0) continue;
+          const int nl = (int)std::min<int64_t>(nst, below / stage);
+          const int nh = nst - nl;
+          const int64_t hi_off = (L - base) + lut;
+          const int64_t misc_off = at_top ? (hi_off + nh * stage + 15) / 16 * 16 : 0;
+          const int64_t end = at_top ? misc_off + misc : (nh > 0 ? hi_off + nh * stage : hi_off);
+          if (end > budget) continue;
+          if (nst > best_nst || (nst == best_nst && end < best_end)) {
+            best_nst = nst;
+            best_end = end;
+            best.lut_win = (uint32_t)L;
+            best.lut_off = (int)(L - base);
+            best.stage_lo_off = (int)(L - base - nl * stage);
+            best.stage_hi_off = (int)hi_off;
+            best.n_low = nl;
+            best.misc_off = (int)misc_off;
+          }
+        }
+        if (best_nst == nst) break;        // the deepest ring this L allows
+      }
+    }
+    if (best_nst > 0) {
+      plan->wph = wph;
+      plan->nst = best_nst;
+      plan->stage_bytes = (int)stage;
+      plan->ids_cap = ids_cap;
+      plan->smem = (size_t)best_end;
+      plan->lut_win = best.lut_win;
+      plan->lut_off = best.lut_off;
+      plan->stage_lo_off = best.stage_lo_off;
+      plan->stage_hi_off = best.stage_hi_off;
+      plan->n_low = best.n_low;
+      plan->misc_off = best.misc_off;
+      found = true;
+    }
   }
-  if ((int)plan->smem > di.max_smem_optin) return TQ_ERR_UNSUPPORTED;
-  plan->max_ctas = 2 * di.num_sms;
-  // workspace: rotated queries, their scales, step prefix sums, partial records
-  plan->qfrag_off = 0;
-  plan->qscale_off = align256((size_t)batch * h_q * dim * 2);
-  plan->prefix_off = plan->qscale_off + align256((size_t)batch * h_q * 4);
-  plan->part_off = plan->prefix_off + align256(((size_t)batch + 1) * 4);
-  plan->ws_bytes = plan->part_off + (size_t)(plan->max_ctas + batch) *
-                                        std::min(kDecodeWarps / h_kv, 4) * h_q * (dim + 2) *
+  if (!found) return TQ_ERR_UNSUPPORTED;
+  // workspace: merge counters (at the start, so that they can be cleared without
+  // knowing a call's geometry), then the partial records (sized for the widest step)
+  plan->counters_off = 0;
+  plan->part_off = align256((size_t)batch * 2 * sizeof(unsigned int));
+  plan->ws_bytes = plan->part_off + (size_t)(plan->max_ctas + batch) * wph_max * h_q * (dim + 2) *
                                         sizeof(float);
   return TQ_OK;
 }
@@ -217,7 +286,7 @@ tq_status decode_prepare(const tq_tensor& out, const tq_tensor& q, const tq_tens
     return TQ_ERR_INVALID_ARG;
   if (pages.shape[1] != kBlockSize) return TQ_ERR_UNSUPPORTED;
   if (D != 64 && D != 128 && D != 256) return TQ_ERR_UNSUPPORTED;
-  if (h_q / h_kv > 16 || h_kv > kDecodeWarps) return TQ_ERR_UNSUPPORTED;
+  if (h_q / h_kv > 16 || h_kv > decode_maxw(D, h_q / h_kv)) return TQ_ERR_UNSUPPORTED;
   if (!decode_bits_supported(kbits, vbits)) return TQ_ERR_UNSUPPORTED;
   call->B = B;
   if (B == 0) return TQ_OK;
@@ -225,10 +294,9 @@ tq_status decode_prepare(const tq_tensor& out, const tq_tensor& q, const tq_tens
   tq_status s = device_state(&ds);
   if (s != TQ_OK) return s;
   const int max_blocks = (int)block_table.shape[1];
-  const bool shared_lut = cb->k.bits == cb->v.bits && cb->k.centroids == cb->v.centroids;
   DecodePlan plan;
-  s = plan_decode(B, h_q, h_kv, D, kbits, vbits, (int)stride, std::max(max_blocks, 1), shared_lut,
-                  true, ds->info, &plan);
+  s = plan_decode(B, h_q, h_kv, D, kbits, vbits, (int)stride, std::max(max_blocks, 1), true,
+                  ds->info, &plan);
   if (s != TQ_OK) return s;
   if ((h_kv * stride) % 8) return TQ_ERR_INVALID_ARG;
   call->h_q = h_q;
@@ -261,20 +329,9 @@ tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tens
       !encode_page_map(&tmap, pages.data, pages.shape[0], h_kv * (int)stride, plan.row_pitch)) {
     // the 1-D bulk layout never needs more shared memory or workspace than the 2-D one
     const tq_status s = plan_decode(B, h_q, h_kv, D, kbits, vbits, (int)stride,
-                                    std::max(max_blocks, 1), plan.shared_lut, false, ds->info, &plan);
+                                    std::max(max_blocks, 1), false, ds->info, &plan);
     if (s != TQ_OK) return s;
   }
-  QPrepParams qp{};
-  qp.q = q.data;
-  qp.q_bstride = q.stride[0];
-  qp.q_hstride = q.stride[1];
-  qp.q_dtype = q.dtype;
-  qp.h_q = h_q;
-  qp.scale_log2 = scale * 1.4426950408889634f;
-  qp.sign_seed = sign_seed;
-  qp.qfrag = (uint32_t*)(ws + plan.qfrag_off);
-  qp.qscale = (float*)(ws + plan.qscale_off);
-
   DecodeParams p{};
   p.pages = (const uint8_t*)pages.data;
   p.num_blocks = (int32_t)pages.shape[0];
@@ -287,40 +344,48 @@ tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tens
   p.max_blocks = max_blocks;
   p.seq_lens = (const int32_t*)seq_lens.data;
   p.batch = B;
+  p.q = q.data;
+  p.q_bstride = q.stride[0];
+  p.q_hstride = q.stride[1];
+  p.q_dtype = q.dtype;
+  p.out = out.data;
+  p.o_bstride = out.stride[0];
+  p.o_hstride = out.stride[1];
+  p.out_dtype = out.dtype;
   p.h_q = h_q;
   p.group = h_q / h_kv;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.sign_seed = sign_seed;
   p.kc = cb->k.centroids;
   p.vc = cb->v.centroids;
-  p.shared_lut = plan.shared_lut;
   p.k_region = kb;
   p.wph = plan.wph;
+  p.nst = plan.nst;
   p.stage_bytes = plan.stage_bytes;
   p.ids_cap = plan.ids_cap;
   p.copy_mode = plan.copy_mode;
-  p.qfrag = qp.qfrag;
-  p.qscale = qp.qscale;
-  p.prefix = (int32_t*)(ws + plan.prefix_off);
+  p.lut_bytes = plan.lut_bytes;
+  p.lut_win = plan.lut_win;
+  p.lut_off = plan.lut_off;
+  p.stage_lo_off = plan.stage_lo_off;
+  p.stage_hi_off = plan.stage_hi_off;
+  p.n_low = plan.n_low;
+  p.misc_off = plan.misc_off;
+  p.smem_end = (int32_t)plan.smem;
   p.part = (float*)(ws + plan.part_off);
+  p.counters = (unsigned int*)(ws + plan.counters_off);
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    ds->counter_bytes = std::max(ds->counter_bytes, plan.part_off);
+  }
   p.err = ds->err;
 
-  MergeParams m{};
-  m.part = p.part;
-  m.prefix = p.prefix;
-  m.out = out.data;
-  m.o_bstride = out.stride[0];
-  m.o_hstride = out.stride[1];
-  m.out_dtype = out.dtype;
-  m.h_q = h_q;
-  m.wph = plan.wph;
-  m.sign_seed = sign_seed;
-
-  const int64_t per_step = plan.wph;
-  const int64_t steps_upper = (int64_t)B * ((max_blocks + per_step - 1) / per_step);
+  const int64_t steps_upper = (int64_t)B * ((max_blocks + plan.wph - 1) / plan.wph);
   cudaStream_t st = as_stream(stream);
   switch (D) {
-    case 64: return launch_decode_d64(kbits, vbits, p, qp, m, plan, tmap, steps_upper, st);
-    case 128: return launch_decode_d128(kbits, vbits, p, qp, m, plan, tmap, steps_upper, st);
-    default: return launch_decode_d256(kbits, vbits, p, qp, m, plan, tmap, steps_upper, st);
+    case 64: return launch_decode_d64(kbits, vbits, p, plan, tmap, steps_upper, st);
+    case 128: return launch_decode_d128(kbits, vbits, p, plan, tmap, steps_upper, st);
+    default: return launch_decode_d256(kbits, vbits, p, plan, tmap, steps_upper, st);
   }
 }
 
@@ -462,8 +527,8 @@ tq_status tq_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t n
   // the record area is sized for the largest warps-per-head count, so any bit widths fit
   DecodePlan plan;
   s = plan_decode(std::max(batch, 1), num_q_heads, num_kv_heads, head_dim, 1, 1,
-                  region_bytes(head_dim, 1) * 2 + 8, std::max(max_blocks, 1), false, false,
-                  ds->info, &plan);
+                  region_bytes(head_dim, 1) * 2 + 8, std::max(max_blocks, 1), false, ds->info,
+                  &plan);
   if (s != TQ_OK) return s;
   *bytes = plan.ws_bytes;
   return TQ_OK;
@@ -474,6 +539,8 @@ tq_status tq_set_workspace(void* ptr, size_t bytes) {
   tq_status s = device_state(&ds);
   if (s != TQ_OK) return s;
   if (ptr != nullptr && (uintptr_t)ptr % 256) return TQ_ERR_INVALID_ARG;
+  // the merge counters at the start of a workspace must read zero before first use
+  if (ptr != nullptr && cudaMemset(ptr, 0, bytes) != cudaSuccess) return TQ_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);
   ds->user_ws = ptr;
   ds->user_ws_bytes = ptr ? bytes : 0;
@@ -491,6 +558,22 @@ tq_status tq_get_device_error(int32_t* out, void* stream) {
     return TQ_ERR_CUDA;
   if (cudaMemsetAsync(ds->err, 0, sizeof(unsigned int), st) != cudaSuccess) return TQ_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return TQ_ERR_CUDA;
+  if (h != 0) {
+    // a launch that reported an error may have stopped with merge counters raised:
+    // clear the counter areas of this device's workspaces
+    std::lock_guard<std::mutex> lock(g_mu);
+    const size_t n = ds->counter_bytes;
+    if (n > 0) {
+      if (ds->user_ws && cudaMemset(ds->user_ws, 0, std::min(n, ds->user_ws_bytes)) != cudaSuccess)
+        return TQ_ERR_CUDA;
+      if (ds->lib_ws && cudaMemset(ds->lib_ws, 0, std::min(n, ds->lib_ws_bytes)) != cudaSuccess)
+        return TQ_ERR_CUDA;
+      if (ds->noalloc_scratch &&
+          cudaMemset(ds->noalloc_scratch, 0, std::min<size_t>(n, TQ_NOALLOC_SCRATCH_BYTES)) !=
+              cudaSuccess)
+        return TQ_ERR_CUDA;
+    }
+  }
   *out = (int32_t)h;
   return TQ_OK;
 }
@@ -516,6 +599,7 @@ tq_status tq_paged_decode(tq_tensor out, tq_tensor q, tq_tensor pages, tq_tensor
         ds->lib_ws_bytes = 0;
         size_t want = std::max<size_t>(plan.ws_bytes, 1 << 20);
         if (cudaMalloc(&ds->lib_ws, want) != cudaSuccess) return TQ_ERR_WORKSPACE;
+        if (cudaMemset(ds->lib_ws, 0, want) != cudaSuccess) return TQ_ERR_CUDA;
         ds->lib_ws_bytes = want;
       }
       ws = (uint8_t*)ds->lib_ws;
@@ -546,9 +630,9 @@ tq_status tq_paged_decode_noalloc(tq_tensor out, tq_tensor q, tq_tensor pages,
     }
     ws = ds->noalloc_scratch;
   }
-  // Nothing in the scratch has to start at zero: every byte a launch reads (rotated
-  // queries, prefix sums, partial records) is written earlier in the same launch
-  // sequence, so the contents left by a previous call do no harm.
+  // The scratch starts zeroed (a static device array) and every call leaves its merge
+  // counters at zero; the partial records a launch reads are written earlier in the
+  // same launch.
   return decode_run(call, out, q, pages, block_table, seq_lens, cb, sign_seed, scale, ws, stream);
 }
 

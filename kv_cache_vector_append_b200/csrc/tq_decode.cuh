@@ -10,22 +10,27 @@
 // Math.  With R the rotation, k_hat_t = nK_t R^T cK[idx_t] and v_hat_t = nV_t R^T cV[.]:
 //   <q, k_hat_t> = nK_t <R q, cK[idx_t]>            (score on the codes)
 //   sum_t p_t v_hat_t = R^T sum_t p_t nV_t cV[.]       (V in the rotated domain)
-// so q is rotated once, and the output is rotated back once (merge kernel).
+// so q is rotated once per sequence, and the output is rotated back once.
 //
-// Kernel layout.  A prep kernel rotates every query once.  The decode kernel is
-// persistent: the (sequence, pair of blocks) steps of the whole batch are laid end
-// to end and CTA c takes the equal contiguous range [c S/C, (c+1) S/C) of the S
-// steps (stream-K style), so ragged batches and single long sequences balance
-// alike.  Inside a CTA one warp serves one (KV head, sub-stream):
+// Kernel layout.  One persistent kernel per call, one CTA per SM.  The (sequence,
+// group of wph blocks) steps of the whole batch are laid end to end and CTA c takes
+// the contiguous range [c S/C, (c+1) S/C) of the S steps (stream-K style), so ragged
+// batches and single long sequences balance alike.  Inside a CTA one warp serves one
+// (KV head, sub-stream):
+//   * when its range enters a sequence the CTA rotates that sequence's queries (sign
+//     flips, FWHT in registers and shuffles, 1/sqrt(D)) into shared memory as unit
+//     fp16 vectors plus |q'| * scale * log2 e;
 //   * page blocks (16 tokens x all KV heads; one per sub-stream and step) are staged
-//     into shared memory by one TMA tensor copy each (a 16-row box one padding wider
-//     than a row, the padding zero-filled out of bounds) into a 4-deep ring of stages
-//     guarded by mbarriers; the last warp to release a stage refills it, so no warp
-//     ever waits for the whole CTA; the padded pitch of 20 (mod 32) words makes the
-//     per-thread code loads below bank-conflict free;
-//   * codes become fp16 through per-lane replicated lookup tables of code PAIRS
-//     (bits <= 4: entry (x | y << bits) = (c[x], c[y])) or single codes, so that
-//     the 32 lanes of a warp always hit 32 different banks;
+//     into shared memory by one TMA copy each (a 2-D box of 16 rows one padding wider
+//     than a row, the padding zero-filled out of bounds, or a 1-D bulk copy) into a
+//     ring of stages guarded by mbarriers; the last warp to release a stage refills
+//     it, so no warp waits for the whole CTA; the padded pitch of 20 (mod 32) words
+//     makes the per-thread code loads bank-conflict free;
+//   * codes become fp16 through shared-memory tables with one 256-byte row per entry
+//     (the K table in the first 128 bytes of a row, the V table in the second, lane l
+//     at byte 4l), so a warp's lookups always hit 32 different banks and the address of
+//     a lookup keyed by a whole byte of codes is one byte permute; tables hold code
+//     PAIRS for bits <= 4 (entry x | y << bits = (c[x], c[y])), single codes for 8 bits;
 //   * S^T = K~ . Qhat^T on mma.sync m16n8k16 (M = 16 tokens, N = 8 query heads of the
 //     group, K = D; fp16 operands, fp32 accumulation); s = acc * nK * |q'| * scale * log2 e;
 //   * online softmax in base 2 against a running reference M >= max(s + e(nV)),
@@ -35,13 +40,15 @@
 //   * O'^T += V~^T . P~^T on mma.sync (M = coordinates, N = query heads, K = tokens);
 //     the fp16 weights go from the C layout of S^T to the B layout of P~^T with one
 //     movmatrix transpose per 8 x 8 tile;
-//   * at every sequence boundary of its range a warp writes its partial (M, l, O')
-//     to record (CTA + sequence), an index no other (CTA, sequence) pair shares
-//     because the ranges are monotone; the merge kernel combines the records of a
-//     sequence, divides by l and applies the inverse rotation.
+//   * when its range leaves a sequence every warp writes its partial (M, l, O') to
+//     record ((CTA + sequence) * wph + sub-stream), an index no other (CTA, sequence)
+//     pair shares because the ranges are monotone; the CTA then takes a ticket on the
+//     sequence's counter, and the CTA holding the last ticket combines the records of
+//     the sequence, divides by l and applies the inverse rotation, while the others
+//     move on.
 // The coordinate order inside each mma tile is free (a permutation applied to both
 // operands of a contraction leaves it unchanged); it is chosen so that every thread
-// reads whole 32-bit words of codes, and undone when O' is written out.
+// reads whole 32-bit words of codes, and undone when O' is written to its record.
 #pragma once
 
 #include "tq_device.cuh"
@@ -49,62 +56,58 @@
 namespace tq {
 
 constexpr int kBlockSize = 16;        // tokens per page block
-constexpr int kDecodeWarps = 8;
-constexpr int kDecodeStages = 4;
-constexpr uint32_t kWaitLimit = 2000;      // polls (each <= ~1 ms) before a wait gives up
+constexpr int kMaxStages = 8;         // deepest stage ring
+constexpr uint32_t kWaitMs = 2000;    // a stage wait gives up after about 2 s
 constexpr float kLazyRescale = 8.0f;  // log2 units
+constexpr int kLutRow = 256;          // bytes per table entry (K half, V half)
 
 struct DecodeParams {
   const uint8_t* pages;
   int32_t num_blocks;
   int32_t h_kv;
   int32_t slot_stride;          // bytes between heads inside a row
-  int32_t row_pitch;            // bytes between rows in shared memory (padded)
+  int32_t row_pitch;            // bytes between rows in shared memory
   int64_t blk_stride;           // bytes between blocks in global memory
   const int32_t* block_table;
   int64_t bt_stride;            // elements between sequences
   int32_t max_blocks;
   const int32_t* seq_lens;
   int32_t batch;
+  const void* q;                // [B, H_q, D]
+  int64_t q_bstride, q_hstride; // elements
+  int32_t q_dtype;
+  void* out;                    // [B, H_q, D]
+  int64_t o_bstride, o_hstride; // elements
+  int32_t out_dtype;
   int32_t h_q;
   int32_t group;                // G = H_q / H_kv
+  float scale_log2;             // softmax scale * log2(e)
+  uint64_t sign_seed;
   const float* kc;              // K centroids
   const float* vc;              // V centroids
-  int32_t shared_lut;           // K and V tables identical (one LUT)
-  int32_t k_region;             // bytes of the K region (offset of V region)
+  int32_t k_region;             // bytes of the K region (offset of the V region)
   int32_t wph;                  // warps (sub-streams) per KV head = blocks per step
+  int32_t nst;                  // stages in the ring (<= kMaxStages)
   int32_t stage_bytes;
   int32_t ids_cap;              // block ids of its step range a CTA preloads (entries)
   int32_t copy_mode;            // 1: 2-D tensor box per block (rows padded to row_pitch)
                                 // 0: 1-D bulk copy per block (row_pitch = row bytes)
-  const uint32_t* qfrag;        // [B][H_q][4 tig][KSTEPS][2] half2, from qprep_kernel
-  const float* qscale;          // [B][H_q]: |q'| * scale * log2(e)
-  int32_t* prefix;              // [B + 1] step prefix sums (written by CTA 0)
-  float* part;                  // records [(C + B)][wph][H_q][D + 2]
+  int32_t lut_bytes;            // bytes of the lookup tables
+  // Dynamic shared memory layout (byte offsets from its start).  The tables sit at
+  // shared-window address lut_win, a multiple of 65536, so that the address of a table
+  // entry is (lut_win | e << 8 | column) with no addition; stages 0 .. n_low-1 lie
+  // below the tables, the others above them.
+  uint32_t lut_win;
+  int32_t lut_off;
+  int32_t stage_lo_off;
+  int32_t stage_hi_off;
+  int32_t n_low;
+  int32_t misc_off;             // barriers, q', prefix sums, block ids, merge scratch
+  int32_t smem_end;             // bytes of dynamic shared memory the layout spans
+  float* part;                  // records [(C + B) * wph][H_q][D + 2]
+  unsigned int* counters;       // [2][B]: records written, merges done (per sequence);
+                                // zero between calls (the last user of a counter clears it)
   unsigned int* err;
-};
-
-struct QPrepParams {
-  const void* q;                // [B, H_q, D]
-  int64_t q_bstride, q_hstride; // elements
-  int32_t q_dtype;
-  int32_t h_q;
-  float scale_log2;             // scale * log2(e)
-  uint64_t sign_seed;
-  uint32_t* qfrag;
-  float* qscale;
-};
-
-struct MergeParams {
-  const float* part;
-  const int32_t* prefix;
-  void* out;
-  int64_t o_bstride, o_hstride;
-  int32_t out_dtype;
-  int32_t h_q;
-  int32_t wph;
-  int32_t nctas;
-  uint64_t sign_seed;
 };
 
 // Step range of CTA c out of C over S steps: [floor(c S / C), floor((c+1) S / C)).
@@ -128,8 +131,7 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                           uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -203,44 +205,94 @@ struct Share {
   }
 };
 
-// Replicated lookup tables.  Entry e of the table for lane l is the 32-bit word at
-// index (e << 5) | l, so lookups by a warp never conflict.  For BITS <= 4 the
-// table holds code pairs: entry (x | y << BITS) = half2(c[x], c[y]); for BITS > 4
-// it holds single codes: entry x = half2(c[x], c[x]).
-template <int BITS>
-struct RepLut {
-  static constexpr bool kPair = BITS <= 4;
-  static constexpr int kEntries = kPair ? (1 << (2 * BITS)) : (1 << BITS);
-  static constexpr int kBytes = kEntries * 32 * 4;
-  // c: the 2^BITS centroids, already in shared memory
-  static __device__ __forceinline__ void build(uint32_t* lut, const float* c, int tid, int nt) {
-    for (int i = tid; i < kEntries * 32; i += nt) {
-      const int e = i >> 5;
-      if constexpr (kPair) lut[i] = pack_half2(c[e & ((1 << BITS) - 1)], c[e >> BITS]);
-      else lut[i] = pack_half2(c[e], c[e]);
-    }
+// ---------------------------------------------------------------------------
+// Lookup tables.  Entry e of a table is row e (kLutRow bytes) of the table area at
+// the start of dynamic shared memory; lane l reads its copy of the K entry at byte
+// 4l of the row and its copy of the V entry at byte 128 + 4l.  For BITS <= 4 an entry
+// is a code pair: entry (x | y << BITS) = half2(c[x], c[y]); for BITS = 8 it is a
+// single code: entry x = half2(c[x], c[x]).
+// ---------------------------------------------------------------------------
+__host__ __device__ constexpr int lut_entries(int bits) {
+  return bits <= 4 ? 1 << (2 * bits) : 1 << bits;
+}
+
+// lut: the first byte of the tables (shared-window address lut_win)
+template <int BITS, int HALF>
+__device__ __forceinline__ void lut_build(uint8_t* lut, const float* c, int tid, int nt) {
+  constexpr int kEntries = lut_entries(BITS);
+  for (int i = tid; i < kEntries * 32; i += nt) {
+    const int e = i >> 5, l = i & 31;
+    uint32_t v;
+    if constexpr (BITS <= 4) v = pack_half2(c[e & ((1 << BITS) - 1)], c[e >> BITS]);
+    else v = pack_half2(c[e], c[e]);
+    *(uint32_t*)(lut + e * kLutRow + HALF * 128 + 4 * l) = v;
   }
-  // half2 (c[x], c[y]); `lane_lut` = lut + lane
-  static __device__ __forceinline__ uint32_t pair(const uint32_t* lane_lut, uint32_t x,
-                                                  uint32_t y) {
-    if constexpr (kPair) {
-      return lane_lut[(x | (y << BITS)) << 5];
+}
+
+// Shared-window address (e << 8) | off of the entry e held in the field of LEN bits at
+// bit POS of the word array; `off` is lut_win | the lane's column (4 lane, + 128 for
+// the V table).
+template <int POS, int LEN, int NW>
+__device__ __forceinline__ uint32_t lut_addr(const uint32_t (&w)[NW], uint32_t off) {
+  constexpr int wi = POS >> 5, o = POS & 31;
+  constexpr uint32_t m8 = ((1u << LEN) - 1u) << 8;
+  if constexpr (o + LEN <= 32) {
+    const uint32_t v = w[wi];
+    if constexpr (LEN == 8 && o % 8 == 0) {
+      // byte 1 <- byte o/8 of v; bytes 0, 2, 3 <- those of off (its byte 1 is 0)
+      return __byte_perm(v, off, 0x7604u | ((uint32_t)(o / 8) << 4));
+    } else if constexpr (o >= 8) {
+      return ((v >> (o - 8)) & m8) | off;
     } else {
-      const uint32_t lo = lane_lut[x << 5], hi = lane_lut[y << 5];
-      return __byte_perm(lo, hi, 0x7610);   // low half of lo, high half of hi
+      return ((v << (8 - o)) & m8) | off;
     }
+  } else {
+    const uint32_t f = (w[wi] >> o) | (w[wi + 1] << (32 - o));
+    return ((f << 8) & m8) | off;
   }
-  // pair packed in one 2*BITS field (x in the low bits)
-  static __device__ __forceinline__ uint32_t pair_field(const uint32_t* lane_lut, uint32_t f) {
-    if constexpr (kPair) return lane_lut[f << 5];
-    else return pair(lane_lut, f & ((1u << BITS) - 1u), f >> BITS);
+}
+template <int POS, int LEN>
+__device__ __forceinline__ uint32_t lut_addr1(uint32_t w, uint32_t off) {
+  const uint32_t a[1] = {w};
+  return lut_addr<POS, LEN, 1>(a, off);
+}
+// Table word at shared-window address addr.
+__device__ __forceinline__ uint32_t lut_ld(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// half2 (c[x], c[y]) of the codes x, y of one thread's share (consecutive codes at
+// bit POS of the word array: one pair field, or two 8-bit fields).
+template <int BITS, int POS, int NW>
+__device__ __forceinline__ uint32_t lut_pair(const uint32_t (&w)[NW], uint32_t off) {
+  if constexpr (BITS <= 4) {
+    return lut_ld(lut_addr<POS, 2 * BITS>(w, off));
+  } else {
+    const uint32_t lo = lut_ld(lut_addr<POS, BITS>(w, off));
+    const uint32_t hi = lut_ld(lut_addr<POS + BITS, BITS>(w, off));
+    return __byte_perm(lo, hi, 0x7610);   // low half of lo, high half of hi
   }
-};
+}
+// half2 (c[x], c[y]) with x the code at bit POS of w0 and y the code at bit POS of w1.
+template <int BITS, int POS, int NW>
+__device__ __forceinline__ uint32_t lut_pair2(const uint32_t (&w0)[NW], const uint32_t (&w1)[NW],
+                                              uint32_t off) {
+  if constexpr (BITS <= 4) {
+    const uint32_t x = field<POS, BITS>(w0), y = field<POS, BITS>(w1);
+    return lut_ld(((x | (y << BITS)) << 8) | off);
+  } else {
+    const uint32_t lo = lut_ld(lut_addr<POS, BITS>(w0, off));
+    const uint32_t hi = lut_ld(lut_addr<POS, BITS>(w1, off));
+    return __byte_perm(lo, hi, 0x7610);
+  }
+}
 
 // Transpose of an 8x8 matrix of 16-bit values held in mma fragment layout.
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
   uint32_t d;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
   return d;
 }
 
@@ -252,35 +304,28 @@ struct DecodeCfg {
   static constexpr int MT = D / 16;
   static constexpr int KPACK = D * KB / 8;   // packed bytes (the norm follows)
   static constexpr int VPACK = D * VB / 8;
-  static constexpr int kLutBytes = RepLut<KB>::kBytes + RepLut<VB>::kBytes;
 };
 
-// q' = R q for every (sequence, query head): sign flips, FWHT, 1/sqrt(D); stored as
-// q'/|q'| in fp16, already in the A-fragment order of the score product (thread
-// tig, k-step ks: coords KS::coord(tig, 4ks .. 4ks+3)), and |q'| * scale * log2 e.
-// One warp per (sequence, query head): each lane holds D/32 consecutive coordinates,
-// the FWHT runs in registers and across lanes with shuffles.
-template <int D, int KB>
-__global__ void __launch_bounds__(256)
-qprep_kernel(QPrepParams p, int32_t rows) {
-  using KS = Share<D, KB, 4>;
-  constexpr int E = D / 32;
-  constexpr int NWORDS = D / 2;          // fragment words per head
-  __shared__ float sbuf[8][D];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + warp;   // = b * H_q + h
-  if (row >= rows) return;
-  const int b = row / p.h_q, h = row - b * p.h_q;
-  float x[E];
-  const int64_t off = (int64_t)b * p.q_bstride + (int64_t)h * p.q_hstride + lane * E;
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    float v;
-    if (p.q_dtype == TQ_F32) v = ((const float*)p.q)[off + e];
-    else if (p.q_dtype == TQ_BF16) v = __bfloat162float(((const __nv_bfloat16*)p.q)[off + e]);
-    else v = __half2float(((const __half*)p.q)[off + e]);
-    x[e] = __uint_as_float(__float_as_uint(v) ^ sign_mask_at(p.sign_seed, lane * E + e));
-  }
+// 2^x with the hardware approximation (relative error about 2^-22; results below
+// 2^-126 flush to 0, and 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// floor(log2 x) + 1 for x > 0 (exponent bits; an upper bound of log2 x within 1),
+// -126 for zero or subnormal x, NaN for NaN.
+__device__ __forceinline__ float log2_ceilish(float x) {
+  const uint32_t e = (__float_as_uint(x) >> 23) & 0xFFu;
+  const float f = __uint_as_float(0x4B000000u | e) - 8388608.0f;   // exact small integer
+  return x != x ? x : f - 126.0f;
+}
+
+// In-warp FWHT of D = 32 E values, lane l holding coordinates l E .. l E + E - 1
+// (natural order in and out; no scaling).
+template <int E>
+__device__ __forceinline__ void warp_fwht(float (&x)[E], int lane) {
 #pragma unroll
   for (int hs = 1; hs < E; hs <<= 1)
 #pragma unroll
@@ -297,79 +342,70 @@ qprep_kernel(QPrepParams p, int32_t rows) {
       const float o = __shfl_xor_sync(0xffffffffu, x[i], lm);
       x[i] = (lane & lm) ? o - x[i] : x[i] + o;
     }
-  float ss = 0.f;
-#pragma unroll
-  for (int i = 0; i < E; ++i) {
-    x[i] *= inv_sqrt_dim<D>();
-    ss = fmaf(x[i], x[i], ss);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  const float nrm = sqrtf(ss);
-  const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
-#pragma unroll
-  for (int i = 0; i < E; ++i) sbuf[warp][lane * E + i] = x[i] * inv;
-  __syncwarp();
-  uint32_t* dst = p.qfrag + (int64_t)row * NWORDS;
-  for (int w = lane; w < NWORDS; w += 32) {
-    // word w = (tig, ks, hi): codes 4ks + 2hi, +1 of thread tig's share
-    const int tig = w / (NWORDS / 4), ks = (w / 2) % (D / 16), hi = w & 1;
-    const int m0 = 4 * ks + 2 * hi;
-    int c0, c1;
-    if constexpr (KS::kInterleaved) {
-      c0 = (tig + 4 * (m0 / KS::PW)) * KS::PW + (m0 % KS::PW);
-      c1 = (tig + 4 * ((m0 + 1) / KS::PW)) * KS::PW + ((m0 + 1) % KS::PW);
-    } else {
-      c0 = tig * KS::NCODES + m0;
-      c1 = c0 + 1;
-    }
-    dst[w] = pack_half2(sbuf[warp][c0], sbuf[warp][c1]);
-  }
-  if (lane == 0) p.qscale[row] = nrm * p.scale_log2;
 }
 
-// floor(log2 x) + 1 for x > 0 (exponent bits; an upper bound of log2 x within 1),
-// -126 for zero or subnormal x, NaN for NaN.
-__device__ __forceinline__ float log2_ceilish(float x) {
-  const uint32_t e = (__float_as_uint(x) >> 23) & 0xFFu;
-  const float f = __uint_as_float(0x4B000000u | e) - 8388608.0f;   // exact small integer
-  return x != x ? x : f - 126.0f;
+__device__ __forceinline__ float load_as_f32(const void* base, int64_t i, int32_t dtype) {
+  if (dtype == TQ_F32) return ((const float*)base)[i];
+  if (dtype == TQ_BF16) return __bfloat162float(((const __nv_bfloat16*)base)[i]);
+  return __half2float(((const __half*)base)[i]);
 }
 
-// Shared memory: [K LUT | V LUT | stages | full mbarriers | release counters | prefix |
-// centroids].
-template <int D, int KB, int VB, int NH>
-__global__ void __launch_bounds__(kDecodeWarps * 32, (NH == 1 && D <= 128) ? 2 : 1)
+__device__ __forceinline__ void store_from_f32(void* base, int64_t i, int32_t dtype, float v) {
+  if (dtype == TQ_F32) ((float*)base)[i] = v;
+  else if (dtype == TQ_BF16) ((__nv_bfloat16*)base)[i] = __float2bfloat16(v);
+  else ((__half*)base)[i] = __float2half(v);
+}
+
+// Shared memory: stages below and above the tables (see DecodeParams), and a misc
+// area [full mbarriers | release counters | present masks | q' (H_q x D fp16) |
+// |q'| scales | step prefix sums | block ids | scan scratch | flag | merge partials].
+template <int D, int KB, int VB, int NH, int MAXW>
+__global__ void __launch_bounds__(MAXW * 32, 1)
 decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   using C = DecodeCfg<D, KB, VB>;
   using KS = typename C::KS;
   using VS = typename C::VS;
-  using LK = RepLut<KB>;
-  using LV = RepLut<VB>;
-  constexpr int NST = kDecodeStages;
+  constexpr int E = D / 32;
   extern __shared__ __align__(16) uint8_t smem[];
-  uint32_t* lutK = (uint32_t*)smem;
-  const bool one_lut = KB == VB && p.shared_lut;
-  uint32_t* lutV = one_lut ? lutK : lutK + LK::kBytes / 4;
-  uint8_t* stages = smem + (one_lut ? LK::kBytes : C::kLutBytes);
-  stages += (128u - (smem_u32(stages) & 127u)) & 127u;   // TMA destinations: 128-byte aligned
-  uint64_t* full = (uint64_t*)(stages + NST * p.stage_bytes);
-  int* released = (int*)(full + NST);
-  uint32_t* present = (uint32_t*)(released + NST);     // per stage: bit k = block k staged
-  int32_t* prefix = (int32_t*)(present + NST);
-  float* cents = (float*)(prefix + p.batch + 1);   // K centroids, then V centroids
-  int32_t* ids = (int32_t*)(cents + (1 << KB) + (1 << VB));   // block ids of the range
+  {
+    // the layout planned on the host must match this launch: tables at lut_win and
+    // everything inside the allocation (else report and stop, touching nothing)
+    uint32_t dyn_bytes;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_bytes));
+    if (smem_u32(smem) + (uint32_t)p.lut_off != p.lut_win || (uint32_t)p.smem_end > dyn_bytes) {
+      if (threadIdx.x == 0) report_error(p.err, TQ_DEVERR_LAYOUT);
+      return;
+    }
+  }
+  const int nst = p.nst;
+  auto stage_ptr = [&](int x) -> uint8_t* {
+    return smem + (x < p.n_low ? p.stage_lo_off + x * p.stage_bytes
+                               : p.stage_hi_off + (x - p.n_low) * p.stage_bytes);
+  };
+  uint64_t* full = (uint64_t*)(smem + p.misc_off);
+  int* released = (int*)(full + nst);
+  uint32_t* present = (uint32_t*)(released + nst);     // per stage: bit k = block k staged
+  __half* qh = (__half*)(present + nst);               // unit q' of the current sequence
+  float* qsc = (float*)(qh + p.h_q * D);               // |q'| * scale * log2 e
+  int32_t* prefix = (int32_t*)(qsc + p.h_q);
+  int32_t* ids = (int32_t*)(prefix + p.batch + 1);     // block ids of the range
+  int* wsum = (int*)(ids + p.ids_cap);                 // [32] per-warp sums of the scan
+  int* timed_out = wsum + 32;                          // a stage wait of this CTA gave up
+  float* scratch = (float*)(timed_out + 4);            // [warps][D + 2] merge partials
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tig = lane & 3;
   const int nthreads = blockDim.x;
   const int nwarps = nthreads >> 5;                    // = h_kv * wph
-  const int per_step = p.wph;                          // blocks per pipeline step
+  const int wph = p.wph;                               // blocks per pipeline step
+  const int B = p.batch;
 
-  // ---- step prefix sums over the sequences (every CTA; CTA 0 publishes them) ----
+  // tables first: they depend on nothing but the centroids
+  lut_build<KB, 0>(smem + p.lut_off, p.kc, tid, nthreads);
+  lut_build<VB, 1>(smem + p.lut_off, p.vc, tid, nthreads);
+
+  // ---- step prefix sums over the sequences (every CTA) ----
   {
-    __shared__ int s_part[kDecodeWarps * 32];
-    const int B = p.batch;
     const int chunk = (B + nthreads - 1) / nthreads;
     const int lo = tid * chunk, hi = min(B, lo + chunk);
     int sum = 0;
@@ -379,39 +415,56 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
       if (len < 0 || len > p.max_blocks * kBlockSize) {
         if (blockIdx.x == 0) report_error(p.err, TQ_DEVERR_SEQLEN_RANGE);
       } else {
-        steps = ((len + kBlockSize - 1) / kBlockSize + per_step - 1) / per_step;
+        steps = ((len + kBlockSize - 1) / kBlockSize + wph - 1) / wph;
       }
       prefix[b + 1] = steps;
       sum += steps;
     }
-    s_part[tid] = sum;
-    if (tid < NST) {
+    if (tid < nst) {
       mbar_init(&full[tid], 1);
       released[tid] = 0;
     }
-    for (int i = tid; i < (1 << KB); i += nthreads) cents[i] = p.kc[i];
-    for (int i = tid; i < (1 << VB); i += nthreads) cents[(1 << KB) + i] = p.vc[i];
+    if (tid == 0) *timed_out = 0;
     fence_mbar_init();
+    // exclusive scan of the per-thread sums: in each warp, then over the warp totals
+    int inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += t;
+    }
+    if (lane == 31) wsum[warp] = inc;
     __syncthreads();
-    if (tid == 0) {
-      int run = 0;
-      for (int t = 0; t < nthreads; ++t) { const int v = s_part[t]; s_part[t] = run; run += v; }
-      prefix[0] = 0;
+    if (warp == 0) {
+      const int w = lane < nwarps ? wsum[lane] : 0;
+      int wi = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += t;
+      }
+      if (lane < nwarps) wsum[lane] = wi - w;
+      if (lane == 0) prefix[0] = 0;
     }
     __syncthreads();
-    int run = s_part[tid];
+    int run = wsum[warp] + inc - sum;
     for (int b = lo; b < hi; ++b) { run += prefix[b + 1]; prefix[b + 1] = run; }
     __syncthreads();
-    if (blockIdx.x == 0)
-      for (int b = tid; b <= B; b += nthreads) p.prefix[b] = prefix[b];
   }
-  const int64_t S = prefix[p.batch];
+  // sequences without steps (empty or rejected) give 0
+  for (int b = blockIdx.x; b < B; b += gridDim.x) {
+    if (prefix[b + 1] != prefix[b]) continue;
+    for (int i = tid; i < p.h_q * D; i += nthreads)
+      store_from_f32(p.out, (int64_t)b * p.o_bstride + (int64_t)(i / D) * p.o_hstride + i % D,
+                     p.out_dtype, 0.f);
+  }
+  const int64_t S = prefix[B];
   const int64_t Cn = gridDim.x;
   const int64_t s0 = cta_begin(blockIdx.x, S, Cn), s1 = cta_begin(blockIdx.x + 1, S, Cn);
   if (s0 >= s1) return;
-  // sequence walk: the largest b with prefix[b] <= s, then advance step by step
+  // sequence walk: the largest b with prefix[b] <= s
   auto locate = [&](int64_t s) {
-    int lo = 0, hi = p.batch;           // prefix[lo] <= s < prefix[hi]
+    int lo = 0, hi = B;                 // prefix[lo] <= s < prefix[hi]
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
       if (prefix[mid] <= s) lo = mid; else hi = mid;
@@ -428,7 +481,7 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   // waits on a global load.
   auto block_id = [&](int64_t s, int k) -> int32_t {
     const int b = locate(s);
-    const int bi = (int)(s - prefix[b]) * per_step + k;
+    const int bi = (int)(s - prefix[b]) * wph + k;
     const int nblk = (p.seq_lens[b] + kBlockSize - 1) / kBlockSize;
     if (bi >= nblk) return -1;
     const int32_t blk = p.block_table[(int64_t)b * p.bt_stride + bi];
@@ -438,22 +491,30 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     }
     return blk;
   };
-  const int64_t nids = (s1 - s0) * per_step;
-  for (int64_t i = tid; i < nids && i < p.ids_cap; i += nthreads)
-    ids[i] = block_id(s0 + i / per_step, (int)(i % per_step));
-  __syncthreads();
+  // Block ids: warp 0 resolves those of the first nst steps and issues their copies at
+  // once (below); the other warps preload the rest of the range meanwhile.
+  const int64_t nids = imin64((s1 - s0) * wph, p.ids_cap);
+  const int64_t nfirst = imin64((int64_t)nst * wph, nids);
+  if (warp == 0) {
+    for (int64_t i = lane; i < nfirst; i += 32) ids[i] = block_id(s0 + i / wph, (int)(i % wph));
+    __syncwarp();
+  }
+  {
+    const int first_t = nwarps > 1 ? 32 : 0;          // a lone warp preloads the rest too
+    if (tid >= first_t)
+      for (int64_t i = nfirst + tid - first_t; i < nids; i += nthreads - first_t)
+        ids[i] = block_id(s0 + i / wph, (int)(i % wph));
+  }
 
-  // Stage refill for global step s (issued by one warp): one TMA copy per block of
-  // the step, completing on full[stage]; present[stage] tells the consumers which
-  // blocks were staged.  With copy_mode 1 the block is a 2-D box of 16 rows whose
-  // width is the padded pitch: the columns past the row end lie outside the tensor
-  // and are zero-filled, which pads every row in shared memory.
-  const uint32_t blk_copy_bytes = p.copy_mode ? (uint32_t)blk_smem : (uint32_t)(kBlockSize * row_bytes);
-  auto refill = [&](int64_t s) {
-    const int x = (int)((s - s0) % NST);
-    const int64_t i0 = (s - s0) * per_step;
+  // Stage refill for global step s into stage x (issued by one warp): one TMA copy per
+  // block of the step, completing on full[x]; present[x] tells the consumers which
+  // blocks were staged.
+  const uint32_t blk_copy_bytes =
+      p.copy_mode ? (uint32_t)blk_smem : (uint32_t)(kBlockSize * row_bytes);
+  auto refill = [&](int64_t s, int x) {
+    const int64_t i0 = (s - s0) * wph;
     int32_t blk = -1;
-    if (lane < per_step) blk = i0 + lane < p.ids_cap ? ids[i0 + lane] : block_id(s, lane);
+    if (lane < wph) blk = i0 + lane < p.ids_cap ? ids[i0 + lane] : block_id(s, lane);
     const uint32_t bits = __ballot_sync(0xffffffffu, blk >= 0);
     if (lane == 0) {
       present[x] = bits;                 // published by the arrive (release) below
@@ -461,38 +522,83 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     }
     __syncwarp();
     if (blk >= 0) {
-      uint8_t* d = stages + x * p.stage_bytes + lane * blk_smem;
+      uint8_t* d = stage_ptr(x) + lane * blk_smem;
       if (p.copy_mode) tensor_g2s_2d(d, &tmap, 0, blk * kBlockSize, &full[x]);
       else bulk_g2s(d, p.pages + (int64_t)blk * p.blk_stride, blk_copy_bytes, &full[x]);
     }
   };
   if (warp == 0)
-    for (int64_t s = s0; s < s1 && s < s0 + NST; ++s) refill(s);
+    for (int i = 0; i < nst && s0 + i < s1; ++i) refill(s0 + i, i);
 
-  LK::build(lutK, cents, tid, nthreads);
-  if (!one_lut) LV::build(lutV, cents + (1 << KB), tid, nthreads);
-  __syncthreads();
+
+  // q' = R q of the query heads of sequence b into qh / qsc (the warps split the heads)
+  auto rotate_q = [&](int b) {
+    uint32_t sg[E];
+#pragma unroll
+    for (int i = 0; i < E; ++i) sg[i] = sign_mask_at(p.sign_seed, lane * E + i);
+    for (int h = warp; h < p.h_q; h += nwarps) {
+      const int64_t off = (int64_t)b * p.q_bstride + (int64_t)h * p.q_hstride + lane * E;
+      float x[E];
+#pragma unroll
+      for (int i = 0; i < E; ++i)
+        x[i] = __uint_as_float(__float_as_uint(load_as_f32(p.q, off + i, p.q_dtype)) ^ sg[i]);
+      warp_fwht<E>(x, lane);
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        x[i] *= inv_sqrt_dim<D>();
+        ss = fmaf(x[i], x[i], ss);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float nrm = sqrtf(ss);
+      const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
+#pragma unroll
+      for (int i = 0; i < E; ++i) qh[h * D + lane * E + i] = __float2half_rn(x[i] * inv);
+      if (lane == 0) qsc[h] = nrm * p.scale_log2;
+    }
+  };
 
   const int kvh = warp % p.h_kv;
   const int sub = warp / p.h_kv;
   const int G = p.group;
-  const uint32_t* lk = lutK + lane;
-  const uint32_t* lv = lutV + lane;
+  const uint32_t lk_off = p.lut_win | (4u * lane), lv_off = p.lut_win | (128u + 4u * lane);
 
-  // Layout of the score product S^T = K~ . Qhat^T (M = 16 tokens, N = 8 query heads
-  // per head group hh, K = coordinates): this thread holds, for m-tile mt (tokens
-  // 16mt..16mt+15) and head group hh, sacc[mt][hh][r] = S^T[token 16mt + gid + 8(r>>1)]
-  // [head 8hh + 2tig + (r&1)].  Every value it needs for the softmax of its two heads
-  // (2tig, 2tig+1) is therefore local, and the O'^T accumulator columns are the same
-  // two heads.
-  uint32_t qb[C::KSTEPS][NH][2];     // B fragments of Qhat^T: head 8hh + gid
-  float qscale[NH][2];               // heads 8hh + 2tig + {0, 1}
+  // per warp: q fragments (B operand of the score product), softmax state, O'^T
+  uint32_t qb[C::KSTEPS][NH][2];
+  float qscale[NH][2];
   float Mrun[NH][2], lrun[NH][2];
   float acc[NH][C::MT][4];
 
-  // record of (CTA c, sequence b): index c + b (unique, see cta_of)
+  auto start = [&]() {
+#pragma unroll
+    for (int hh = 0; hh < NH; ++hh) {
+      const int g = 8 * hh + gid;
+      const bool have = g < G;
+      const __half* qrow = qh + (kvh * G + (have ? g : 0)) * D;
+#pragma unroll
+      for (int ks = 0; ks < C::KSTEPS; ++ks) {
+        const int c0 = KS::coord(tig, 4 * ks), c2 = KS::coord(tig, 4 * ks + 2);
+        qb[ks][hh][0] = have ? *(const uint32_t*)(qrow + c0) : 0u;
+        qb[ks][hh][1] = have ? *(const uint32_t*)(qrow + c2) : 0u;
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int ge = 8 * hh + 2 * tig + e;
+        qscale[hh][e] = ge < G ? qsc[kvh * G + ge] : 0.f;
+        Mrun[hh][e] = -INFINITY;
+        lrun[hh][e] = 0.f;
+      }
+#pragma unroll
+      for (int mt = 0; mt < C::MT; ++mt)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[hh][mt][k] = 0.f;
+    }
+  };
+
+  // this warp's partial of sequence b -> its record
   auto flush = [&](int b) {
-    float* base = p.part + ((int64_t)(blockIdx.x + b) * p.wph + sub) * (int64_t)p.h_q * (D + 2);
+    float* base = p.part + ((int64_t)(blockIdx.x + b) * wph + sub) * (int64_t)p.h_q * (D + 2);
 #pragma unroll
     for (int hh = 0; hh < NH; ++hh) {
 #pragma unroll
@@ -520,47 +626,198 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
       });
     }
   };
-  auto start = [&](int b) {
-#pragma unroll
-    for (int hh = 0; hh < NH; ++hh) {
-      const int g = 8 * hh + gid;
-      const bool have = g < G;
-      const int64_t h = (int64_t)b * p.h_q + kvh * G + (have ? g : 0);
-      const uint4* src = (const uint4*)(p.qfrag + (h * 4 + tig) * (2 * C::KSTEPS));
-#pragma unroll
-      for (int v = 0; v < C::KSTEPS / 2; ++v) {
-        const uint4 w = have ? src[v] : make_uint4(0u, 0u, 0u, 0u);
-        qb[2 * v][hh][0] = w.x; qb[2 * v][hh][1] = w.y;
-        qb[2 * v + 1][hh][0] = w.z; qb[2 * v + 1][hh][1] = w.w;
-      }
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int ge = 8 * hh + 2 * tig + e;
-        qscale[hh][e] = ge < G ? p.qscale[(int64_t)b * p.h_q + kvh * G + ge] : 0.f;
-        Mrun[hh][e] = -INFINITY;
-        lrun[hh][e] = 0.f;
-      }
-#pragma unroll
-      for (int mt = 0; mt < C::MT; ++mt)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[hh][mt][k] = 0.f;
+
+  auto nonempty = [&](int64_t c) {
+    return S >= Cn || cta_begin(c, S, Cn) < cta_begin(c + 1, S, Cn);
+  };
+  unsigned int* arrived = p.counters;                // records of sequence b written
+  unsigned int* merged = p.counters + B;             // covering CTAs done merging b
+
+  // Merge of query head h of sequence b over records i = i_first, i_first + i_step, ...
+  // (record i: CTA c_lo + i / wph, sub-stream i % wph) into this warp's partial
+  // (M, l, O'[lane E .. lane E + E - 1]).
+  auto merge_part = [&](int b, int h, int64_t c_lo, int R, int i_first, int i_step, float& M,
+                        float& l, float (&o)[E]) {
+    const int64_t rstride = (int64_t)p.h_q * (D + 2);
+    const float* hb = p.part + (int64_t)h * (D + 2);
+    auto rec_of = [&](int i) -> int64_t {
+      const int64_t c = c_lo + i / wph;
+      return nonempty(c) ? ((c + b) * wph + i % wph) * rstride : -1;
+    };
+    M = -INFINITY;
+    for (int i = i_first + lane * i_step; i < R; i += 32 * i_step) {
+      const int64_t r = rec_of(i);
+      if (r >= 0) M = fmaxf(M, __ldcg(hb + r));
     }
+#pragma unroll
+    for (int of = 16; of > 0; of >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, of));
+    l = 0.f;
+#pragma unroll
+    for (int i = 0; i < E; ++i) o[i] = 0.f;
+    if (M == -INFINITY) return;
+    for (int i0 = i_first; i0 < R; i0 += 32 * i_step) {
+      // lane j of this pass: weight and offset of record i0 + j i_step
+      const int i = i0 + lane * i_step;
+      const int64_t r = i < R ? rec_of(i) : -1;
+      float wt = 0.f;
+      if (r >= 0) {
+        const float mi = __ldcg(hb + r);
+        wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
+        l += wt * __ldcg(hb + r + 1);
+      }
+      const int nr = min(32, (R - i0 + i_step - 1) / i_step);
+      for (int j = 0; j < nr; j += 4) {
+        float wv[4], v[4][E];
+        int64_t rr[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int src = min(j + u, 31);
+          wv[u] = __shfl_sync(0xffffffffu, wt, src);
+          rr[u] = __shfl_sync(0xffffffffu, r, src);
+          if (j + u >= nr) wv[u] = 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (wv[u] != 0.f) {
+            const float2* src = (const float2*)(hb + rr[u] + 2 + lane * E);
+#pragma unroll
+            for (int k = 0; k < E / 2; ++k) {
+              const float2 t = __ldcg(src + k);
+              v[u][2 * k] = t.x;
+              v[u][2 * k + 1] = t.y;
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < E; ++k) v[u][k] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int k = 0; k < E; ++k) o[k] = fmaf(wv[u], v[u][k], o[k]);
+      }
+    }
+#pragma unroll
+    for (int of = 16; of > 0; of >>= 1) l += __shfl_xor_sync(0xffffffffu, l, of);
+  };
+
+  // End phase for sequence b: once every CTA covering b has written its records, this
+  // CTA (rank k of the n covering CTAs) merges query heads k, k + n, ...: groups of g
+  // warps take one head each, split its records, and the group's first warp combines
+  // the g partials, divides by l and applies o = R^T O' (FWHT, 1/sqrt(D), sign flips).
+  auto coop_merge = [&](int b) {
+    const int64_t c_lo = cta_of(prefix[b], S, Cn), c_hi = cta_of(prefix[b + 1] - 1, S, Cn);
+    int n = 0, rank = 0;
+    for (int64_t c = c_lo; c <= c_hi; ++c)
+      if (nonempty(c)) {
+        if (c < (int64_t)blockIdx.x) ++rank;
+        ++n;
+      }
+    const int R = (int)(c_hi - c_lo + 1) * wph;
+    if (tid == 0) {
+      // wait until all n covering CTAs have arrived (bounded)
+      const uint64_t t0 = globaltimer_ns();
+      while (*(volatile unsigned int*)&arrived[b] < (unsigned)n) {
+        if (globaltimer_ns() - t0 > (uint64_t)kWaitMs * 1000000ull) {
+          report_error(p.err, TQ_DEVERR_TIMEOUT);
+          break;
+        }
+        __nanosleep(256);
+      }
+      __threadfence();
+    }
+    __syncthreads();
+    const int nh = rank < p.h_q ? (p.h_q - rank + n - 1) / n : 0;   // heads of this CTA
+    int g = 1;
+    while (nh > 0 && 2 * g * min(nh, nwarps) <= nwarps) g *= 2;
+    const int groups = nwarps / g, gi = warp / g, mi = warp % g;
+    uint32_t sg[E];
+#pragma unroll
+    for (int i = 0; i < E; ++i) sg[i] = sign_mask_at(p.sign_seed, lane * E + i);
+    for (int j0 = 0; j0 < nh; j0 += groups) {
+      const int j = j0 + gi;
+      const int h = rank + j * n;
+      float M, l, o[E];
+      if (j < nh) {
+        merge_part(b, h, c_lo, R, mi, g, M, l, o);
+        float* sc = scratch + warp * (D + 2);
+        if (lane == 0) { sc[0] = M; sc[1] = l; }
+#pragma unroll
+        for (int i = 0; i < E; ++i) sc[2 + lane * E + i] = o[i];
+      }
+      __syncthreads();
+      if (j < nh && mi == 0) {
+        float Mx = -INFINITY;
+        for (int w = 0; w < g; ++w) Mx = fmaxf(Mx, scratch[(warp + w) * (D + 2)]);
+        float L = 0.f, acc_o[E];
+#pragma unroll
+        for (int i = 0; i < E; ++i) acc_o[i] = 0.f;
+        if (Mx != -INFINITY) {
+          for (int w = 0; w < g; ++w) {
+            const float* sc = scratch + (warp + w) * (D + 2);
+            const float mw = sc[0];
+            const float f = mw == -INFINITY ? 0.f : exp2f(mw - Mx);
+            L += f * sc[1];
+#pragma unroll
+            for (int i = 0; i < E; ++i) acc_o[i] = fmaf(f, sc[2 + lane * E + i], acc_o[i]);
+          }
+        }
+        const float inv = L > 0.f ? 1.0f / L : 0.f;
+#pragma unroll
+        for (int i = 0; i < E; ++i) acc_o[i] *= inv;
+        warp_fwht<E>(acc_o, lane);
+        const int64_t ob = (int64_t)b * p.o_bstride + (int64_t)h * p.o_hstride + lane * E;
+#pragma unroll
+        for (int i = 0; i < E; ++i)
+          store_from_f32(p.out, ob + i, p.out_dtype,
+                         __uint_as_float(__float_as_uint(acc_o[i] * inv_sqrt_dim<D>()) ^ sg[i]));
+      }
+      __syncthreads();
+    }
+    // the last covering CTA to finish clears both counters (ready for a replay)
+    if (tid == 0 && atomicAdd(&merged[b], 1u) == (unsigned)n - 1) {
+      atomicExch(&arrived[b], 0u);
+      atomicExch(&merged[b], 0u);
+    }
+  };
+
+  // Leave sequence b for nb (the next sequence of the range): write the records of b,
+  // count them on b's counter, rotate the queries of nb.
+  auto boundary = [&](int b, int nb) {
+    flush(b);
+    __syncthreads();                    // records of b written; q' of b no longer read
+    if (tid == 0) {
+      __threadfence();
+      atomicAdd(&arrived[b], 1u);
+    }
+    rotate_q(nb);
+    __syncthreads();
+    start();
   };
 
   int cur_b = locate(s0);
   int local = (int)(s0 - prefix[cur_b]);
   int cur_len = p.seq_lens[cur_b];
-  start(cur_b);
+  rotate_q(cur_b);
+  __syncthreads();                      // tables and q' ready
+  start();
+
+  int x = 0;
+  uint32_t phase = 0;
+  bool dead = false;                    // a stage wait of this warp gave up
   for (int64_t s = s0; s < s1; ++s) {
-    const int x = (int)((s - s0) % NST);
-    if (!mbar_wait(&full[x], (uint32_t)(((s - s0) / NST) & 1), kWaitLimit)) {
-      if (lane == 0) report_error(p.err, TQ_DEVERR_TIMEOUT);
-      return;
+    if (!dead && !mbar_wait(&full[x], phase, kWaitMs)) {
+      if (lane == 0) {
+        report_error(p.err, TQ_DEVERR_TIMEOUT);
+        *timed_out = 1;
+      }
+      dead = true;
     }
-    const int bi = local * per_step + sub;                // this warp's block
-    const int valid = ((present[x] >> sub) & 1u) ? min(kBlockSize, cur_len - bi * kBlockSize) : 0;
+    const int bi = local * wph + sub;                 // this warp's block
+    const int valid =
+        (!dead && ((present[x] >> sub) & 1u)) ? min(kBlockSize, cur_len - bi * kBlockSize) : 0;
     if (valid > 0) {
-      const uint8_t* base = stages + x * p.stage_bytes + sub * blk_smem + kvh * p.slot_stride;
+      const uint8_t* base = stage_ptr(x) + sub * blk_smem + kvh * p.slot_stride;
       // token t (0..15) of this block lives at base + t * pitch
 
       // ---- S^T = K~ . Qhat^T: one m-tile of 16 tokens ----
@@ -575,10 +832,10 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
         KS::load(kw1, base + (gid + 8) * pitch, tig);
         static_for<C::KSTEPS>([&](auto KSI) {
           constexpr int ks = decltype(KSI)::value;
-          const uint32_t a0 = LK::pair_field(lk, field<KS::pos(4 * ks), 2 * KB>(kw0));
-          const uint32_t a1 = LK::pair_field(lk, field<KS::pos(4 * ks), 2 * KB>(kw1));
-          const uint32_t a2 = LK::pair_field(lk, field<KS::pos(4 * ks + 2), 2 * KB>(kw0));
-          const uint32_t a3 = LK::pair_field(lk, field<KS::pos(4 * ks + 2), 2 * KB>(kw1));
+          const uint32_t a0 = lut_pair<KB, KS::pos(4 * ks)>(kw0, lk_off);
+          const uint32_t a1 = lut_pair<KB, KS::pos(4 * ks)>(kw1, lk_off);
+          const uint32_t a2 = lut_pair<KB, KS::pos(4 * ks + 2)>(kw0, lk_off);
+          const uint32_t a3 = lut_pair<KB, KS::pos(4 * ks + 2)>(kw1, lk_off);
 #pragma unroll
           for (int hh = 0; hh < NH; ++hh)
             mma_16816(sacc[hh], a0, a1, a2, a3, qb[ks][hh][0], qb[ks][hh][1]);
@@ -591,34 +848,43 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
       for (int r = 0; r < 2; ++r) {
         const int t = gid + 8 * r;
         const uint8_t* sl = base + t * pitch;
+        ok[r] = t < valid;
         nK[r] = *(const float*)(sl + C::KPACK);
-        nV[r] = *(const float*)(sl + p.k_region + C::VPACK);
+        // masked tokens may hold stale norms (even NaN): their V norm is taken as 0
+        nV[r] = ok[r] ? *(const float*)(sl + p.k_region + C::VPACK) : 0.f;
         // floor at 2^-100 keeps 2^(s - M) finite for rows of (near) zero V norm
         eV[r] = fmaxf(log2_ceilish(nV[r]), -100.0f);
-        ok[r] = t < valid;
       }
       uint32_t pb[NH][2];   // [head group][b0b1 | b2b3]
 #pragma unroll
       for (int hh = 0; hh < NH; ++hh) {
         float sv[2][2];        // [head e][token r]
-        float zmax[2];
+        float zloc[2];         // this thread's max of s + e(nV) per head
+        bool need = false;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          zmax[e] = -INFINITY;
+          zloc[e] = -INFINITY;
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
             const float a = sacc[hh][2 * r + e];
             sv[e][r] = ok[r] ? a * nK[r] * qscale[hh][e] : -INFINITY;
-            zmax[e] = fmaxf(zmax[e], sv[e][r] + eV[r]);
+            zloc[e] = fmaxf(zloc[e], sv[e][r] + eV[r]);
           }
-#pragma unroll
-          for (int o = 4; o < 32; o <<= 1)
-            zmax[e] = fmaxf(zmax[e], __shfl_xor_sync(0xffffffffu, zmax[e], o));
+          need |= zloc[e] > Mrun[hh][e] + kLazyRescale;
         }
-        // lazy reference: raise M only when the tile beats it by more than 2^8
-        const bool raise0 = zmax[0] > Mrun[hh][0] + kLazyRescale;
-        const bool raise1 = zmax[1] > Mrun[hh][1] + kLazyRescale;
-        if (__any_sync(0xffffffffu, raise0 || raise1)) {
+        // lazy reference: raise M only when the tile beats it by more than 2^8 (the
+        // tile maxima over the 16 tokens are only formed when some lane needs them)
+        if (__any_sync(0xffffffffu, need)) {
+          float zmax[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            zmax[e] = zloc[e];
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1)
+              zmax[e] = fmaxf(zmax[e], __shfl_xor_sync(0xffffffffu, zmax[e], o));
+          }
+          const bool raise0 = zmax[0] > Mrun[hh][0] + kLazyRescale;
+          const bool raise1 = zmax[1] > Mrun[hh][1] + kLazyRescale;
           float alpha[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
@@ -641,10 +907,9 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
           float lsum = 0.f;
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
-            const float w = ok[r] ? exp2f(sv[e][r] - M) : 0.f;
+            const float w = ex2_approx(sv[e][r] - M);   // exactly 0 for masked tokens
             lsum += w;
-            // masked tokens may hold stale norms (even NaN): their weight is exactly 0
-            pv[e][r] = ok[r] ? w * nV[r] : 0.f;
+            pv[e][r] = w * nV[r];
           }
           lrun[hh][e] += lsum;
         }
@@ -676,10 +941,10 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
             static_for<PER>([&](auto KI) {
               constexpr int k = decltype(KI)::value;
               constexpr int mt = j * PER + k;
-              const uint32_t a0 = LV::pair_field(lv, bits_of<2 * VB * k, 2 * VB>(loAB));
-              const uint32_t a1 = LV::pair_field(lv, bits_of<2 * VB * k, 2 * VB>(hiAB));
-              const uint32_t a2 = LV::pair_field(lv, bits_of<2 * VB * k, 2 * VB>(loCD));
-              const uint32_t a3 = LV::pair_field(lv, bits_of<2 * VB * k, 2 * VB>(hiCD));
+              const uint32_t a0 = lut_ld(lut_addr1<2 * VB * k, 2 * VB>(loAB, lv_off));
+              const uint32_t a1 = lut_ld(lut_addr1<2 * VB * k, 2 * VB>(hiAB, lv_off));
+              const uint32_t a2 = lut_ld(lut_addr1<2 * VB * k, 2 * VB>(loCD, lv_off));
+              const uint32_t a3 = lut_ld(lut_addr1<2 * VB * k, 2 * VB>(hiCD, lv_off));
 #pragma unroll
               for (int hh = 0; hh < NH; ++hh)
                 mma_16816(acc[hh][mt], a0, a1, a2, a3, pb[hh][0], pb[hh][1]);
@@ -689,10 +954,10 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
           static_for<C::MT>([&](auto MI) {
             constexpr int mt = decltype(MI)::value;
             constexpr int p0 = VS::pos(2 * mt), p1 = VS::pos(2 * mt + 1);
-            const uint32_t a0 = LV::pair(lv, field<p0, VB>(vw[0]), field<p0, VB>(vw[1]));
-            const uint32_t a1 = LV::pair(lv, field<p1, VB>(vw[0]), field<p1, VB>(vw[1]));
-            const uint32_t a2 = LV::pair(lv, field<p0, VB>(vw[2]), field<p0, VB>(vw[3]));
-            const uint32_t a3 = LV::pair(lv, field<p1, VB>(vw[2]), field<p1, VB>(vw[3]));
+            const uint32_t a0 = lut_pair2<VB, p0>(vw[0], vw[1], lv_off);
+            const uint32_t a1 = lut_pair2<VB, p1>(vw[0], vw[1], lv_off);
+            const uint32_t a2 = lut_pair2<VB, p0>(vw[2], vw[3], lv_off);
+            const uint32_t a3 = lut_pair2<VB, p1>(vw[2], vw[3], lv_off);
 #pragma unroll
             for (int hh = 0; hh < NH; ++hh)
               mma_16816(acc[hh][mt], a0, a1, a2, a3, pb[hh][0], pb[hh][1]);
@@ -700,7 +965,7 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
         }
       }
     }
-    // release the stage; the last warp to do so refills it with step s + NST
+    // release the stage; the last warp to do so refills it with step s + nst
     __syncwarp();
     int last = 0;
     if (lane == 0) {
@@ -708,112 +973,43 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
       if (last) released[x] = 0;
     }
     last = __shfl_sync(0xffffffffu, last, 0);
-    if (last && s + NST < s1) refill(s + NST);
-    // advance the sequence walk; flush the partial at a sequence boundary
+    if (last && s + nst < s1) refill(s + nst, x);
+    if (++x == nst) {
+      x = 0;
+      phase ^= 1u;
+    }
+    // advance the sequence walk; at a sequence boundary: flush, ticket, maybe merge
     if (s + 1 < s1) {
       ++local;
-      int nb = cur_b;
-      while (local >= prefix[nb + 1] - prefix[nb]) { ++nb; local = 0; }
-      if (nb != cur_b) {
-        flush(cur_b);
+      if (local >= prefix[cur_b + 1] - prefix[cur_b]) {
+        int nb = cur_b + 1;
+        while (prefix[nb + 1] == prefix[nb]) ++nb;
+        boundary(cur_b, nb);
         cur_b = nb;
+        local = 0;
         cur_len = p.seq_lens[cur_b];
-        start(cur_b);
       }
     }
   }
+  // end phase: publish the records of the last sequence, then merge each sequence of
+  // the range together with the other CTAs that cover it
   flush(cur_b);
-}
-
-// Merge the partial records of one (sequence, query head), then o = R^T (O' / l):
-// a FWHT of the rotated-domain output, sign flips and the 1/sqrt(D) scale.  The
-// records of sequence b come from CTAs cta_of(first step) .. cta_of(last step),
-// record index c + b.  Eight warps split the records; each lane owns D/32
-// coordinates.
-template <int D>
-__global__ void __launch_bounds__(256)
-merge_kernel(MergeParams p) {
-  constexpr int NW = 8, CPL = D / 32;
-  __shared__ float buf[D];
-  __shared__ float part_o[NW][D];
-  __shared__ float part_l[NW];
-  __shared__ float red[NW];
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t sb = p.prefix[b], eb = p.prefix[b + 1];
-  const int64_t S = p.prefix[gridDim.y], Cn = p.nctas;
-  const int64_t rstride = (int64_t)p.h_q * (D + 2);
-  const float* hbase = p.part + (int64_t)h * (D + 2);
-  float o[CPL];
-#pragma unroll
-  for (int k = 0; k < CPL; ++k) o[k] = 0.f;
-  float l = 0.f;
-  int n = 0;
-  int64_t c_lo = 0;
-  const int wshift = __ffs(p.wph) - 1;               // wph is a power of two
-  if (eb > sb) {
-    c_lo = cta_of(sb, S, Cn);
-    n = (int)(cta_of(eb - 1, S, Cn) - c_lo + 1) << wshift;
-  }
-  // record i -> record offset, or -1 for a CTA whose step range is empty
-  auto rec_index = [&](int i) -> int64_t {
-    const int64_t c = c_lo + (i >> wshift);
-    if (cta_begin(c, S, Cn) >= cta_begin(c + 1, S, Cn)) return -1;
-    return (c + b) * p.wph + (i & (p.wph - 1));
-  };
-  float M = -INFINITY;
-  for (int i = tid; i < n; i += 256) {
-    const int64_t r = rec_index(i);
-    if (r >= 0) M = fmaxf(M, hbase[r * rstride]);
-  }
-#pragma unroll
-  for (int of = 16; of > 0; of >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, of));
-  if (lane == 0) red[warp] = M;
   __syncthreads();
-  M = red[0];
-#pragma unroll
-  for (int w = 1; w < NW; ++w) M = fmaxf(M, red[w]);
-  if (M != -INFINITY) {
-    for (int i = warp; i < n; i += NW) {
-      const int64_t r = rec_index(i);
-      if (r < 0) continue;
-      const float* rec = hbase + r * rstride;
-      const float mi = rec[0];
-      const float w = mi == -INFINITY ? 0.f : exp2f(mi - M);
-      l += w * rec[1];
-#pragma unroll
-      for (int k = 0; k < CPL; ++k) o[k] += w * rec[2 + lane + 32 * k];
-    }
-  }
-#pragma unroll
-  for (int k = 0; k < CPL; ++k) part_o[warp][lane + 32 * k] = o[k];
-  if (lane == 0) part_l[warp] = l;
-  __syncthreads();
-  if (tid < D) {
-    float os = 0.f, ls = 0.f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) { os += part_o[w][tid]; ls += part_l[w]; }
-    buf[tid] = ls > 0.f ? os / ls : 0.f;
-  }
-  __syncthreads();
-  for (int hs = 1; hs < D; hs <<= 1) {
-    float v = 0.f;
-    if (tid < D) {
-      const float mine = buf[tid], other = buf[tid ^ hs];
-      v = (tid & hs) ? other - mine : mine + other;
+  if (*timed_out) {
+    // copies may still be landing in the stages: give them time (bounded), skip the merge
+    if (tid == 0) {
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 100000000ull) __nanosleep(1000);
     }
     __syncthreads();
-    if (tid < D) buf[tid] = v;
-    __syncthreads();
+    return;
   }
-  if (tid < D) {
-    float r = buf[tid] * inv_sqrt_dim<D>();
-    r = __uint_as_float(__float_as_uint(r) ^ sign_mask_at(p.sign_seed, tid));
-    const int64_t off = (int64_t)b * p.o_bstride + (int64_t)h * p.o_hstride + tid;
-    if (p.out_dtype == TQ_F32) ((float*)p.out)[off] = r;
-    else if (p.out_dtype == TQ_BF16) ((__nv_bfloat16*)p.out)[off] = __float2bfloat16(r);
-    else ((__half*)p.out)[off] = __float2half(r);
+  if (tid == 0) {
+    __threadfence();
+    atomicAdd(&arrived[cur_b], 1u);
   }
+  for (int b = locate(s0); b <= cur_b; ++b)
+    if (prefix[b + 1] > prefix[b]) coop_merge(b);
 }
 
 }  // namespace tq

@@ -79,8 +79,8 @@ __device__ __forceinline__ void cp_async_wait() {
 
 // ---------------------------------------------------------------------------
 // mbarrier + bulk (TMA) copies.  Plain global->shared bulk copies of this CTA's own
-// memory, never with multicast.  Every wait is bounded: after `limit` polls it gives
-// up and the caller reports TQ_DEVERR_TIMEOUT.
+// memory, never with multicast.  Every wait is bounded in time: when it gives up the
+// caller reports TQ_DEVERR_TIMEOUT.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -99,24 +99,33 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
       "r"(bytes)
       : "memory");
 }
-// One poll; the hardware may suspend the warp (up to ~suspend_ns) until the phase
-// completes, so waiting warps do not compete for issue slots.
+// One poll (the hardware may hold the warp for a short, system-defined time while
+// the phase is still open).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
       " selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
-// Wait for the phase with the given parity to complete; false after `limit` polls
-// (each poll suspends for at most about 1 ms).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
-  for (uint32_t i = 0; i < limit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for the phase with the given parity to complete; false once about `limit_ms`
+// milliseconds have passed without it.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit_ms) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > (uint64_t)limit_ms * 1000000ull) return false;
+  }
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(

@@ -15,18 +15,24 @@ namespace tq {
 struct DeviceInfo {
   int num_sms = 0;
   int max_smem_optin = 0;
+  uint32_t dyn_smem_base = 0;   // shared-window address where dynamic shared memory starts
+                                // (kernels without static shared memory)
 };
 
 struct DecodePlan {
+  int maxw = 16;          // warps per CTA the kernel is compiled for (16 or 8)
+  uint32_t lut_win = 0;   // shared-memory layout (see DecodeParams)
+  int lut_off = 0, stage_lo_off = 0, stage_hi_off = 0, n_low = 0, misc_off = 0;
   int wph = 1;            // warps (sub-streams) per KV head
-  int row_pitch = 0;      // padded shared-memory row pitch (bytes)
+  int nst = 4;            // stages in the ring
+  int row_pitch = 0;      // shared-memory row pitch (bytes)
   int stage_bytes = 0;    // one pipeline stage: wph blocks
   int ids_cap = 0;        // block ids a CTA preloads into shared memory
   int copy_mode = 0;      // 1: 2-D tensor box per block (padded rows); 0: 1-D bulk copy
-  int shared_lut = 0;     // K and V share one lookup table
+  int lut_bytes = 0;      // lookup tables at the start of shared memory
   size_t smem = 0;        // dynamic shared memory of the decode kernel
-  int max_ctas = 0;       // upper bound of the persistent grid
-  size_t qfrag_off = 0, qscale_off = 0, prefix_off = 0, part_off = 0;
+  int max_ctas = 0;       // upper bound of the persistent grid (one CTA per SM)
+  size_t part_off = 0, counters_off = 0;
   size_t ws_bytes = 0;
 };
 
@@ -38,14 +44,11 @@ tq_status launch_append_any(int dim, int dtype, const AppendParams& p, const Dev
                             cudaStream_t st);
 tq_status launch_rotate_any(int dim, int dtype, const RotateParams& p, const DeviceInfo& di,
                             cudaStream_t st);
-tq_status launch_decode_d64(int kb, int vb, const DecodeParams& p, const QPrepParams& qp,
-                            const MergeParams& m, const DecodePlan& plan,
+tq_status launch_decode_d64(int kb, int vb, const DecodeParams& p, const DecodePlan& plan,
                             const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st);
-tq_status launch_decode_d128(int kb, int vb, const DecodeParams& p, const QPrepParams& qp,
-                             const MergeParams& m, const DecodePlan& plan,
+tq_status launch_decode_d128(int kb, int vb, const DecodeParams& p, const DecodePlan& plan,
                              const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st);
-tq_status launch_decode_d256(int kb, int vb, const DecodeParams& p, const QPrepParams& qp,
-                             const MergeParams& m, const DecodePlan& plan,
+tq_status launch_decode_d256(int kb, int vb, const DecodeParams& p, const DecodePlan& plan,
                              const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st);
 
 // (K bits, V bits) pairs with a compiled decode kernel.
@@ -56,52 +59,52 @@ inline bool decode_bits_supported(int kb, int vb) {
   return false;
 }
 
-template <int D, int KB, int VB, int NH>
-tq_status launch_decode_t(DecodeParams p, QPrepParams qp, MergeParams m, const DecodePlan& plan,
-                          const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st) {
-  auto kern = decode_kernel<D, KB, VB, NH>;
+template <int D, int KB, int VB, int NH, int MAXW>
+tq_status launch_decode_t(const DecodeParams& p, const DecodePlan& plan, const CUtensorMap& tmap,
+                          int64_t steps_upper, cudaStream_t st) {
+  auto kern = decode_kernel<D, KB, VB, NH, MAXW>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem) !=
       cudaSuccess)
     return TQ_ERR_CUDA;
   const int threads = p.h_kv * plan.wph * 32;
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, plan.smem) !=
-      cudaSuccess)
-    return TQ_ERR_CUDA;
-  per_sm = std::max(1, std::min(per_sm, 2));
-  int num_sms = plan.max_ctas / 2;
-  // persistent grid, but at least two steps per CTA so that tiny batches do not pay
-  // one prologue per step
-  const int64_t ctas = std::max<int64_t>(
-      1, std::min<int64_t>(std::min<int64_t>((int64_t)num_sms * per_sm, plan.max_ctas),
-                           (steps_upper + 1) / 2));
-  m.nctas = (int32_t)ctas;
-  const int qrows = p.batch * p.h_q;
-  qprep_kernel<D, KB><<<(qrows + 7) / 8, 256, 0, st>>>(qp, qrows);
-  tq_status s = launch_status();
-  if (s != TQ_OK) return s;
-  kern<<<(unsigned)ctas, threads, plan.smem, st>>>(p, tmap);
-  s = launch_status();
-  if (s != TQ_OK) return s;
-  merge_kernel<D><<<dim3(p.h_q, p.batch), 256, 0, st>>>(m);
+  // persistent grid of one CTA per SM, but at least two steps per CTA so that tiny
+  // batches do not pay one prologue per step
+  const int64_t ctas =
+      std::max<int64_t>(1, std::min<int64_t>(plan.max_ctas, (steps_upper + 1) / 2));
+  // cooperative: the CTAs of a sequence wait for one another before merging it, so all
+  // of them must be resident at once
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ctas);
+  cfg.blockDim = dim3((unsigned)threads);
+  cfg.dynamicSmemBytes = plan.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, p, tmap) != cudaSuccess) return TQ_ERR_CUDA;
   return launch_status();
 }
 
+// Warps per CTA the decode kernel is compiled for: 16 (<= 128 registers a thread) when
+// the per-warp state fits, else 8.
+inline int decode_maxw(int dim, int group) { return dim <= 128 && group <= 8 ? 16 : 8; }
+
 template <int D, int KB, int VB>
-tq_status launch_decode_bits(const DecodeParams& p, const QPrepParams& qp, const MergeParams& m,
-                             const DecodePlan& plan, const CUtensorMap& tmap,
-                             int64_t steps_upper, cudaStream_t st) {
-  return p.group > 8 ? launch_decode_t<D, KB, VB, 2>(p, qp, m, plan, tmap, steps_upper, st)
-                     : launch_decode_t<D, KB, VB, 1>(p, qp, m, plan, tmap, steps_upper, st);
+tq_status launch_decode_bits(const DecodeParams& p, const DecodePlan& plan,
+                             const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st) {
+  if (p.group > 8) return launch_decode_t<D, KB, VB, 2, 8>(p, plan, tmap, steps_upper, st);
+  if constexpr (D <= 128) return launch_decode_t<D, KB, VB, 1, 16>(p, plan, tmap, steps_upper, st);
+  else return launch_decode_t<D, KB, VB, 1, 8>(p, plan, tmap, steps_upper, st);
 }
 
 template <int D>
-tq_status launch_decode_dim(int kb, int vb, const DecodeParams& p, const QPrepParams& qp,
-                            const MergeParams& m, const DecodePlan& plan,
+tq_status launch_decode_dim(int kb, int vb, const DecodeParams& p, const DecodePlan& plan,
                             const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st) {
 #define TQ_BITS_CASE(KB_, VB_) \
   if (kb == KB_ && vb == VB_)  \
-    return launch_decode_bits<D, KB_, VB_>(p, qp, m, plan, tmap, steps_upper, st);
+    return launch_decode_bits<D, KB_, VB_>(p, plan, tmap, steps_upper, st);
   TQ_BITS_CASE(2, 2)
   TQ_BITS_CASE(3, 3)
   TQ_BITS_CASE(4, 4)
@@ -114,10 +117,9 @@ tq_status launch_decode_dim(int kb, int vb, const DecodeParams& p, const QPrepPa
   return TQ_ERR_UNSUPPORTED;
 }
 
-// Bytes of the replicated lookup table(s) of the decode kernel.
-inline size_t decode_lut_bytes(int kb, int vb, bool shared) {
-  auto one = [](int b) { return (size_t)(b <= 4 ? (1 << (2 * b)) : (1 << b)) * 32 * 4; };
-  return shared ? one(kb) : one(kb) + one(vb);
+// Bytes of the lookup tables of the decode kernel (one 256-byte row per entry).
+inline size_t decode_lut_bytes(int kb, int vb) {
+  return (size_t)std::max(lut_entries(kb), lut_entries(vb)) * kLutRow;
 }
 
 }  // namespace tq
