@@ -109,6 +109,28 @@ def ncu_traffic(kernel_name, config_name):
 
 
 # ---------------------------------------------------------------------------
+# ranks (one process per GPU; replicas, no data-path collective)
+# ---------------------------------------------------------------------------
+
+def max_over_ranks(values, device):
+    """Element-wise max of a list of floats over all ranks (identity when the
+    process group is not initialised).  Device-measured times are combined this
+    way: the job is as slow as its slowest rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_gbs(world, bytes_per_step, ms_per_step):
+    """Whole-job throughput: every rank processes its own replica of the step."""
+    return world * bytes_per_step / (ms_per_step * 1e-3) / 1e9
+
+
+# ---------------------------------------------------------------------------
 # clocks
 # ---------------------------------------------------------------------------
 
@@ -335,10 +357,7 @@ def run_gpu(args):
     total_ms = t_start.elapsed_time(t_end)
     app_ms = float(np.mean([a.elapsed_time(b) for a, b, _ in ev]))
     dec_ms = float(np.mean([b.elapsed_time(c) for _, b, c in ev]))
-    if world > 1:
-        tt = torch.tensor([total_ms, app_ms, dec_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms, app_ms, dec_ms = [float(x) for x in tt.tolist()]
+    total_ms, app_ms, dec_ms = max_over_ranks([total_ms, app_ms, dec_ms], dev)
     err = tq.get_device_error(stream)
     if err:
         raise RuntimeError(f"device error word {err:#x} during the bench")
@@ -378,12 +397,8 @@ def run_gpu(args):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
-        e2e = {"value": world * step_bytes * args.steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e2e_ms, = max_over_ranks([e0.elapsed_time(e1)], dev)
+        e2e = {"value": job_gbs(world, step_bytes, e2e_ms / args.steps), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms / args.steps}
 
@@ -395,7 +410,7 @@ def run_gpu(args):
 
     peak, peak_kind = measured_peaks()
     ms_per_step = total_ms / args.steps
-    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+    value = job_gbs(world, step_bytes, ms_per_step)
     app_gbs = a_bytes / (app_ms * 1e-3) / 1e9
     dec_gbs = d_bytes / (dec_ms * 1e-3) / 1e9
     dec_packed_gbs = d_packed / (dec_ms * 1e-3) / 1e9
