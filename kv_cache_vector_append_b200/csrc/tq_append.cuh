@@ -7,18 +7,20 @@
 // rotate, normalize, Lloyd-Max encode, bit-pack, store uint8).
 //
 // Work layout.  A row is one (token, KV head) vector of K or of V.  Every lane holds
-// 64 consecutive coordinates of a row in registers (D/64 lanes per row), so the FWHT
-// is six register stages plus log2(D/64) shuffle stages.  A warp owns a tile of
-// 32*64/D rows of one kind (K or V); lane l serves row l % ROWS, part l / ROWS, so
-// that each 8-lane phase of a 16-byte shared load touches 8 different rows (padded
-// pitch, no bank conflicts).  Input tiles are staged in shared memory by cp.async
-// (double-buffered per warp); packed regions are staged in shared memory and
-// written back one contiguous region per store instruction.
+// 64 consecutive coordinates of a row in 32 registers of fp32 pairs (D/64 lanes per
+// row), so the FWHT is six register stages (f32x2 add / sub: two fp32 operations per
+// instruction) plus log2(D/64) shuffle stages.  A warp owns a tile of 32*64/D
+// consecutive (token, KV head) pairs and does its K rows, then its V rows; lane l
+// serves row l % ROWS, part l / ROWS, so that each 8-lane phase of a 16-byte shared
+// load touches 8 different rows (padded pitch, no bank conflicts).  Input rows are
+// staged in shared memory by cp.async one half-tile ahead; the tile's full slots are
+// staged in shared memory and written back with lanes running over (slot, word), so
+// each slot's bytes go out together.
 //
 // Encode.  idx = #{i : b_i < u} over the fp32 boundaries.  For bits <= 4 (and when no
 // two boundaries share a bucket) the top 12 bits of u's float encoding (sign,
-// exponent, 3 mantissa bits) index a byte table k0 = #{b_i < lowest float of the
-// bucket}; one compare against b[k0] then gives idx exactly.  Otherwise a
+// exponent, 3 mantissa bits) index a byte table holding 4 k0, k0 = #{b_i < lowest
+// float of the bucket}; one compare against b[k0] then gives idx exactly.  Otherwise a
 // branch-free binary search over the boundaries in Eytzinger order.
 #pragma once
 
@@ -70,42 +72,44 @@ struct AppendGeom {
   static constexpr int E = 64;                        // elements per lane
   static constexpr int TPR = D / E;                   // lanes per row
   static constexpr int ROWS = 32 / TPR;               // rows per warp tile
-  static constexpr int MAXW = D * 8 / 32 + 1;         // packed words + norm, 8-bit
-  static constexpr int OUTPITCH = MAXW | 1;           // odd pitch: conflict-free
 };
 
-// Shared tables of one kind (K or V).
-struct alignas(16) EncodeTables {
-  uint8_t k0[kBuckets];     // #{b_i < lowest float of the bucket}
-  float bnd[257];           // boundaries b_0..b_{L-2}, then +inf
-  float eytz[256];          // Eytzinger image (t[0] unused)
-  int fast;                 // bucket encode valid for this table
+// Shared tables of one kind (K or V), 6 KiB.  The bucket of u is the top 12 bits of
+// its float encoding (sign, exponent, 3 mantissa bits); its byte holds 4 k0, where
+// k0 = #{b_i < lowest float of the bucket}.  The boundaries start 64-byte aligned, so
+// b[k0] sits at shared-window address (bnd address | 4 k0) for bits <= 4; one compare
+// against it then gives idx exactly.  Every 12-bit bucket has an entry.
+struct alignas(64) EncodeTables {
+  uint8_t k4[kBuckets];     // 4 * k0 per bucket
+  float bnd[257];           // boundaries b_0..b_{L-2}, then +inf (64-byte aligned)
+  float eytz[255];          // Eytzinger image, node e at eytz[e - 1]
 };
+static_assert(sizeof(EncodeTables) == 6144, "table layout");
 
-// Phase 1 (then a CTA barrier, then phase 2): boundaries, Eytzinger image, and the
-// check that no two boundaries share a bucket.
+// Phase 1 (then a CTA barrier, then phase 2): boundaries and Eytzinger image; thread 0
+// records whether the bucket encode applies (no two boundaries share a bucket, and
+// the boundaries are 64-byte aligned).
 __device__ __forceinline__ void build_tables(EncodeTables* t, const float* b, int bits, int tid,
-                                             int nthreads) {
+                                             int nthreads, int* fast) {
   const int n = (1 << bits) - 1;
   for (int i = tid; i <= n; i += nthreads) t->bnd[i] = i < n ? b[i] : INFINITY;
   for (int i = 1 + tid; i <= n; i += nthreads) {
     const int d = 31 - __clz(i);
     const int k = i - (1 << d);
-    t->eytz[i] = b[((2 * k + 1) << (bits - 1 - d)) - 1];
+    t->eytz[i - 1] = b[((2 * k + 1) << (bits - 1 - d)) - 1];
   }
   if (tid == 0) {
-    int ok = bits <= 4;
+    int ok = bits <= 4 && (smem_u32(t->bnd) & 63u) == 0;
     for (int i = 0; i + 1 < n; ++i)
       if ((__float_as_uint(b[i]) >> kBucketShift) == (__float_as_uint(b[i + 1]) >> kBucketShift))
         ok = 0;
-    t->fast = ok;
+    *fast = ok;
   }
 }
 
-// Phase 2: k0 of each bucket = #{b_i < lowest float of the bucket}, by binary search
-// over the boundaries already in shared memory.  The lowest float of bucket g is
-// g << 20 for a positive bucket and -((g & 0x7ff) << 20 | 0xfffff) for a negative one.
-// Only used for bits <= 4.
+// Phase 2: 4 k0 of each bucket (binary search over the boundaries already in shared
+// memory).  The lowest float of bucket g is g << 20 for a positive bucket and
+// -((g & 0x7ff) << 20 | 0xfffff) for a negative one.  Only used for bits <= 4.
 __device__ __forceinline__ void build_bucket_table(EncodeTables* t, int bits, int tid,
                                                    int nthreads) {
   if (bits > 4) return;
@@ -119,8 +123,14 @@ __device__ __forceinline__ void build_bucket_table(EncodeTables* t, int bits, in
       const int m = (a + c) >> 1;
       if (t->bnd[m] < lo) a = m + 1; else c = m;
     }
-    t->k0[g] = (uint8_t)a;
+    t->k4[g] = (uint8_t)(4 * a);
   }
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
 }
 
 // Stage `nrows` rows of RB bytes into shared memory (pitch `pitch`); row r starts at
@@ -149,142 +159,215 @@ __device__ __forceinline__ void stage_rows(uint8_t* dst, int pitch, int nrows, R
   }
 }
 
-// Load this lane's 64 input elements from shared memory as fp32 with the rotation
-// signs applied (the sign flip is an xor of the sign bit; for bf16 it rides along
-// with the widening: bits << 16 plus the mask, or the high half masked and xor-ed).
+// ---------------------------------------------------------------------------
+// Packed fp32 pairs.  A lane's 64 coordinates live in 32 64-bit registers, element
+// 2i in the low half of register i and 2i+1 in the high half; the add / sub / fma /
+// mul of two registers is one f32x2 instruction (two independent IEEE fp32
+// operations, each rounded to nearest even, so the results equal those of the
+// scalar operations).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float f2lo(uint64_t v) {
+  return __uint_as_float((uint32_t)v);
+}
+__device__ __forceinline__ float f2hi(uint64_t v) {
+  return __uint_as_float((uint32_t)(v >> 32));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// Load this lane's 64 input elements from shared memory as fp32 pairs with the
+// rotation signs applied (the sign flip is an xor of the sign bit; for bf16 it rides
+// along with the widening), and do the first FWHT stage (h = 1, the two halves of a
+// register): (a, b) -> (a + b, a - b).
 template <typename Tin>
-__device__ __forceinline__ void load_signed(float (&x)[64], const uint8_t* p,
+__device__ __forceinline__ void load_signed(uint64_t (&xp)[32], const uint8_t* p,
                                             const uint32_t* m) {
-  if constexpr (sizeof(Tin) == 4) {
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const uint4 q = *(const uint4*)(p + 16 * c);
-      const uint4 s = *(const uint4*)(m + 4 * c);
-      x[4 * c + 0] = __uint_as_float(q.x ^ s.x);
-      x[4 * c + 1] = __uint_as_float(q.y ^ s.y);
-      x[4 * c + 2] = __uint_as_float(q.z ^ s.z);
-      x[4 * c + 3] = __uint_as_float(q.w ^ s.w);
-    }
-  } else {
+  for (int c = 0; c < 8; ++c) {
+    float a[8];
+    const uint4 s0 = *(const uint4*)(m + 8 * c);
+    const uint4 s1 = *(const uint4*)(m + 8 * c + 4);
+    const uint32_t s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    if constexpr (sizeof(Tin) == 4) {
+      const uint4 q0 = *(const uint4*)(p + 32 * c);
+      const uint4 q1 = *(const uint4*)(p + 32 * c + 16);
+      const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+      for (int k = 0; k < 8; ++k) a[k] = __uint_as_float(w[k] ^ s[k]);
+    } else {
       const uint4 q = *(const uint4*)(p + 16 * c);
-      const uint4 s0 = *(const uint4*)(m + 8 * c);
-      const uint4 s1 = *(const uint4*)(m + 8 * c + 4);
       const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-      const uint32_t s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
-          x[8 * c + 2 * k + 0] = __uint_as_float((w[k] << 16) ^ s[2 * k]);
-          x[8 * c + 2 * k + 1] = __uint_as_float((w[k] & 0xFFFF0000u) ^ s[2 * k + 1]);
+          a[2 * k + 0] = __uint_as_float((w[k] << 16) ^ s[2 * k]);
+          a[2 * k + 1] = __uint_as_float((w[k] & 0xFFFF0000u) ^ s[2 * k + 1]);
         } else {
           __half2 h = *reinterpret_cast<const __half2*>(&w[k]);
           const float2 f = __half22float2(h);
-          x[8 * c + 2 * k + 0] = __uint_as_float(__float_as_uint(f.x) ^ s[2 * k]);
-          x[8 * c + 2 * k + 1] = __uint_as_float(__float_as_uint(f.y) ^ s[2 * k + 1]);
+          a[2 * k + 0] = __uint_as_float(__float_as_uint(f.x) ^ s[2 * k]);
+          a[2 * k + 1] = __uint_as_float(__float_as_uint(f.y) ^ s[2 * k + 1]);
         }
       }
     }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      xp[4 * c + k] = f2(__fadd_rn(a[2 * k], a[2 * k + 1]), __fsub_rn(a[2 * k], a[2 * k + 1]));
   }
 }
 
-// The rotation shared by quantize-append and its test export.  On entry x holds
+// The rotation shared by quantize-append and its test export.  On entry xp holds
 // this lane's 64 sign-flipped input elements (coordinates 64*part .. 64*part+63 of
-// the row); on exit x holds the unnormalised transform H (s * x) of those
-// coordinates, and the function returns r with u = x * r; *norm_out = ||x||_2.
+// the row) after the first butterfly stage (load_signed); on exit it holds the
+// unnormalised transform H (s * x) of those coordinates, and the function returns r
+// with u = x * r; *norm_out = ||x||_2.
 // Order of operations (fixed, so the export reproduces the kernel exactly):
-//   ss = sum of x_j^2 by fused multiply-add in coordinate order within a lane, then
-//   the lanes of a row add their sums pairwise (xor butterfly over the part bits);
-//   n = sqrt(ss) (IEEE); FWHT butterflies in stages h = 1, 2, 4, ..., D/2;
+//   FWHT butterflies in stages h = 1 (in load_signed), 2, 4, ..., 32 in registers, then
+//   h = 64, 128 across the lanes of the row; ss = sum of squares of the transformed
+//   coordinates: even and odd coordinates accumulated separately by fused
+//   multiply-add in register order, added, then the lanes of a row add their sums
+//   pairwise (xor butterfly over the part bits); n = sqrt(ss / D) (IEEE);
 //   r = 1 / (n * sqrt(D)) (IEEE reciprocal), or 0 when n == 0.
 template <int D>
-__device__ __forceinline__ float rotate_row(float (&x)[64], int part, float* norm_out) {
+__device__ __forceinline__ float rotate_row(uint64_t (&xp)[32], int part, float* norm_out) {
   using G = AppendGeom<D>;
-  float ss = 0.f;
 #pragma unroll
-  for (int j = 0; j < 64; ++j) ss = __fmaf_rn(x[j], x[j], ss);
+  for (int h = 1; h < 32; h <<= 1) {           // element stride 2h
 #pragma unroll
-  for (int m = 1; m < G::TPR; m <<= 1)
-    ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, G::ROWS * m));
-  const float n = sqrtf(ss);
-#pragma unroll
-  for (int h = 1; h < 64; h <<= 1) {
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {
+    for (int i = 0; i < 32; ++i) {
       if ((i & h) == 0) {
-        const float a = x[i], b = x[i + h];
-        x[i] = __fadd_rn(a, b);
-        x[i + h] = __fsub_rn(a, b);
+        const uint64_t a = xp[i], b = xp[i + h];
+        xp[i] = add2(a, b);
+        xp[i + h] = sub2(a, b);
       }
     }
   }
 #pragma unroll
   for (int m = 1; m < G::TPR; m <<= 1) {
+    const float sg = (part & m) ? -1.0f : 1.0f;
+    const uint64_t sg2 = f2(sg, sg);
 #pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      const float o = __shfl_xor_sync(0xffffffffu, x[i], G::ROWS * m);
-      x[i] = (part & m) ? __fsub_rn(o, x[i]) : __fadd_rn(x[i], o);
+    for (int i = 0; i < 32; ++i) {
+      const float olo = __shfl_xor_sync(0xffffffffu, f2lo(xp[i]), G::ROWS * m);
+      const float ohi = __shfl_xor_sync(0xffffffffu, f2hi(xp[i]), G::ROWS * m);
+      // part bit set: o - x; clear: x + o
+      xp[i] = fma2(xp[i], sg2, f2(olo, ohi));
     }
   }
+  uint64_t ss2 = 0ull;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) ss2 = fma2(xp[i], xp[i], ss2);
+  float ss = __fadd_rn(f2lo(ss2), f2hi(ss2));
+#pragma unroll
+  for (int m = 1; m < G::TPR; m <<= 1)
+    ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, G::ROWS * m));
+  // ||H s x||^2 = D ||x||^2
+  const float n = sqrtf(__fmul_rn(ss, 1.0f / D));
   *norm_out = n;
   const float sqrt_d = D == 64 ? 8.0f : (D == 128 ? 11.313708498984761f : 16.0f);
   return n > 0.f ? __frcp_rn(__fmul_rn(n, sqrt_d)) : 0.f;
 }
 
-// Encode u = x[j] * r and pack the 64 codes LSB-first into 2*BITS words.
+// Encode u = x * r and pack the 64 codes LSB-first into 2*BITS words.
 template <int BITS, bool FAST>
-__device__ __forceinline__ void encode_pack(const float (&x)[64], float r, const EncodeTables* t,
-                                            uint32_t* words) {
+__device__ __forceinline__ void encode_pack(const uint64_t (&xp)[32], float r,
+                                            const EncodeTables* t, uint32_t* words) {
   constexpr int W = 64 * BITS / 32;
   uint32_t acc[W];
 #pragma unroll
   for (int w = 0; w < W; ++w) acc[w] = 0u;
+  const uint64_t r2 = f2(r, r);
+  const uint32_t bnd_win = smem_u32(t->bnd);
 #pragma unroll
-  for (int j = 0; j < 64; ++j) {
-    const float u = __fmul_rn(x[j], r);
-    uint32_t code;
-    if constexpr (FAST) {
-      const uint32_t k0 = t->k0[__float_as_uint(u) >> kBucketShift];
-      code = k0 + (u > t->bnd[k0] ? 1u : 0u);
-    } else {
-      int i = 1;
+  for (int i = 0; i < 32; ++i) {
+    const uint64_t u2 = mul2(xp[i], r2);
 #pragma unroll
-      for (int s = 0; s < BITS; ++s) i = 2 * i + (u > t->eytz[i] ? 1 : 0);
-      code = (uint32_t)(i - (1 << BITS));
+    for (int hf = 0; hf < 2; ++hf) {
+      const float u = hf ? f2hi(u2) : f2lo(u2);
+      const int j = 2 * i + hf;
+      uint32_t code;
+      if constexpr (FAST) {
+        const uint32_t k4 = t->k4[__float_as_uint(u) >> kBucketShift];
+        code = (k4 + (u > lds_f32(bnd_win | k4) ? 4u : 0u)) >> 2;
+      } else {
+        int e = 1;
+#pragma unroll
+        for (int st = 0; st < BITS; ++st) e = 2 * e + (u > t->eytz[e - 1] ? 1 : 0);
+        code = (uint32_t)(e - (1 << BITS));
+      }
+      const int bit = j * BITS;
+      const int w0 = bit >> 5, o0 = bit & 31;
+      acc[w0] |= code << o0;
+      if (o0 + BITS > 32) acc[w0 + 1] |= code >> (32 - o0);
     }
-    const int bit = j * BITS;
-    const int w0 = bit >> 5, o0 = bit & 31;
-    acc[w0] |= code << o0;
-    if (o0 + BITS > 32) acc[w0 + 1] |= code >> (32 - o0);
   }
 #pragma unroll
   for (int w = 0; w < W; ++w) words[w] = acc[w];
 }
 
 template <int BITS>
-__device__ __forceinline__ void encode_pack_any(const float (&x)[64], float r,
-                                                const EncodeTables* t, uint32_t* words) {
+__device__ __forceinline__ void encode_pack_any(const uint64_t (&xp)[32], float r,
+                                                const EncodeTables* t, int fast,
+                                                uint32_t* words) {
   if constexpr (BITS <= 4) {
-    if (t->fast) {
-      encode_pack<BITS, true>(x, r, t, words);
+    if (fast) {
+      encode_pack<BITS, true>(xp, r, t, words);
       return;
     }
   }
-  encode_pack<BITS, false>(x, r, t, words);
+  encode_pack<BITS, false>(xp, r, t, words);
 }
 
+// Per-warp shared memory: K rows, V rows (one tile of ROWS (token, head) pairs each),
+// the tile's full slots (K region then V region; `out_pitch` words a slot, odd, sized
+// for the launch's bit widths), and the per-tile slot offsets and row addresses (two
+// tiles in flight).
 template <int D, typename Tin>
 struct AppendSmem {
   using G = AppendGeom<D>;
   static constexpr int RB = D * InType<Tin>::kBytes;
   static constexpr int INPITCH = RB + 16;
-  static constexpr int PER_WARP =
-      2 * G::ROWS * INPITCH + G::ROWS * G::OUTPITCH * 4 + 2 * G::ROWS * 8 + 2 * G::ROWS * 8;
-  static constexpr int TABLES = ((2 * (int)sizeof(EncodeTables) + 4 * D) + 127) / 128 * 128;
-  static constexpr int BYTES = TABLES + kAppendWarps * PER_WARP;
+  static constexpr int TABLES = ((2 * (int)sizeof(EncodeTables) + 4 * D + 8) + 127) / 128 * 128;
+  static __host__ __device__ constexpr int out_pitch(int kbits, int vbits) {
+    return ((D * kbits / 8 + 4 + D * vbits / 8 + 4) / 4) | 1;
+  }
+  static __host__ __device__ constexpr int per_warp(int out_pitch) {
+    return 2 * G::ROWS * INPITCH + 2 * G::ROWS * 8 + 2 * 2 * G::ROWS * 8 +
+           (G::ROWS * out_pitch * 4 + 15) / 16 * 16;
+  }
+  static __host__ __device__ constexpr int bytes(int kbits, int vbits) {
+    return TABLES + kAppendWarps * per_warp(out_pitch(kbits, vbits));
+  }
 };
 
+// Quantize-append.  A warp owns tiles of ROWS consecutive (token, KV head) pairs and
+// does both halves of each: the K rows, then the V rows (each row: D/64 lanes, 64
+// coordinates a lane), into the tile's slots staged in shared memory; then it writes
+// the full slots out (contiguous whole-slot stores, so every DRAM sector of a slot is
+// written by one store pass).  Input rows are staged by cp.async one half-tile ahead.
 template <int D, typename Tin>
 __global__ void __launch_bounds__(kAppendWarps * 32, 2)
 append_kernel(AppendParams p) {
@@ -293,31 +376,36 @@ append_kernel(AppendParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   EncodeTables* tabs = (EncodeTables*)smem;                       // [2]: K, V
   uint32_t* smask = (uint32_t*)(smem + 2 * sizeof(EncodeTables));  // D sign masks
+  int* fast = (int*)(smask + D);                                    // [2] bucket encode valid
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint8_t* in_s = smem + SM::TABLES + warp * SM::PER_WARP;
-  uint32_t* out_s = (uint32_t*)(in_s + 2 * G::ROWS * SM::INPITCH);
-  int64_t* dst_s = (int64_t*)(out_s + G::ROWS * G::OUTPITCH);     // [2][ROWS] region offsets
-  const uint8_t** src_s = (const uint8_t**)(dst_s + 2 * G::ROWS);  // [2][ROWS] row addresses
+  const int out_pitch = SM::out_pitch(p.bits[0], p.bits[1]);
+  uint8_t* in_s = smem + SM::TABLES + warp * SM::per_warp(out_pitch);   // [2 kinds][ROWS]
+  int64_t* dst_s = (int64_t*)(in_s + 2 * G::ROWS * SM::INPITCH);   // [2 tiles][ROWS] slots
+  const uint8_t** src_s = (const uint8_t**)(dst_s + 2 * G::ROWS);  // [2 tiles][2 kinds][ROWS]
+  uint32_t* out_s = (uint32_t*)(src_s + 2 * 2 * G::ROWS);          // [ROWS][out_pitch]
 
-  const int64_t rows_per_kind = p.num_tokens * p.h_kv;            // < 2^31 (host check)
-  const int64_t tiles_per_kind = (rows_per_kind + G::ROWS - 1) / G::ROWS;
-  const int64_t ntiles = 2 * tiles_per_kind;
+  const int64_t npairs = p.num_tokens * p.h_kv;                    // < 2^31 (host check)
+  const int64_t ntiles = (npairs + G::ROWS - 1) / G::ROWS;
   const int64_t gwarp = (int64_t)blockIdx.x * kAppendWarps + warp;
   const int64_t nwarps = (int64_t)gridDim.x * kAppendWarps;
+  const int kwords = (D * p.bits[0] + 7) / 8 / 4 + 1;             // K region words
+  const int vwords = (D * p.bits[1] + 7) / 8 / 4 + 1;
+  const int swords = kwords + vwords;                              // slot words written
 
-  // Stage tile `tile` into buffer `buf`: lane r < ROWS resolves row r0 + r once (its
-  // input address and its slot's region offset), then the warp copies the rows.
-  auto issue = [&](int64_t tile, int buf) {
-    const int kind = tile >= tiles_per_kind;
-    const int r0 = (int)((tile - kind * tiles_per_kind) * G::ROWS);
-    const int nr = (int)imin64((int64_t)G::ROWS, rows_per_kind - r0);
+  // Resolve tile `tile` (slot offsets, K and V row addresses; lane r < ROWS handles
+  // pair r0 + r) into slot `tb`.
+  auto resolve = [&](int64_t tile, int tb) {
+    const int r0 = (int)(tile * G::ROWS);
+    const int nr = (int)imin64((int64_t)G::ROWS, npairs - r0);
     if (lane < nr) {
       const uint32_t row = (uint32_t)(r0 + lane);
       const uint32_t t = row / (uint32_t)p.h_kv;
       const uint32_t h = row - t * (uint32_t)p.h_kv;
-      src_s[buf * G::ROWS + lane] =
-          (const uint8_t*)p.src[kind] +
-          ((int64_t)t * p.tok_stride[kind] + (int64_t)h * p.head_stride_in[kind]) * SM::RB / D;
+#pragma unroll
+      for (int kind = 0; kind < 2; ++kind)
+        src_s[(tb * 2 + kind) * G::ROWS + lane] =
+            (const uint8_t*)p.src[kind] +
+            ((int64_t)t * p.tok_stride[kind] + (int64_t)h * p.head_stride_in[kind]) * SM::RB / D;
       const int64_t slot = p.slot_mapping[(int64_t)t * p.slot_map_stride];
       int64_t off = -1;
       if (slot >= 0) {
@@ -330,23 +418,30 @@ append_kernel(AppendParams p) {
             blk = slot / p.block_size;
             rr = slot - blk * p.block_size;
           }
-          off = blk * p.blk_stride + rr * p.row_stride + h * p.head_stride + p.region_off[kind];
+          off = blk * p.blk_stride + rr * p.row_stride + h * p.head_stride;
         } else {
           report_error(p.err, TQ_DEVERR_SLOT_RANGE);
         }
       }
-      dst_s[buf * G::ROWS + lane] = off;
+      dst_s[tb * G::ROWS + lane] = off;
     }
     __syncwarp();
-    stage_rows<SM::RB>(in_s + buf * G::ROWS * SM::INPITCH, SM::INPITCH, nr,
-                       [&](int r) { return (const void*)src_s[buf * G::ROWS + r]; },
+  };
+  // Stage the `kind` rows of the tile resolved in slot tb into buffer `kind`.
+  auto stage = [&](int64_t tile, int tb, int kind) {
+    const int nr = (int)imin64((int64_t)G::ROWS, npairs - tile * G::ROWS);
+    stage_rows<SM::RB>(in_s + kind * G::ROWS * SM::INPITCH, SM::INPITCH, nr,
+                       [&](int r) { return (const void*)src_s[(tb * 2 + kind) * G::ROWS + r]; },
                        p.align_mode, lane);
   };
-  // the first tile's rows are in flight while the tables are built
-  if (gwarp < ntiles) issue(gwarp, 0);
+  // the first tile's K rows are in flight while the tables are built
+  if (gwarp < ntiles) {
+    resolve(gwarp, 0);
+    stage(gwarp, 0, 0);
+  }
   cp_async_commit();
-  build_tables(&tabs[0], p.boundaries[0], p.bits[0], threadIdx.x, blockDim.x);
-  build_tables(&tabs[1], p.boundaries[1], p.bits[1], threadIdx.x, blockDim.x);
+  build_tables(&tabs[0], p.boundaries[0], p.bits[0], threadIdx.x, blockDim.x, &fast[0]);
+  build_tables(&tabs[1], p.boundaries[1], p.bits[1], threadIdx.x, blockDim.x, &fast[1]);
   for (int j = threadIdx.x; j < D; j += blockDim.x) smask[j] = sign_mask_at(p.sign_seed, j);
   __syncthreads();
   build_bucket_table(&tabs[0], p.bits[0], threadIdx.x, blockDim.x);
@@ -355,57 +450,67 @@ append_kernel(AppendParams p) {
 
   const int rl = lane % G::ROWS;           // row within the tile
   const int part = lane / G::ROWS;         // which 64 coordinates of the row
-  int buf = 0;
+  int tb = 0;
   for (int64_t tile = gwarp; tile < ntiles; tile += nwarps) {
+    const int nr = (int)imin64((int64_t)G::ROWS, npairs - tile * G::ROWS);
     const int64_t next = tile + nwarps;
-    if (next < ntiles) issue(next, buf ^ 1);
-    cp_async_commit();
-    const int kind = tile >= tiles_per_kind;
-    const int64_t r0 = (tile - kind * tiles_per_kind) * G::ROWS;
-    const int nr = (int)imin64((int64_t)G::ROWS, rows_per_kind - r0);
-    const int bits = p.bits[kind];
-    const int nw = D * bits / 32 + 1;   // packed words + norm word
-    cp_async_wait<1>();
-    __syncwarp();
-    {
-      float x[64];
-      load_signed<Tin>(x, in_s + buf * G::ROWS * SM::INPITCH + rl * SM::INPITCH +
-                              part * 64 * InType<Tin>::kBytes,
+#pragma unroll 1
+    for (int kind = 0; kind < 2; ++kind) {
+      // prefetch one half-tile ahead: this tile's V rows, or the next tile's K rows
+      if (kind == 0) {
+        stage(tile, tb, 1);
+      } else if (next < ntiles) {
+        resolve(next, tb ^ 1);
+        stage(next, tb ^ 1, 0);
+      }
+      cp_async_commit();
+      cp_async_wait<1>();
+      __syncwarp();
+      const int bits = p.bits[kind];
+      const int rwords = kind ? vwords : kwords;          // packed words + norm word
+      uint64_t xp[32];
+      load_signed<Tin>(xp, in_s + kind * G::ROWS * SM::INPITCH + rl * SM::INPITCH +
+                               part * 64 * InType<Tin>::kBytes,
                        smask + part * 64);
       float n;
-      const float r = rotate_row<D>(x, part, &n);
+      const float r = rotate_row<D>(xp, part, &n);
       const bool bad = !(fabsf(n) <= 3.402823466e38f);   // inf or NaN
-      uint32_t* orow = out_s + rl * G::OUTPITCH;
+      uint32_t* orow = out_s + rl * out_pitch + (kind ? kwords : 0);
       const EncodeTables* t = &tabs[kind];
-      const int wpl = (nw - 1) / G::TPR;                  // words per lane
+      const int wpl = (rwords - 1) / G::TPR;               // words per lane
       uint32_t* mine = orow + part * wpl;
-      switch (bits) {
-        case 1: encode_pack_any<1>(x, r, t, mine); break;
-        case 2: encode_pack_any<2>(x, r, t, mine); break;
-        case 3: encode_pack_any<3>(x, r, t, mine); break;
-        case 4: encode_pack_any<4>(x, r, t, mine); break;
-        case 5: encode_pack_any<5>(x, r, t, mine); break;
-        case 6: encode_pack_any<6>(x, r, t, mine); break;
-        case 7: encode_pack_any<7>(x, r, t, mine); break;
-        default: encode_pack_any<8>(x, r, t, mine); break;
-      }
-      if (bad) {
+      if (!bad) {
+        const int use_fast = fast[kind];
+        switch (bits) {
+          case 1: encode_pack_any<1>(xp, r, t, use_fast, mine); break;
+          case 2: encode_pack_any<2>(xp, r, t, use_fast, mine); break;
+          case 3: encode_pack_any<3>(xp, r, t, use_fast, mine); break;
+          case 4: encode_pack_any<4>(xp, r, t, use_fast, mine); break;
+          case 5: encode_pack_any<5>(xp, r, t, use_fast, mine); break;
+          case 6: encode_pack_any<6>(xp, r, t, use_fast, mine); break;
+          case 7: encode_pack_any<7>(xp, r, t, use_fast, mine); break;
+          default: encode_pack_any<8>(xp, r, t, use_fast, mine); break;
+        }
+      } else {
         for (int w = 0; w < wpl; ++w) mine[w] = 0u;
         if (part == 0 && rl < nr) report_error(p.err, TQ_DEVERR_NONFINITE);
       }
-      if (part == G::TPR - 1) orow[nw - 1] = bad ? 0x7FC00000u : __float_as_uint(n);
+      if (part == G::TPR - 1) orow[rwords - 1] = bad ? 0x7FC00000u : __float_as_uint(n);
+      __syncwarp();
+    }
+    // write back the tile's full slots: lanes run over (pair, word)
+    {
+      int rr = 0, w = lane;
+      while (w >= swords) { w -= swords; ++rr; }
+      for (; rr < nr;) {
+        const int64_t off = dst_s[tb * G::ROWS + rr];
+        if (off >= 0) ((uint32_t*)(p.pages + off))[w] = out_s[rr * out_pitch + w];
+        w += 32;
+        while (w >= swords) { w -= swords; ++rr; }
+      }
     }
     __syncwarp();
-    // write back: one row region per pass (contiguous words)
-    for (int rr = 0; rr < nr; ++rr) {
-      const int64_t off = dst_s[buf * G::ROWS + rr];
-      if (off < 0) continue;
-      uint32_t* dst = (uint32_t*)(p.pages + off);
-      const uint32_t* src = out_s + rr * G::OUTPITCH;
-      for (int w = lane; w < nw; w += 32) dst[w] = src[w];
-    }
-    __syncwarp();
-    buf ^= 1;
+    tb ^= 1;
   }
   cp_async_wait<0>();
 }
@@ -436,14 +541,20 @@ rotate_unit_kernel(RotateParams p) {
     cp_async_commit();
     cp_async_wait<0>();
     __syncwarp();
-    float x[64];
-    load_signed<Tin>(x, in_s + rl * INPITCH + part * 64 * InType<Tin>::kBytes, smask + part * 64);
+    uint64_t xp[32];
+    load_signed<Tin>(xp, in_s + rl * INPITCH + part * 64 * InType<Tin>::kBytes,
+                     smask + part * 64);
     float n;
-    const float r = rotate_row<D>(x, part, &n);
+    const float r = rotate_row<D>(xp, part, &n);
     if (rl < nr) {
       float* u = p.u + (r0 + rl) * p.u_row_stride + part * 64;
+      const uint64_t r2 = f2(r, r);
 #pragma unroll
-      for (int j = 0; j < 64; ++j) u[j] = __fmul_rn(x[j], r);
+      for (int i = 0; i < 32; ++i) {
+        const uint64_t u2 = mul2(xp[i], r2);
+        u[2 * i] = f2lo(u2);
+        u[2 * i + 1] = f2hi(u2);
+      }
       if (part == 0) p.norm[(r0 + rl) * p.norm_stride] = n;
     }
     __syncwarp();

@@ -8,14 +8,14 @@ namespace tq {
 
 template <int D, typename Tin>
 tq_status launch_append_t(const AppendParams& p, const DeviceInfo& di, cudaStream_t st) {
-  const size_t smem = AppendSmem<D, Tin>::BYTES;
+  const size_t smem = AppendSmem<D, Tin>::bytes(p.bits[0], p.bits[1]);
   if ((int)smem > di.max_smem_optin) return TQ_ERR_UNSUPPORTED;
   auto kern = append_kernel<D, Tin>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return TQ_ERR_CUDA;
   using G = AppendGeom<D>;
-  const int64_t tiles = 2 * ((p.num_tokens * p.h_kv + G::ROWS - 1) / G::ROWS);
+  const int64_t tiles = (p.num_tokens * p.h_kv + G::ROWS - 1) / G::ROWS;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kAppendWarps * 32, smem) !=
       cudaSuccess)

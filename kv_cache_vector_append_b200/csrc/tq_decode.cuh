@@ -17,9 +17,10 @@
 // the contiguous range [c S/C, (c+1) S/C) of the S steps (stream-K style), so ragged
 // batches and single long sequences balance alike.  Inside a CTA one warp serves one
 // (KV head, sub-stream):
-//   * when its range enters a sequence the CTA rotates that sequence's queries (sign
-//     flips, FWHT in registers and shuffles, 1/sqrt(D)) into shared memory as unit
-//     fp16 vectors plus |q'| * scale * log2 e;
+//   * a CTA walks its range as segments, one per sequence; at the start of a segment
+//     the CTA rotates that sequence's queries (sign flips, FWHT in registers and
+//     shuffles, 1/sqrt(D)) into shared memory as unit fp16 vectors plus
+//     |q'| * scale * log2 e, and each warp loads its fragments;
 //   * page blocks (16 tokens x all KV heads; one per sub-stream and step) are staged
 //     into shared memory by one TMA copy each (a 2-D box of 16 rows one padding wider
 //     than a row, the padding zero-filled out of bounds, or a 1-D bulk copy) into a
@@ -28,9 +29,10 @@
 //     makes the per-thread code loads bank-conflict free;
 //   * codes become fp16 through shared-memory tables with one 256-byte row per entry
 //     (the K table in the first 128 bytes of a row, the V table in the second, lane l
-//     at byte 4l), so a warp's lookups always hit 32 different banks and the address of
-//     a lookup keyed by a whole byte of codes is one byte permute; tables hold code
-//     PAIRS for bits <= 4 (entry x | y << bits = (c[x], c[y])), single codes for 8 bits;
+//     at byte 4l), so a warp's lookups always hit 32 different banks; the tables sit at
+//     a 64 KiB-aligned shared-window address, so the address of a lookup keyed by a
+//     whole byte of codes is one byte permute; tables hold code PAIRS for bits <= 4
+//     (entry x | y << bits = (c[x], c[y])), single codes for 8 bits;
 //   * S^T = K~ . Qhat^T on mma.sync m16n8k16 (M = 16 tokens, N = 8 query heads of the
 //     group, K = D; fp16 operands, fp32 accumulation); s = acc * nK * |q'| * scale * log2 e;
 //   * online softmax in base 2 against a running reference M >= max(s + e(nV)),
@@ -40,12 +42,13 @@
 //   * O'^T += V~^T . P~^T on mma.sync (M = coordinates, N = query heads, K = tokens);
 //     the fp16 weights go from the C layout of S^T to the B layout of P~^T with one
 //     movmatrix transpose per 8 x 8 tile;
-//   * when its range leaves a sequence every warp writes its partial (M, l, O') to
-//     record ((CTA + sequence) * wph + sub-stream), an index no other (CTA, sequence)
-//     pair shares because the ranges are monotone; the CTA then takes a ticket on the
-//     sequence's counter, and the CTA holding the last ticket combines the records of
-//     the sequence, divides by l and applies the inverse rotation, while the others
-//     move on.
+//   * at the end of a segment every warp writes its partial (M, l, O') to record
+//     ((CTA + sequence) * wph + sub-stream), an index no other (CTA, sequence) pair
+//     shares because the ranges are monotone;
+//   * end phase: the CTA counts its records on each sequence's counter, waits (bounded)
+//     until every CTA covering the sequence has done so, and merges a share of the
+//     sequence's query heads: divide by l, then o = R^T O' (FWHT, 1/sqrt(D), sign
+//     flips).  The launch is cooperative, so the CTAs that wait are co-resident.
 // The coordinate order inside each mma tile is free (a permutation applied to both
 // operands of a contraction leaves it unchanged); it is chosen so that every thread
 // reads whole 32-bit words of codes, and undone when O' is written to its record.
@@ -357,8 +360,8 @@ __device__ __forceinline__ void store_from_f32(void* base, int64_t i, int32_t dt
 }
 
 // Shared memory: stages below and above the tables (see DecodeParams), and a misc
-// area [full mbarriers | release counters | present masks | q' (H_q x D fp16) |
-// |q'| scales | step prefix sums | block ids | scan scratch | flag | merge partials].
+// area [full mbarriers | release counters | present masks | q' (H_q x D fp16) | |q'|
+// scales | step prefix sums | block ids | scan scratch | flag | merge partials].
 template <int D, int KB, int VB, int NH, int MAXW>
 __global__ void __launch_bounds__(MAXW * 32, 1)
 decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
@@ -531,34 +534,6 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     for (int i = 0; i < nst && s0 + i < s1; ++i) refill(s0 + i, i);
 
 
-  // q' = R q of the query heads of sequence b into qh / qsc (the warps split the heads)
-  auto rotate_q = [&](int b) {
-    uint32_t sg[E];
-#pragma unroll
-    for (int i = 0; i < E; ++i) sg[i] = sign_mask_at(p.sign_seed, lane * E + i);
-    for (int h = warp; h < p.h_q; h += nwarps) {
-      const int64_t off = (int64_t)b * p.q_bstride + (int64_t)h * p.q_hstride + lane * E;
-      float x[E];
-#pragma unroll
-      for (int i = 0; i < E; ++i)
-        x[i] = __uint_as_float(__float_as_uint(load_as_f32(p.q, off + i, p.q_dtype)) ^ sg[i]);
-      warp_fwht<E>(x, lane);
-      float ss = 0.f;
-#pragma unroll
-      for (int i = 0; i < E; ++i) {
-        x[i] *= inv_sqrt_dim<D>();
-        ss = fmaf(x[i], x[i], ss);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      const float nrm = sqrtf(ss);
-      const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
-#pragma unroll
-      for (int i = 0; i < E; ++i) qh[h * D + lane * E + i] = __float2half_rn(x[i] * inv);
-      if (lane == 0) qsc[h] = nrm * p.scale_log2;
-    }
-  };
-
   const int kvh = warp % p.h_kv;
   const int sub = warp / p.h_kv;
   const int G = p.group;
@@ -570,7 +545,38 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   float Mrun[NH][2], lrun[NH][2];
   float acc[NH][C::MT][4];
 
-  auto start = [&]() {
+  // Start sequence b (all warps): q' = R q of its query heads into shared memory, the
+  // warps splitting the heads (lane l holds coordinates l E .. l E + E - 1: sign flips,
+  // FWHT in registers and shuffles, 1/sqrt(D), then normalised to unit fp16), then
+  // every warp reads its B fragments and scales and resets its softmax state and O'.
+  // Two CTA barriers; called where all warps are between segments.
+  auto start = [&](int b) {
+    __syncthreads();                    // the previous segment's q' is no longer read
+    uint32_t sg[E];
+#pragma unroll
+    for (int i = 0; i < E; ++i) sg[i] = sign_mask_at(p.sign_seed, lane * E + i);
+    for (int h = warp; h < p.h_q; h += nwarps) {
+      const int64_t off = (int64_t)b * p.q_bstride + (int64_t)h * p.q_hstride + lane * E;
+      float xq[E];
+#pragma unroll
+      for (int i = 0; i < E; ++i)
+        xq[i] = __uint_as_float(__float_as_uint(load_as_f32(p.q, off + i, p.q_dtype)) ^ sg[i]);
+      warp_fwht<E>(xq, lane);
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        xq[i] *= inv_sqrt_dim<D>();
+        ss = fmaf(xq[i], xq[i], ss);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float nrm = sqrtf(ss);
+      const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
+#pragma unroll
+      for (int i = 0; i < E; ++i) qh[h * D + lane * E + i] = __float2half_rn(xq[i] * inv);
+      if (lane == 0) qsc[h] = nrm * p.scale_log2;
+    }
+    __syncthreads();
 #pragma unroll
     for (int hh = 0; hh < NH; ++hh) {
       const int g = 8 * hh + gid;
@@ -781,220 +787,203 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     }
   };
 
-  // Leave sequence b for nb (the next sequence of the range): write the records of b,
-  // count them on b's counter, rotate the queries of nb.
-  auto boundary = [&](int b, int nb) {
-    flush(b);
-    __syncthreads();                    // records of b written; q' of b no longer read
-    if (tid == 0) {
-      __threadfence();
-      atomicAdd(&arrived[b], 1u);
-    }
-    rotate_q(nb);
-    __syncthreads();
-    start();
-  };
-
-  int cur_b = locate(s0);
-  int local = (int)(s0 - prefix[cur_b]);
-  int cur_len = p.seq_lens[cur_b];
-  rotate_q(cur_b);
-  __syncthreads();                      // tables and q' ready
-  start();
-
+  // Outer loop: the segments (one per sequence) of this CTA's step range; inner loop:
+  // the steps of a segment.  Segment set-up and write-out stay out of the step loop.
+  const int b_first = locate(s0);
+  int cur_b = b_first;
   int x = 0;
   uint32_t phase = 0;
   bool dead = false;                    // a stage wait of this warp gave up
-  for (int64_t s = s0; s < s1; ++s) {
-    if (!dead && !mbar_wait(&full[x], phase, kWaitMs)) {
-      if (lane == 0) {
-        report_error(p.err, TQ_DEVERR_TIMEOUT);
-        *timed_out = 1;
+  for (int64_t s = s0;;) {
+    const int64_t seg_end = imin64(s1, prefix[cur_b + 1]);
+    const int cur_len = p.seq_lens[cur_b];
+    int bi = (int)(s - prefix[cur_b]) * wph + sub;    // this warp's block in the sequence
+    start(cur_b);
+    for (; s < seg_end; ++s, bi += wph) {
+      if (!dead && !mbar_wait(&full[x], phase, kWaitMs)) {
+        if (lane == 0) {
+          report_error(p.err, TQ_DEVERR_TIMEOUT);
+          *timed_out = 1;
+        }
+        dead = true;
       }
-      dead = true;
-    }
-    const int bi = local * wph + sub;                 // this warp's block
-    const int valid =
-        (!dead && ((present[x] >> sub) & 1u)) ? min(kBlockSize, cur_len - bi * kBlockSize) : 0;
-    if (valid > 0) {
-      const uint8_t* base = stage_ptr(x) + sub * blk_smem + kvh * p.slot_stride;
-      // token t (0..15) of this block lives at base + t * pitch
+      const int valid =
+          (!dead && ((present[x] >> sub) & 1u)) ? min(kBlockSize, cur_len - bi * kBlockSize) : 0;
+      if (valid > 0) {
+        const uint8_t* base = stage_ptr(x) + sub * blk_smem + kvh * p.slot_stride;
+        // token t (0..15) of this block lives at base + t * pitch
 
-      // ---- S^T = K~ . Qhat^T: one m-tile of 16 tokens ----
-      float sacc[NH][4];
-#pragma unroll
-      for (int hh = 0; hh < NH; ++hh)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) sacc[hh][k] = 0.f;
-      {
-        uint32_t kw0[KS::NW], kw1[KS::NW];
-        KS::load(kw0, base + gid * pitch, tig);
-        KS::load(kw1, base + (gid + 8) * pitch, tig);
-        static_for<C::KSTEPS>([&](auto KSI) {
-          constexpr int ks = decltype(KSI)::value;
-          const uint32_t a0 = lut_pair<KB, KS::pos(4 * ks)>(kw0, lk_off);
-          const uint32_t a1 = lut_pair<KB, KS::pos(4 * ks)>(kw1, lk_off);
-          const uint32_t a2 = lut_pair<KB, KS::pos(4 * ks + 2)>(kw0, lk_off);
-          const uint32_t a3 = lut_pair<KB, KS::pos(4 * ks + 2)>(kw1, lk_off);
-#pragma unroll
-          for (int hh = 0; hh < NH; ++hh)
-            mma_16816(sacc[hh], a0, a1, a2, a3, qb[ks][hh][0], qb[ks][hh][1]);
-        });
-      }
-      // this thread's tokens: r = 0, 1  <->  token gid + 8 r
-      float nK[2], nV[2], eV[2];
-      bool ok[2];
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int t = gid + 8 * r;
-        const uint8_t* sl = base + t * pitch;
-        ok[r] = t < valid;
-        nK[r] = *(const float*)(sl + C::KPACK);
-        // masked tokens may hold stale norms (even NaN): their V norm is taken as 0
-        nV[r] = ok[r] ? *(const float*)(sl + p.k_region + C::VPACK) : 0.f;
-        // floor at 2^-100 keeps 2^(s - M) finite for rows of (near) zero V norm
-        eV[r] = fmaxf(log2_ceilish(nV[r]), -100.0f);
-      }
-      uint32_t pb[NH][2];   // [head group][b0b1 | b2b3]
-#pragma unroll
-      for (int hh = 0; hh < NH; ++hh) {
-        float sv[2][2];        // [head e][token r]
-        float zloc[2];         // this thread's max of s + e(nV) per head
-        bool need = false;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          zloc[e] = -INFINITY;
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const float a = sacc[hh][2 * r + e];
-            sv[e][r] = ok[r] ? a * nK[r] * qscale[hh][e] : -INFINITY;
-            zloc[e] = fmaxf(zloc[e], sv[e][r] + eV[r]);
-          }
-          need |= zloc[e] > Mrun[hh][e] + kLazyRescale;
+        // ---- S^T = K~ . Qhat^T: one m-tile of 16 tokens ----
+        float sacc[NH][4];
+  #pragma unroll
+        for (int hh = 0; hh < NH; ++hh)
+  #pragma unroll
+          for (int k = 0; k < 4; ++k) sacc[hh][k] = 0.f;
+        {
+          uint32_t kw0[KS::NW], kw1[KS::NW];
+          KS::load(kw0, base + gid * pitch, tig);
+          KS::load(kw1, base + (gid + 8) * pitch, tig);
+          static_for<C::KSTEPS>([&](auto KSI) {
+            constexpr int ks = decltype(KSI)::value;
+            const uint32_t a0 = lut_pair<KB, KS::pos(4 * ks)>(kw0, lk_off);
+            const uint32_t a1 = lut_pair<KB, KS::pos(4 * ks)>(kw1, lk_off);
+            const uint32_t a2 = lut_pair<KB, KS::pos(4 * ks + 2)>(kw0, lk_off);
+            const uint32_t a3 = lut_pair<KB, KS::pos(4 * ks + 2)>(kw1, lk_off);
+  #pragma unroll
+            for (int hh = 0; hh < NH; ++hh)
+              mma_16816(sacc[hh], a0, a1, a2, a3, qb[ks][hh][0], qb[ks][hh][1]);
+          });
         }
-        // lazy reference: raise M only when the tile beats it by more than 2^8 (the
-        // tile maxima over the 16 tokens are only formed when some lane needs them)
-        if (__any_sync(0xffffffffu, need)) {
-          float zmax[2];
-#pragma unroll
+        // this thread's tokens: r = 0, 1  <->  token gid + 8 r
+        float nK[2], nV[2], eV[2];
+        bool ok[2];
+  #pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int t = gid + 8 * r;
+          const uint8_t* sl = base + t * pitch;
+          ok[r] = t < valid;
+          nK[r] = *(const float*)(sl + C::KPACK);
+          // masked tokens may hold stale norms (even NaN): their V norm is taken as 0
+          nV[r] = ok[r] ? *(const float*)(sl + p.k_region + C::VPACK) : 0.f;
+          // floor at 2^-100 keeps 2^(s - M) finite for rows of (near) zero V norm
+          eV[r] = fmaxf(log2_ceilish(nV[r]), -100.0f);
+        }
+        uint32_t pb[NH][2];   // [head group][b0b1 | b2b3]
+  #pragma unroll
+        for (int hh = 0; hh < NH; ++hh) {
+          float sv[2][2];        // [head e][token r]
+          float zloc[2];         // this thread's max of s + e(nV) per head
+          bool need = false;
+  #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            zmax[e] = zloc[e];
-#pragma unroll
-            for (int o = 4; o < 32; o <<= 1)
-              zmax[e] = fmaxf(zmax[e], __shfl_xor_sync(0xffffffffu, zmax[e], o));
+            zloc[e] = -INFINITY;
+  #pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              const float a = sacc[hh][2 * r + e];
+              sv[e][r] = ok[r] ? a * nK[r] * qscale[hh][e] : -INFINITY;
+              zloc[e] = fmaxf(zloc[e], sv[e][r] + eV[r]);
+            }
+            need |= zloc[e] > Mrun[hh][e] + kLazyRescale;
           }
-          const bool raise0 = zmax[0] > Mrun[hh][0] + kLazyRescale;
-          const bool raise1 = zmax[1] > Mrun[hh][1] + kLazyRescale;
-          float alpha[2];
-#pragma unroll
+          // lazy reference: raise M only when the tile beats it by more than 2^8 (the
+          // tile maxima over the 16 tokens are only formed when some lane needs them)
+          if (__any_sync(0xffffffffu, need)) {
+            float zmax[2];
+  #pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              zmax[e] = zloc[e];
+  #pragma unroll
+              for (int o = 4; o < 32; o <<= 1)
+                zmax[e] = fmaxf(zmax[e], __shfl_xor_sync(0xffffffffu, zmax[e], o));
+            }
+            const bool raise0 = zmax[0] > Mrun[hh][0] + kLazyRescale;
+            const bool raise1 = zmax[1] > Mrun[hh][1] + kLazyRescale;
+            float alpha[2];
+  #pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const bool raise = e ? raise1 : raise0;
+              const float Mnew = raise ? zmax[e] : Mrun[hh][e];
+              alpha[e] = (Mrun[hh][e] == -INFINITY) ? 0.f : exp2f(Mrun[hh][e] - Mnew);
+              lrun[hh][e] *= alpha[e];
+              Mrun[hh][e] = Mnew;
+            }
+  #pragma unroll
+            for (int mt = 0; mt < C::MT; ++mt) {
+              acc[hh][mt][0] *= alpha[0]; acc[hh][mt][1] *= alpha[1];
+              acc[hh][mt][2] *= alpha[0]; acc[hh][mt][3] *= alpha[1];
+            }
+          }
+          float pv[2][2];
+  #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const bool raise = e ? raise1 : raise0;
-            const float Mnew = raise ? zmax[e] : Mrun[hh][e];
-            alpha[e] = (Mrun[hh][e] == -INFINITY) ? 0.f : exp2f(Mrun[hh][e] - Mnew);
-            lrun[hh][e] *= alpha[e];
-            Mrun[hh][e] = Mnew;
+            const float M = Mrun[hh][e];
+            float lsum = 0.f;
+  #pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              const float w = ex2_approx(sv[e][r] - M);   // exactly 0 for masked tokens
+              lsum += w;
+              pv[e][r] = w * nV[r];
+            }
+            lrun[hh][e] += lsum;
           }
-#pragma unroll
-          for (int mt = 0; mt < C::MT; ++mt) {
-            acc[hh][mt][0] *= alpha[0]; acc[hh][mt][1] *= alpha[1];
-            acc[hh][mt][2] *= alpha[0]; acc[hh][mt][3] *= alpha[1];
-          }
+          // P~ (token, head) pairs in the C layout, transposed to the B layout of P~^T:
+          // b0b1 <- tokens 0..7, b2b3 <- tokens 8..15
+          pb[hh][0] = movmatrix_trans(pack_half2(pv[0][0], pv[1][0]));
+          pb[hh][1] = movmatrix_trans(pack_half2(pv[0][1], pv[1][1]));
         }
-        float pv[2][2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float M = Mrun[hh][e];
-          float lsum = 0.f;
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const float w = ex2_approx(sv[e][r] - M);   // exactly 0 for masked tokens
-            lsum += w;
-            pv[e][r] = w * nV[r];
-          }
-          lrun[hh][e] += lsum;
-        }
-        // P~ (token, head) pairs in the C layout, transposed to the B layout of P~^T:
-        // b0b1 <- tokens 0..7, b2b3 <- tokens 8..15
-        pb[hh][0] = movmatrix_trans(pack_half2(pv[0][0], pv[1][0]));
-        pb[hh][1] = movmatrix_trans(pack_half2(pv[0][1], pv[1][1]));
-      }
 
-      // ---- O'^T += V~^T . P~^T : one k-step of 16 tokens ----
-      {
-        uint32_t vw[4][VS::NW];   // tokens A, B, C, D = 2tig + {0, 1, 8, 9}
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int t = 2 * tig + (i & 1) + 8 * (i >> 1);
-          VS::load(vw[i], base + t * pitch + p.k_region, gid);
-        }
-        if constexpr (VS::kInterleaved && (VB == 4 || VB == 2)) {
-          // transpose the code nibbles (or crumbs) of tokens A/B and C/D into pair
-          // indices: lo holds the even codes of a word, hi the odd ones
-          constexpr uint32_t M1 = VB == 4 ? 0x0F0F0F0Fu : 0x33333333u;
-          static_for<VS::NW>([&](auto JI) {
-            constexpr int j = decltype(JI)::value;
-            const uint32_t loAB = (vw[0][j] & M1) | ((vw[1][j] << VB) & ~M1);
-            const uint32_t hiAB = ((vw[0][j] >> VB) & M1) | (vw[1][j] & ~M1);
-            const uint32_t loCD = (vw[2][j] & M1) | ((vw[3][j] << VB) & ~M1);
-            const uint32_t hiCD = ((vw[2][j] >> VB) & M1) | (vw[3][j] & ~M1);
-            constexpr int PER = VS::PW / 2;            // m-tiles per word
-            static_for<PER>([&](auto KI) {
-              constexpr int k = decltype(KI)::value;
-              constexpr int mt = j * PER + k;
-              const uint32_t a0 = lut_ld(lut_addr1<2 * VB * k, 2 * VB>(loAB, lv_off));
-              const uint32_t a1 = lut_ld(lut_addr1<2 * VB * k, 2 * VB>(hiAB, lv_off));
-              const uint32_t a2 = lut_ld(lut_addr1<2 * VB * k, 2 * VB>(loCD, lv_off));
-              const uint32_t a3 = lut_ld(lut_addr1<2 * VB * k, 2 * VB>(hiCD, lv_off));
-#pragma unroll
+        // ---- O'^T += V~^T . P~^T : one k-step of 16 tokens ----
+        {
+          uint32_t vw[4][VS::NW];   // tokens A, B, C, D = 2tig + {0, 1, 8, 9}
+  #pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int t = 2 * tig + (i & 1) + 8 * (i >> 1);
+            VS::load(vw[i], base + t * pitch + p.k_region, gid);
+          }
+          if constexpr (VS::kInterleaved && (VB == 4 || VB == 2)) {
+            // transpose the code nibbles (or crumbs) of tokens A/B and C/D into pair
+            // indices: lo holds the even codes of a word, hi the odd ones
+            constexpr uint32_t M1 = VB == 4 ? 0x0F0F0F0Fu : 0x33333333u;
+            static_for<VS::NW>([&](auto JI) {
+              constexpr int j = decltype(JI)::value;
+              const uint32_t loAB = (vw[0][j] & M1) | ((vw[1][j] << VB) & ~M1);
+              const uint32_t hiAB = ((vw[0][j] >> VB) & M1) | (vw[1][j] & ~M1);
+              const uint32_t loCD = (vw[2][j] & M1) | ((vw[3][j] << VB) & ~M1);
+              const uint32_t hiCD = ((vw[2][j] >> VB) & M1) | (vw[3][j] & ~M1);
+              constexpr int PER = VS::PW / 2;            // m-tiles per word
+              static_for<PER>([&](auto KI) {
+                constexpr int k = decltype(KI)::value;
+                constexpr int mt = j * PER + k;
+                const uint32_t a0 = lut_ld(lut_addr1<2 * VB * k, 2 * VB>(loAB, lv_off));
+                const uint32_t a1 = lut_ld(lut_addr1<2 * VB * k, 2 * VB>(hiAB, lv_off));
+                const uint32_t a2 = lut_ld(lut_addr1<2 * VB * k, 2 * VB>(loCD, lv_off));
+                const uint32_t a3 = lut_ld(lut_addr1<2 * VB * k, 2 * VB>(hiCD, lv_off));
+  #pragma unroll
+                for (int hh = 0; hh < NH; ++hh)
+                  mma_16816(acc[hh][mt], a0, a1, a2, a3, pb[hh][0], pb[hh][1]);
+              });
+            });
+          } else {
+            static_for<C::MT>([&](auto MI) {
+              constexpr int mt = decltype(MI)::value;
+              constexpr int p0 = VS::pos(2 * mt), p1 = VS::pos(2 * mt + 1);
+              const uint32_t a0 = lut_pair2<VB, p0>(vw[0], vw[1], lv_off);
+              const uint32_t a1 = lut_pair2<VB, p1>(vw[0], vw[1], lv_off);
+              const uint32_t a2 = lut_pair2<VB, p0>(vw[2], vw[3], lv_off);
+              const uint32_t a3 = lut_pair2<VB, p1>(vw[2], vw[3], lv_off);
+  #pragma unroll
               for (int hh = 0; hh < NH; ++hh)
                 mma_16816(acc[hh][mt], a0, a1, a2, a3, pb[hh][0], pb[hh][1]);
             });
-          });
-        } else {
-          static_for<C::MT>([&](auto MI) {
-            constexpr int mt = decltype(MI)::value;
-            constexpr int p0 = VS::pos(2 * mt), p1 = VS::pos(2 * mt + 1);
-            const uint32_t a0 = lut_pair2<VB, p0>(vw[0], vw[1], lv_off);
-            const uint32_t a1 = lut_pair2<VB, p1>(vw[0], vw[1], lv_off);
-            const uint32_t a2 = lut_pair2<VB, p0>(vw[2], vw[3], lv_off);
-            const uint32_t a3 = lut_pair2<VB, p1>(vw[2], vw[3], lv_off);
-#pragma unroll
-            for (int hh = 0; hh < NH; ++hh)
-              mma_16816(acc[hh][mt], a0, a1, a2, a3, pb[hh][0], pb[hh][1]);
-          });
+          }
         }
       }
-    }
-    // release the stage; the last warp to do so refills it with step s + nst
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) {
-      last = atomicAdd(&released[x], 1) == nwarps - 1;
-      if (last) released[x] = 0;
-    }
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (last && s + nst < s1) refill(s + nst, x);
-    if (++x == nst) {
-      x = 0;
-      phase ^= 1u;
-    }
-    // advance the sequence walk; at a sequence boundary: flush, ticket, maybe merge
-    if (s + 1 < s1) {
-      ++local;
-      if (local >= prefix[cur_b + 1] - prefix[cur_b]) {
-        int nb = cur_b + 1;
-        while (prefix[nb + 1] == prefix[nb]) ++nb;
-        boundary(cur_b, nb);
-        cur_b = nb;
-        local = 0;
-        cur_len = p.seq_lens[cur_b];
+      // release the stage; the last warp to do so refills it with step s + nst
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) {
+        last = atomicAdd(&released[x], 1) == nwarps - 1;
+        if (last) released[x] = 0;
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last && s + nst < s1) refill(s + nst, x);
+      if (++x == nst) {
+        x = 0;
+        phase ^= 1u;
       }
     }
+    flush(cur_b);
+    if (s >= s1) break;
+    do ++cur_b; while (prefix[cur_b + 1] == prefix[cur_b]);   // next sequence with steps
   }
-  // end phase: publish the records of the last sequence, then merge each sequence of
-  // the range together with the other CTAs that cover it
-  flush(cur_b);
+  // end phase: publish the records of every sequence of the range, then merge each
+  // of them together with the other CTAs that cover it
   __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    for (int b = b_first; b <= cur_b; ++b)
+      if (prefix[b + 1] > prefix[b]) atomicAdd(&arrived[b], 1u);
+  }
   if (*timed_out) {
     // copies may still be landing in the stages: give them time (bounded), skip the merge
     if (tid == 0) {
@@ -1004,11 +993,7 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     __syncthreads();
     return;
   }
-  if (tid == 0) {
-    __threadfence();
-    atomicAdd(&arrived[cur_b], 1u);
-  }
-  for (int b = locate(s0); b <= cur_b; ++b)
+  for (int b = b_first; b <= cur_b; ++b)
     if (prefix[b + 1] > prefix[b]) coop_merge(b);
 }
 
