@@ -165,7 +165,8 @@ tq_status plan_decode(int batch, int h_q, int h_kv, int dim, int kb, int vb, int
       const int64_t low = L - base, high = base + budget - (L + lut);
       for (int nst = kMaxStages; nst >= min_st; --nst) {
         const int64_t misc = 16 * nst + 2LL * h_q * dim + 4LL * h_q + 4LL * (batch + 1) +
-                             4LL * ids_cap + 4 * 36 + (int64_t)plan->maxw * (dim + 2) * 4 + 16;
+                             4LL * ids_cap + 4 * 36 + (int64_t)plan->maxw * (dim + 2) * 4 +
+                             4LL * dim + 16;
         for (int at_top = 0; at_top < 2; ++at_top) {
           const int64_t below = at_top ? low : low - misc;   // room for stages below
           if (below < 0) continue;

@@ -361,7 +361,8 @@ __device__ __forceinline__ void store_from_f32(void* base, int64_t i, int32_t dt
 
 // Shared memory: stages below and above the tables (see DecodeParams), and a misc
 // area [full mbarriers | release counters | present masks | q' (H_q x D fp16) | |q'|
-// scales | step prefix sums | block ids | scan scratch | flag | merge partials].
+// scales | step prefix sums | block ids | scan scratch | flag | merge partials |
+// record positions].
 template <int D, int KB, int VB, int NH, int MAXW>
 __global__ void __launch_bounds__(MAXW * 32, 1)
 decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
@@ -395,6 +396,7 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   int* wsum = (int*)(ids + p.ids_cap);                 // [32] per-warp sums of the scan
   int* timed_out = wsum + 32;                          // a stage wait of this CTA gave up
   float* scratch = (float*)(timed_out + 4);            // [warps][D + 2] merge partials
+  int* rpos = (int*)(scratch + blockDim.x / 32 * (D + 2));  // [D] coordinate at a record position
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tig = lane & 3;
@@ -403,9 +405,6 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   const int wph = p.wph;                               // blocks per pipeline step
   const int B = p.batch;
 
-  // tables first: they depend on nothing but the centroids
-  lut_build<KB, 0>(smem + p.lut_off, p.kc, tid, nthreads);
-  lut_build<VB, 1>(smem + p.lut_off, p.vc, tid, nthreads);
 
   // ---- step prefix sums over the sequences (every CTA) ----
   {
@@ -475,6 +474,20 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     return lo;
   };
 
+  // the first segment's query heads (the first KPRE of this warp), loaded now so that
+  // their latency overlaps the block-id loads and the table build
+  const int b_first = locate(s0);
+  constexpr int KPRE = 2;
+  float qpre[KPRE][E];
+#pragma unroll
+  for (int k = 0; k < KPRE; ++k) {
+    const int h = warp + k * nwarps;
+    const int64_t off = (int64_t)b_first * p.q_bstride + (int64_t)(h < p.h_q ? h : 0) * p.q_hstride +
+                        lane * E;
+#pragma unroll
+    for (int i = 0; i < E; ++i) qpre[k][i] = h < p.h_q ? load_as_f32(p.q, off + i, p.q_dtype) : 0.f;
+  }
+
   const int pitch = p.row_pitch;
   const int blk_smem = kBlockSize * pitch;
   const int row_bytes = p.h_kv * p.slot_stride;
@@ -533,6 +546,16 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   if (warp == 0)
     for (int i = 0; i < nst && s0 + i < s1; ++i) refill(s0 + i, i);
 
+  // tables (they depend on nothing but the centroids) while the copies and the query
+  // loads are in flight
+  lut_build<KB, 0>(smem + p.lut_off, p.kc, tid, nthreads);
+  lut_build<VB, 1>(smem + p.lut_off, p.vc, tid, nthreads);
+  // coordinate held at each record position 2 + i (the fragment order; see flush)
+  for (int i = tid; i < D; i += nthreads) {
+    const int g = i & 7, m = i >> 3;
+    rpos[2 * (8 * (m >> 1) + g) + (m & 1)] = VS::coord(g, m);
+  }
+
 
   const int kvh = warp % p.h_kv;
   const int sub = warp / p.h_kv;
@@ -550,17 +573,14 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   // FWHT in registers and shuffles, 1/sqrt(D), then normalised to unit fp16), then
   // every warp reads its B fragments and scales and resets its softmax state and O'.
   // Two CTA barriers; called where all warps are between segments.
-  auto start = [&](int b) {
+  auto start = [&](int b, bool pre) {
     __syncthreads();                    // the previous segment's q' is no longer read
     uint32_t sg[E];
 #pragma unroll
     for (int i = 0; i < E; ++i) sg[i] = sign_mask_at(p.sign_seed, lane * E + i);
-    for (int h = warp; h < p.h_q; h += nwarps) {
-      const int64_t off = (int64_t)b * p.q_bstride + (int64_t)h * p.q_hstride + lane * E;
-      float xq[E];
+    auto rotate_head = [&](int h, float (&xq)[E]) {
 #pragma unroll
-      for (int i = 0; i < E; ++i)
-        xq[i] = __uint_as_float(__float_as_uint(load_as_f32(p.q, off + i, p.q_dtype)) ^ sg[i]);
+      for (int i = 0; i < E; ++i) xq[i] = __uint_as_float(__float_as_uint(xq[i]) ^ sg[i]);
       warp_fwht<E>(xq, lane);
       float ss = 0.f;
 #pragma unroll
@@ -575,6 +595,30 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
 #pragma unroll
       for (int i = 0; i < E; ++i) qh[h * D + lane * E + i] = __float2half_rn(xq[i] * inv);
       if (lane == 0) qsc[h] = nrm * p.scale_log2;
+    };
+    auto load_head = [&](int h, float (&xq)[E]) {
+      const int64_t off = (int64_t)b * p.q_bstride + (int64_t)h * p.q_hstride + lane * E;
+#pragma unroll
+      for (int i = 0; i < E; ++i) xq[i] = load_as_f32(p.q, off + i, p.q_dtype);
+    };
+#pragma unroll
+    for (int k = 0; k < KPRE; ++k) {
+      const int h = warp + k * nwarps;
+      if (h < p.h_q) {
+        float xq[E];
+        if (pre) {
+#pragma unroll
+          for (int i = 0; i < E; ++i) xq[i] = qpre[k][i];
+        } else {
+          load_head(h, xq);
+        }
+        rotate_head(h, xq);
+      }
+    }
+    for (int h = warp + KPRE * nwarps; h < p.h_q; h += nwarps) {
+      float xq[E];
+      load_head(h, xq);
+      rotate_head(h, xq);
     }
     __syncthreads();
 #pragma unroll
@@ -602,7 +646,10 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     }
   };
 
-  // this warp's partial of sequence b -> its record
+  // This warp's partial of sequence b -> its record.  Record of query head h:
+  // [M, l, O'] with O' in fragment order: coordinate VS::coord(g, 2 mt + c) at
+  // 2 + 2 (8 mt + g) + c, so that each store (one mt, one head column per thread) writes
+  // eight contiguous pairs per head.
   auto flush = [&](int b) {
     float* base = p.part + ((int64_t)(blockIdx.x + b) * wph + sub) * (int64_t)p.h_q * (D + 2);
 #pragma unroll
@@ -614,22 +661,15 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
         l += __shfl_xor_sync(0xffffffffu, l, 8);
         l += __shfl_xor_sync(0xffffffffu, l, 16);
         const int g = 8 * hh + 2 * tig + e;
-        if (gid == 0 && g < G) {
+        if (g < G) {
           float* rec = base + (int64_t)(kvh * G + g) * (D + 2);
-          rec[0] = Mrun[hh][e];
-          rec[1] = l;
+          if (gid == 0) *(float2*)rec = make_float2(Mrun[hh][e], l);
+#pragma unroll
+          for (int mt = 0; mt < C::MT; ++mt)
+            *(float2*)(rec + 2 + 2 * (8 * mt + gid)) =
+                make_float2(acc[hh][mt][e], acc[hh][mt][e + 2]);
         }
       }
-      static_for<C::MT>([&](auto MI) {
-        constexpr int mt = decltype(MI)::value;
-        const int c0 = VS::coord(gid, 2 * mt), c1 = VS::coord(gid, 2 * mt + 1);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int g2 = 8 * hh + 2 * tig + (k & 1);
-          const int c = (k >> 1) ? c1 : c0;
-          if (g2 < G) base[(int64_t)(kvh * G + g2) * (D + 2) + 2 + c] = acc[hh][mt][k];
-        }
-      });
     }
   };
 
@@ -641,70 +681,57 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
 
   // Merge of query head h of sequence b over records i = i_first, i_first + i_step, ...
   // (record i: CTA c_lo + i / wph, sub-stream i % wph) into this warp's partial
-  // (M, l, O'[lane E .. lane E + E - 1]).
+  // (M, l, and o[k] = O' at record position 2 + lane E + k).  One pass: records are read
+  // in batches (contiguous loads) and folded in with an online rescale.
   auto merge_part = [&](int b, int h, int64_t c_lo, int R, int i_first, int i_step, float& M,
                         float& l, float (&o)[E]) {
+    constexpr int NB = 4;                             // records per batch
     const int64_t rstride = (int64_t)p.h_q * (D + 2);
     const float* hb = p.part + (int64_t)h * (D + 2);
-    auto rec_of = [&](int i) -> int64_t {
-      const int64_t c = c_lo + i / wph;
-      return nonempty(c) ? ((c + b) * wph + i % wph) * rstride : -1;
-    };
     M = -INFINITY;
-    for (int i = i_first + lane * i_step; i < R; i += 32 * i_step) {
-      const int64_t r = rec_of(i);
-      if (r >= 0) M = fmaxf(M, __ldcg(hb + r));
-    }
-#pragma unroll
-    for (int of = 16; of > 0; of >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, of));
     l = 0.f;
 #pragma unroll
-    for (int i = 0; i < E; ++i) o[i] = 0.f;
-    if (M == -INFINITY) return;
-    for (int i0 = i_first; i0 < R; i0 += 32 * i_step) {
-      // lane j of this pass: weight and offset of record i0 + j i_step
-      const int i = i0 + lane * i_step;
-      const int64_t r = i < R ? rec_of(i) : -1;
-      float wt = 0.f;
-      if (r >= 0) {
-        const float mi = __ldcg(hb + r);
-        wt = mi == -INFINITY ? 0.f : exp2f(mi - M);
-        l += wt * __ldcg(hb + r + 1);
-      }
-      const int nr = min(32, (R - i0 + i_step - 1) / i_step);
-      for (int j = 0; j < nr; j += 4) {
-        float wv[4], v[4][E];
-        int64_t rr[4];
+    for (int k = 0; k < E; ++k) o[k] = 0.f;
+    for (int i0 = i_first; i0 < R; i0 += NB * i_step) {
+      float mj[NB], lj[NB], vj[NB][E];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int src = min(j + u, 31);
-          wv[u] = __shfl_sync(0xffffffffu, wt, src);
-          rr[u] = __shfl_sync(0xffffffffu, r, src);
-          if (j + u >= nr) wv[u] = 0.f;
-        }
+      for (int j = 0; j < NB; ++j) {
+        const int i = i0 + j * i_step;
+        const int64_t c = c_lo + i / wph;
+        mj[j] = -INFINITY;
+        lj[j] = 0.f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (wv[u] != 0.f) {
-            const float2* src = (const float2*)(hb + rr[u] + 2 + lane * E);
+        for (int k = 0; k < E; ++k) vj[j][k] = 0.f;
+        if (i < R && nonempty(c)) {
+          const float* rec = hb + ((c + b) * wph + i % wph) * rstride;
+          const float2 ml = __ldcg((const float2*)rec);
+          mj[j] = ml.x;
+          lj[j] = ml.y;
 #pragma unroll
-            for (int k = 0; k < E / 2; ++k) {
-              const float2 t = __ldcg(src + k);
-              v[u][2 * k] = t.x;
-              v[u][2 * k + 1] = t.y;
-            }
-          } else {
-#pragma unroll
-            for (int k = 0; k < E; ++k) v[u][k] = 0.f;
+          for (int k = 0; k < E / 2; ++k) {
+            const float2 t = __ldcg((const float2*)(rec + 2 + lane * E) + k);
+            vj[j][2 * k] = t.x;
+            vj[j][2 * k + 1] = t.y;
           }
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-          for (int k = 0; k < E; ++k) o[k] = fmaf(wv[u], v[u][k], o[k]);
       }
-    }
+      float mx = M;
 #pragma unroll
-    for (int of = 16; of > 0; of >>= 1) l += __shfl_xor_sync(0xffffffffu, l, of);
+      for (int j = 0; j < NB; ++j) mx = fmaxf(mx, mj[j]);
+      if (mx == -INFINITY) continue;
+      const float f = M == -INFINITY ? 0.f : exp2f(M - mx);
+      l *= f;
+#pragma unroll
+      for (int k = 0; k < E; ++k) o[k] *= f;
+#pragma unroll
+      for (int j = 0; j < NB; ++j) {
+        const float w = mj[j] == -INFINITY ? 0.f : exp2f(mj[j] - mx);
+        l = fmaf(w, lj[j], l);
+#pragma unroll
+        for (int k = 0; k < E; ++k) o[k] = fmaf(w, vj[j][k], o[k]);
+      }
+      M = mx;
+    }
   };
 
   // End phase for sequence b: once every CTA covering b has written its records, this
@@ -737,6 +764,9 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     int g = 1;
     while (nh > 0 && 2 * g * min(nh, nwarps) <= nwarps) g *= 2;
     const int groups = nwarps / g, gi = warp / g, mi = warp % g;
+    int nat[E];                          // coordinate at record position 2 + lane E + k
+#pragma unroll
+    for (int k = 0; k < E; ++k) nat[k] = rpos[lane * E + k];
     uint32_t sg[E];
 #pragma unroll
     for (int i = 0; i < E; ++i) sg[i] = sign_mask_at(p.sign_seed, lane * E + i);
@@ -746,10 +776,10 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
       float M, l, o[E];
       if (j < nh) {
         merge_part(b, h, c_lo, R, mi, g, M, l, o);
-        float* sc = scratch + warp * (D + 2);
+        float* sc = scratch + warp * (D + 2);    // natural coordinate order
         if (lane == 0) { sc[0] = M; sc[1] = l; }
 #pragma unroll
-        for (int i = 0; i < E; ++i) sc[2 + lane * E + i] = o[i];
+        for (int i = 0; i < E; ++i) sc[2 + nat[i]] = o[i];
       }
       __syncthreads();
       if (j < nh && mi == 0) {
@@ -789,7 +819,6 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
 
   // Outer loop: the segments (one per sequence) of this CTA's step range; inner loop:
   // the steps of a segment.  Segment set-up and write-out stay out of the step loop.
-  const int b_first = locate(s0);
   int cur_b = b_first;
   int x = 0;
   uint32_t phase = 0;
@@ -798,7 +827,7 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     const int64_t seg_end = imin64(s1, prefix[cur_b + 1]);
     const int cur_len = p.seq_lens[cur_b];
     int bi = (int)(s - prefix[cur_b]) * wph + sub;    // this warp's block in the sequence
-    start(cur_b);
+    start(cur_b, cur_b == b_first);
     for (; s < seg_end; ++s, bi += wph) {
       if (!dead && !mbar_wait(&full[x], phase, kWaitMs)) {
         if (lane == 0) {
