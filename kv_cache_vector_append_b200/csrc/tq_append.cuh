@@ -308,20 +308,23 @@ __device__ __forceinline__ void encode_pack(const uint64_t (&xp)[32], float r,
     for (int hf = 0; hf < 2; ++hf) {
       const float u = hf ? f2hi(u2) : f2lo(u2);
       const int j = 2 * i + hf;
-      uint32_t code;
+      const int bit = j * BITS;
+      const int w0 = bit >> 5, o0 = bit & 31;
+      // the fields of a word do not overlap, so a shifted add packs the code
       if constexpr (FAST) {
         const uint32_t k4 = t->k4[__float_as_uint(u) >> kBucketShift];
-        code = (k4 + (u > lds_f32(bnd_win | k4) ? 4u : 0u)) >> 2;
+        const uint32_t c4 = k4 + (u > lds_f32(bnd_win | k4) ? 4u : 0u);   // 4 * code
+        if (o0 >= 2) acc[w0] += c4 << (o0 - 2);
+        else acc[w0] += c4 >> (2 - o0);
+        if (o0 + BITS > 32) acc[w0 + 1] += c4 >> (32 - o0 + 2);
       } else {
         int e = 1;
 #pragma unroll
         for (int st = 0; st < BITS; ++st) e = 2 * e + (u > t->eytz[e - 1] ? 1 : 0);
-        code = (uint32_t)(e - (1 << BITS));
+        const uint32_t code = (uint32_t)(e - (1 << BITS));
+        acc[w0] += code << o0;
+        if (o0 + BITS > 32) acc[w0 + 1] += code >> (32 - o0);
       }
-      const int bit = j * BITS;
-      const int w0 = bit >> 5, o0 = bit & 31;
-      acc[w0] |= code << o0;
-      if (o0 + BITS > 32) acc[w0 + 1] |= code >> (32 - o0);
     }
   }
 #pragma unroll

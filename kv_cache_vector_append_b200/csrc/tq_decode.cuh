@@ -823,12 +823,16 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   int x = 0;
   uint32_t phase = 0;
   bool dead = false;                    // a stage wait of this warp gave up
-  for (int64_t s = s0;;) {
-    const int64_t seg_end = imin64(s1, prefix[cur_b + 1]);
-    const int cur_len = p.seq_lens[cur_b];
-    int bi = (int)(s - prefix[cur_b]) * wph + sub;    // this warp's block in the sequence
+  // step counters relative to s0 (a range is < 2^31 steps); soff = offset of stage x
+  const int nsteps = (int)(s1 - s0);
+  const int warp_off = sub * blk_smem + kvh * p.slot_stride;
+  int soff = p.n_low > 0 ? p.stage_lo_off : p.stage_hi_off;
+  for (int r = 0;;) {
+    const int seg_end = (int)(imin64(s1, prefix[cur_b + 1]) - s0);
+    // tokens of this warp's block still to come in the sequence
+    int rem = p.seq_lens[cur_b] - ((int)(s0 + r - prefix[cur_b]) * wph + sub) * kBlockSize;
     start(cur_b, cur_b == b_first);
-    for (; s < seg_end; ++s, bi += wph) {
+    for (; r < seg_end; ++r, rem -= wph * kBlockSize) {
       if (!dead && !mbar_wait(&full[x], phase, kWaitMs)) {
         if (lane == 0) {
           report_error(p.err, TQ_DEVERR_TIMEOUT);
@@ -836,10 +840,9 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
         }
         dead = true;
       }
-      const int valid =
-          (!dead && ((present[x] >> sub) & 1u)) ? min(kBlockSize, cur_len - bi * kBlockSize) : 0;
+      const int valid = (!dead && ((present[x] >> sub) & 1u)) ? min(kBlockSize, rem) : 0;
       if (valid > 0) {
-        const uint8_t* base = stage_ptr(x) + sub * blk_smem + kvh * p.slot_stride;
+        const uint8_t* base = smem + soff + warp_off;
         // token t (0..15) of this block lives at base + t * pitch
 
         // ---- S^T = K~ . Qhat^T: one m-tile of 16 tokens ----
@@ -995,14 +998,17 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
         if (last) released[x] = 0;
       }
       last = __shfl_sync(0xffffffffu, last, 0);
-      if (last && s + nst < s1) refill(s + nst, x);
-      if (++x == nst) {
+      if (last && r + nst < nsteps) refill(s0 + r + nst, x);
+      ++x;
+      soff = x == p.n_low ? p.stage_hi_off : soff + p.stage_bytes;
+      if (x == nst) {
         x = 0;
         phase ^= 1u;
+        soff = p.n_low > 0 ? p.stage_lo_off : p.stage_hi_off;
       }
     }
     flush(cur_b);
-    if (s >= s1) break;
+    if (r >= nsteps) break;
     do ++cur_b; while (prefix[cur_b + 1] == prefix[cur_b]);   // next sequence with steps
   }
   // end phase: publish the records of every sequence of the range, then merge each
