@@ -192,32 +192,51 @@ class ClockSampler:
 # CPU oracle (baseline and reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample_step(wl, tables, n_append=1024, n_decode_tokens=2048):
+def oracle_sample_step(wl, tables, n_append=1024, n_decode_tokens=2048, seq=0):
     """One bounded oracle step on the workload: quantize-append of n_append tokens
-    of sequence 0 into a page pool, then a decode step of sequence 0 over its
-    first n_decode_tokens tokens.  Returns (seconds, algorithmic bytes)."""
+    of sequence `seq` into a page pool, then a decode step of that sequence over
+    its first n_decode_tokens tokens.  Returns (seconds, algorithmic bytes, text)."""
     from oracle import tq_oracle as O
     spec = wl.spec
     kt, vt = tables
-    n_dec = int(min(n_decode_tokens, wl.seq_lens[0]))
+    seq = int(seq) % max(1, spec.batch)
+    start = int(wl.seq_lens[:seq].astype(np.int64).sum())
+    n_dec = int(min(n_decode_tokens, wl.seq_lens[seq]))
     n_app = int(min(n_append, n_dec))
     pages = np.zeros((wl.num_blocks, 16, spec.num_kv_heads, wl.slot_bytes), dtype=np.uint8)
-    idx = np.arange(n_dec)
-    k = wl.k[:n_dec].float().numpy()
-    v = wl.v[:n_dec].float().numpy()
+    slots = wl.slot_mapping[start:start + n_dec]
+    k = wl.k[start:start + n_dec].float().numpy()
+    v = wl.v[start:start + n_dec].float().numpy()
     # the untimed part fills the decode range; the timed part re-appends n_app tokens
-    pages = O.quantize_append(pages, wl.slot_mapping[idx], k, v, kt, vt, spec.sign_seed)
+    pages = O.quantize_append(pages, slots, k, v, kt, vt, spec.sign_seed)
     t0 = time.perf_counter()
-    pages = O.quantize_append(pages, wl.slot_mapping[:n_app], k[:n_app], v[:n_app], kt, vt,
+    pages = O.quantize_append(pages, slots[:n_app], k[:n_app], v[:n_app], kt, vt,
                               spec.sign_seed)
-    q = wl.q[:1].float().numpy().astype(np.float64)
-    O.paged_decode(q, pages, wl.block_table[:1], np.array([n_dec], dtype=np.int32), kt, vt,
-                   spec.sign_seed, spec.scale)
+    q = wl.q[seq:seq + 1].float().numpy().astype(np.float64)
+    O.paged_decode(q, pages, wl.block_table[seq:seq + 1], np.array([n_dec], dtype=np.int32),
+                   kt, vt, spec.sign_seed, spec.scale)
     dt = time.perf_counter() - t0
     nbytes = append_bytes(spec, n_app) + decode_bytes(spec, [n_dec])[0]
     desc = (f"{n_app} tokens x {spec.num_kv_heads} KV heads appended + 1 sequence x {n_dec} "
             f"tokens x {spec.num_q_heads} q heads decoded")
     return dt, nbytes, desc
+
+
+def cpu_baseline(wl, tables, min_seconds=10.0, max_samples=64):
+    """The oracle timed on host cores over repeated bounded samples (one per
+    sequence, cycling) until at least min_seconds of oracle work has run."""
+    oracle_sample_step(wl, tables, 256, 512)   # warm caches
+    total_t = total_b = 0.0
+    n = 0
+    desc = ""
+    while n < max_samples and (total_t < min_seconds or n == 0):
+        dt, nb, desc = oracle_sample_step(wl, tables, seq=n)
+        total_t += dt
+        total_b += nb
+        n += 1
+    return {"value": total_b / total_t / 1e9, "unit": "GB/s", "cores": blas_threads(),
+            "kind": "oracle", "sample": f"{n} samples (sequences 0..{n - 1}, cycling) of: {desc}",
+            "seconds": total_t}
 
 
 def oracle_tables(spec):
@@ -244,12 +263,12 @@ def run_reference(args):
     spec = W.CONFIGS[args.config]
     wl = W.generate(spec)
     tables = oracle_tables(spec)
-    for _ in range(args.warmup):
-        oracle_sample_step(wl, tables)
+    for i in range(args.warmup):
+        oracle_sample_step(wl, tables, seq=i)
     total_t = total_b = 0.0
     desc = ""
-    for _ in range(args.steps):
-        dt, nb, desc = oracle_sample_step(wl, tables)
+    for i in range(args.steps):
+        dt, nb, desc = oracle_sample_step(wl, tables, seq=args.warmup + i)
         total_t += dt
         total_b += nb
     value = total_b / total_t / 1e9
@@ -451,11 +470,7 @@ def run_gpu(args):
     if e2e is not None:
         line["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:
-        tables = oracle_tables(spec)
-        oracle_sample_step(wl, tables, 256, 512)   # warm caches
-        dt, nb, desc = oracle_sample_step(wl, tables)
-        line["cpu_baseline"] = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": blas_threads(),
-                                "kind": "oracle", "sample": desc, "seconds": dt}
+        line["cpu_baseline"] = cpu_baseline(wl, oracle_tables(spec))
     print(json.dumps(line), flush=True)
     if world > 1:
         tq.set_workspace(None)
