@@ -249,6 +249,22 @@ bool encode_page_map(CUtensorMap* map, const void* pages, int64_t num_blocks, in
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor map of a (tokens, h_kv, D) 16-bit K or V input seen as (D, h_kv, tokens)
+// elements, read in boxes of 64 elements x `box_h` heads x `box_t` tokens with the
+// 128-byte swizzle.  Returns false when the driver rejects the map.
+bool encode_input_map(CUtensorMap* map, const void* data, int64_t T, int h_kv, int D,
+                      int64_t tok_stride, int64_t head_stride, int box_h, int box_t) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (fn == nullptr || T > 0x7fffffffll) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)h_kv, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {(cuuint64_t)(head_stride * 2), (cuuint64_t)(tok_stride * 2)};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_h, (cuuint32_t)box_t};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(data), dims, strides, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct DecodeCall {
   int B = 0, h_q = 0, h_kv = 0, D = 0, kbits = 0, vbits = 0, kb = 0, max_blocks = 0;
   int64_t stride = 0;
@@ -486,7 +502,27 @@ tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_tensor 
        align_mode_of(v.data, es, {v.stride[0], v.stride[1]}) != 16))
     p.align_mode = 4;
   if (k.dtype == TQ_F32 && p.align_mode == 0) return TQ_ERR_INVALID_ARG;
-  return launch_append_any(D, k.dtype, p, ds->info, as_stream(stream));
+
+  // Tiles of `rows` consecutive (token, head) pairs are whole runs of one token's heads
+  // when h_kv divides rows or rows divides h_kv.
+  const int rows = 2048 / D;
+  p.run_heads = (h_kv <= rows && rows % h_kv == 0) ? h_kv : (h_kv % rows == 0 ? rows : 0);
+  const int slot = kb + vb;
+  p.bulk_out = p.run_heads > 0 && pages.shape[3] == slot && pages.stride[2] == slot &&
+               (uintptr_t)pages.data % 16 == 0 && pages.stride[0] % 16 == 0 &&
+               pages.stride[1] % 16 == 0 && ((int64_t)p.run_heads * slot) % 16 == 0;
+  AppendMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  p.tma_in = 0;
+  if (p.run_heads > 0 && es == 2 && (uintptr_t)k.data % 16 == 0 && (uintptr_t)v.data % 16 == 0 &&
+      k.stride[0] % 8 == 0 && k.stride[1] % 8 == 0 && v.stride[0] % 8 == 0 &&
+      v.stride[1] % 8 == 0 &&
+      encode_input_map(&maps.k, k.data, T, h_kv, D, k.stride[0], k.stride[1], p.run_heads,
+                       rows / p.run_heads) &&
+      encode_input_map(&maps.v, v.data, T, h_kv, D, v.stride[0], v.stride[1], p.run_heads,
+                       rows / p.run_heads))
+    p.tma_in = 1;
+  return launch_append_any(D, k.dtype, p, maps, ds->info, as_stream(stream));
 }
 
 tq_status tq_rotate_unit(tq_tensor u, tq_tensor norm, tq_tensor x, uint64_t sign_seed,

@@ -11,11 +11,15 @@
 // row), so the FWHT is six register stages (f32x2 add / sub: two fp32 operations per
 // instruction) plus log2(D/64) shuffle stages.  A warp owns a tile of 32*64/D
 // consecutive (token, KV head) pairs and does its K rows, then its V rows; lane l
-// serves row l % ROWS, part l / ROWS, so that each 8-lane phase of a 16-byte shared
-// load touches 8 different rows (padded pitch, no bank conflicts).  Input rows are
-// staged in shared memory by cp.async one half-tile ahead; the tile's full slots are
-// staged in shared memory and written back with lanes running over (slot, word), so
-// each slot's bytes go out together.
+// serves row l % ROWS, part l / ROWS.  A kind's rows of a tile sit in shared memory as
+// [part][row][64 elements], the 16-byte chunk c of a part row stored at chunk
+// c ^ (row & 7) (the 128-byte swizzle of the tensor-copy unit), so that each 8-lane
+// phase of a 16-byte shared load touches 8 different bank groups.  Input rows are
+// staged one half-tile ahead: by tensor copies (one box per part: 64 elements x the
+// tile's heads x its tokens) when the tile is a box of the input, else by cp.async
+// into the same layout.  The tile's full slots are staged in shared memory and stored
+// with one bulk copy per token when the page pool holds each token's slots
+// back to back with 16-byte alignment, else with lanes running over (slot, word).
 //
 // Encode.  idx = #{i : b_i < u} over the fp32 boundaries.  For bits <= 4 (and when no
 // two boundaries share a bucket) the top 12 bits of u's float encoding (sign,
@@ -49,6 +53,15 @@ struct AppendParams {
   unsigned int* err;
   int32_t align_mode;       // 16: rows 16-byte aligned; 4: 4-byte aligned; 0: any
   int32_t bs_shift;         // log2(block_size) when it is a power of two, else -1
+  int32_t run_heads;        // heads of one token in a tile (tiles token-aligned), else 0
+  int32_t tma_in;           // 1: input rows staged by tensor copies (maps K, V)
+  int32_t bulk_out;         // 1: slots stored by one bulk copy per token run
+};
+
+// Tensor maps of K and V as (D, h_kv, tokens) 16-bit elements, boxes of
+// (64, run_heads, ROWS / run_heads) with the 128-byte swizzle; unused unless tma_in.
+struct AppendMaps {
+  CUtensorMap k, v;
 };
 
 struct RotateParams {      // test export of the rotation (tq_rotate_unit)
@@ -133,28 +146,33 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
   return v;
 }
 
-// Stage `nrows` rows of RB bytes into shared memory (pitch `pitch`); row r starts at
-// row_ptr(r).  Issued by one warp.
-template <int RB, typename RowPtr>
-__device__ __forceinline__ void stage_rows(uint8_t* dst, int pitch, int nrows, RowPtr row_ptr,
+// Stage `nrows` rows of RB bytes into the tile layout [part][row][PB] (16-byte chunk c of
+// a part row stored at chunk c ^ (row & 7)); row r starts at row_ptr(r).  Issued by one
+// warp.
+template <int RB, int PB, int ROWS>
+__device__ __forceinline__ uint8_t* tile_at(uint8_t* dst, int r, int b) {
+  return dst + (b / PB) * (ROWS * PB) + r * PB + ((((b % PB) >> 4) ^ (r & 7)) << 4) + (b & 15);
+}
+template <int RB, int PB, int ROWS, typename RowPtr>
+__device__ __forceinline__ void stage_rows(uint8_t* dst, int nrows, RowPtr row_ptr,
                                            int align_mode, int lane) {
   if (align_mode == 16) {
     constexpr int NC = RB / 16;
     for (int f = lane; f < nrows * NC; f += 32) {
-      const int r = f / NC, c = f % NC;
-      cp_async16(dst + r * pitch + c * 16, (const uint8_t*)row_ptr(r) + c * 16);
+      const int r = f / NC, b = (f % NC) * 16;
+      cp_async16(tile_at<RB, PB, ROWS>(dst, r, b), (const uint8_t*)row_ptr(r) + b);
     }
   } else if (align_mode == 4) {
     constexpr int NC = RB / 4;
     for (int f = lane; f < nrows * NC; f += 32) {
-      const int r = f / NC, c = f % NC;
-      cp_async4(dst + r * pitch + c * 4, (const uint8_t*)row_ptr(r) + c * 4);
+      const int r = f / NC, b = (f % NC) * 4;
+      cp_async4(tile_at<RB, PB, ROWS>(dst, r, b), (const uint8_t*)row_ptr(r) + b);
     }
   } else {
     constexpr int NC = RB / 2;
     for (int f = lane; f < nrows * NC; f += 32) {
-      const int r = f / NC, c = f % NC;
-      *(uint16_t*)(dst + r * pitch + c * 2) = *((const uint16_t*)row_ptr(r) + c);
+      const int r = f / NC, b = (f % NC) * 2;
+      *(uint16_t*)tile_at<RB, PB, ROWS>(dst, r, b) = *(const uint16_t*)((const uint8_t*)row_ptr(r) + b);
     }
   }
 }
@@ -202,8 +220,10 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
 // rotation signs applied (the sign flip is an xor of the sign bit; for bf16 it rides
 // along with the widening), and do the first FWHT stage (h = 1, the two halves of a
 // register): (a, b) -> (a + b, a - b).
+// `row` is the shared-window address of this lane's part row (aligned to its size) with
+// the row's swizzle (row & 7) in bits 4-6, so chunk c sits at row ^ (c << 4).
 template <typename Tin>
-__device__ __forceinline__ void load_signed(uint64_t (&xp)[32], const uint8_t* p,
+__device__ __forceinline__ void load_signed(uint64_t (&xp)[32], uint32_t row,
                                             const uint32_t* m) {
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
@@ -212,13 +232,13 @@ __device__ __forceinline__ void load_signed(uint64_t (&xp)[32], const uint8_t* p
     const uint4 s1 = *(const uint4*)(m + 8 * c + 4);
     const uint32_t s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
     if constexpr (sizeof(Tin) == 4) {
-      const uint4 q0 = *(const uint4*)(p + 32 * c);
-      const uint4 q1 = *(const uint4*)(p + 32 * c + 16);
+      const uint4 q0 = lds128(row ^ (uint32_t)(32 * c));
+      const uint4 q1 = lds128(row ^ (uint32_t)(32 * c + 16));
       const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
       for (int k = 0; k < 8; ++k) a[k] = __uint_as_float(w[k] ^ s[k]);
     } else {
-      const uint4 q = *(const uint4*)(p + 16 * c);
+      const uint4 q = lds128(row ^ (uint32_t)(16 * c));
       const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -344,36 +364,36 @@ __device__ __forceinline__ void encode_pack_any(const uint64_t (&xp)[32], float 
   encode_pack<BITS, false>(xp, r, t, words);
 }
 
-// Per-warp shared memory: K rows, V rows (one tile of ROWS (token, head) pairs each),
-// the tile's full slots (K region then V region; `out_pitch` words a slot, odd, sized
-// for the launch's bit widths), and the per-tile slot offsets and row addresses (two
-// tiles in flight).
+// Shared memory: the K and V tables and sign masks; then (1024-byte aligned, as the
+// swizzled tensor copies need) each warp's two input buffers (K rows, V rows of one
+// tile, KIND bytes each); then each warp's small arrays: two mbarriers, the slot
+// offsets and row addresses of two tiles, and the tile's slots ([ROWS][slot words]).
 template <int D, typename Tin>
 struct AppendSmem {
   using G = AppendGeom<D>;
-  static constexpr int RB = D * InType<Tin>::kBytes;
-  static constexpr int INPITCH = RB + 16;
+  static constexpr int RB = D * InType<Tin>::kBytes;    // bytes of one input row
+  static constexpr int PB = 64 * InType<Tin>::kBytes;   // bytes of one lane's part of a row
+  static constexpr int KIND = G::TPR * G::ROWS * PB;    // one kind's rows of a tile
   static constexpr int TABLES = ((2 * (int)sizeof(EncodeTables) + 4 * D + 8) + 127) / 128 * 128;
-  static __host__ __device__ constexpr int out_pitch(int kbits, int vbits) {
-    return ((D * kbits / 8 + 4 + D * vbits / 8 + 4) / 4) | 1;
+  static __host__ __device__ constexpr int slot_words(int kbits, int vbits) {
+    return (D * kbits / 8 + 4 + D * vbits / 8 + 4) / 4;
   }
-  static __host__ __device__ constexpr int per_warp(int out_pitch) {
-    return 2 * G::ROWS * INPITCH + 2 * G::ROWS * 8 + 2 * 2 * G::ROWS * 8 +
-           (G::ROWS * out_pitch * 4 + 15) / 16 * 16;
+  static __host__ __device__ constexpr int misc_per_warp(int swords) {
+    return 16 + 2 * G::ROWS * 8 + 2 * 2 * G::ROWS * 8 + (G::ROWS * swords * 4 + 15) / 16 * 16;
   }
   static __host__ __device__ constexpr int bytes(int kbits, int vbits) {
-    return TABLES + kAppendWarps * per_warp(out_pitch(kbits, vbits));
+    return TABLES + 1024 + kAppendWarps * (2 * KIND + misc_per_warp(slot_words(kbits, vbits)));
   }
 };
 
 // Quantize-append.  A warp owns tiles of ROWS consecutive (token, KV head) pairs and
 // does both halves of each: the K rows, then the V rows (each row: D/64 lanes, 64
-// coordinates a lane), into the tile's slots staged in shared memory; then it writes
-// the full slots out (contiguous whole-slot stores, so every DRAM sector of a slot is
-// written by one store pass).  Input rows are staged by cp.async one half-tile ahead.
+// coordinates a lane), into the tile's slots staged in shared memory; then it stores
+// the full slots (whole-slot stores, so every DRAM sector of a slot is written by one
+// store pass).  Input rows are staged one half-tile ahead.
 template <int D, typename Tin>
 __global__ void __launch_bounds__(kAppendWarps * 32, 2)
-append_kernel(AppendParams p) {
+append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
   using G = AppendGeom<D>;
   using SM = AppendSmem<D, Tin>;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -381,22 +401,32 @@ append_kernel(AppendParams p) {
   uint32_t* smask = (uint32_t*)(smem + 2 * sizeof(EncodeTables));  // D sign masks
   int* fast = (int*)(smask + D);                                    // [2] bucket encode valid
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int out_pitch = SM::out_pitch(p.bits[0], p.bits[1]);
-  uint8_t* in_s = smem + SM::TABLES + warp * SM::per_warp(out_pitch);   // [2 kinds][ROWS]
-  int64_t* dst_s = (int64_t*)(in_s + 2 * G::ROWS * SM::INPITCH);   // [2 tiles][ROWS] slots
+  const int kwords = (D * p.bits[0] + 7) / 8 / 4 + 1;             // K region words
+  const int vwords = (D * p.bits[1] + 7) / 8 / 4 + 1;
+  const int swords = kwords + vwords;                              // slot words written
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t in_off = ((sbase + SM::TABLES + 1023u) & ~1023u) - sbase;
+  uint8_t* in_s = smem + in_off + warp * 2 * SM::KIND;             // [2 kinds][KIND]
+  uint8_t* misc = smem + in_off + kAppendWarps * 2 * SM::KIND + warp * SM::misc_per_warp(swords);
+  uint64_t* bars = (uint64_t*)misc;                                // [2 kinds]
+  int64_t* dst_s = (int64_t*)(misc + 16);                          // [2 tiles][ROWS] slots
   const uint8_t** src_s = (const uint8_t**)(dst_s + 2 * G::ROWS);  // [2 tiles][2 kinds][ROWS]
-  uint32_t* out_s = (uint32_t*)(src_s + 2 * 2 * G::ROWS);          // [ROWS][out_pitch]
+  uint32_t* out_s = (uint32_t*)(src_s + 2 * 2 * G::ROWS);          // [ROWS][swords]
 
   const int64_t npairs = p.num_tokens * p.h_kv;                    // < 2^31 (host check)
   const int64_t ntiles = (npairs + G::ROWS - 1) / G::ROWS;
   const int64_t gwarp = (int64_t)blockIdx.x * kAppendWarps + warp;
   const int64_t nwarps = (int64_t)gridDim.x * kAppendWarps;
-  const int kwords = (D * p.bits[0] + 7) / 8 / 4 + 1;             // K region words
-  const int vwords = (D * p.bits[1] + 7) / 8 / 4 + 1;
-  const int swords = kwords + vwords;                              // slot words written
 
-  // Resolve tile `tile` (slot offsets, K and V row addresses; lane r < ROWS handles
-  // pair r0 + r) into slot `tb`.
+  if (lane == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  // Resolve tile `tile` (slot offsets; for cp.async staging also the K and V row
+  // addresses; lane r < ROWS handles pair r0 + r) into slot `tb`.
   auto resolve = [&](int64_t tile, int tb) {
     const int r0 = (int)(tile * G::ROWS);
     const int nr = (int)imin64((int64_t)G::ROWS, npairs - r0);
@@ -404,11 +434,13 @@ append_kernel(AppendParams p) {
       const uint32_t row = (uint32_t)(r0 + lane);
       const uint32_t t = row / (uint32_t)p.h_kv;
       const uint32_t h = row - t * (uint32_t)p.h_kv;
+      if (!p.tma_in) {
 #pragma unroll
-      for (int kind = 0; kind < 2; ++kind)
-        src_s[(tb * 2 + kind) * G::ROWS + lane] =
-            (const uint8_t*)p.src[kind] +
-            ((int64_t)t * p.tok_stride[kind] + (int64_t)h * p.head_stride_in[kind]) * SM::RB / D;
+        for (int kind = 0; kind < 2; ++kind)
+          src_s[(tb * 2 + kind) * G::ROWS + lane] =
+              (const uint8_t*)p.src[kind] +
+              ((int64_t)t * p.tok_stride[kind] + (int64_t)h * p.head_stride_in[kind]) * SM::RB / D;
+      }
       const int64_t slot = p.slot_mapping[(int64_t)t * p.slot_map_stride];
       int64_t off = -1;
       if (slot >= 0) {
@@ -430,12 +462,26 @@ append_kernel(AppendParams p) {
     }
     __syncwarp();
   };
-  // Stage the `kind` rows of the tile resolved in slot tb into buffer `kind`.
+  // Start staging the `kind` rows of the tile resolved in slot tb into buffer `kind`.
   auto stage = [&](int64_t tile, int tb, int kind) {
-    const int nr = (int)imin64((int64_t)G::ROWS, npairs - tile * G::ROWS);
-    stage_rows<SM::RB>(in_s + kind * G::ROWS * SM::INPITCH, SM::INPITCH, nr,
-                       [&](int r) { return (const void*)src_s[(tb * 2 + kind) * G::ROWS + r]; },
-                       p.align_mode, lane);
+    uint8_t* buf = in_s + kind * SM::KIND;
+    if (p.tma_in) {
+      if (lane == 0) {
+        const int r0 = (int)(tile * G::ROWS);
+        const int t0 = r0 / p.h_kv;
+        const int h0 = r0 - t0 * p.h_kv;
+        const CUtensorMap* map = kind ? &maps.v : &maps.k;
+        mbar_arrive_expect_tx(&bars[kind], SM::KIND);
+#pragma unroll
+        for (int part = 0; part < G::TPR; ++part)
+          tensor_g2s_3d(buf + part * G::ROWS * SM::PB, map, 64 * part, h0, t0, &bars[kind]);
+      }
+    } else {
+      const int nr = (int)imin64((int64_t)G::ROWS, npairs - tile * G::ROWS);
+      stage_rows<SM::RB, SM::PB, G::ROWS>(
+          buf, nr, [&](int r) { return (const void*)src_s[(tb * 2 + kind) * G::ROWS + r]; },
+          p.align_mode, lane);
+    }
   };
   // the first tile's K rows are in flight while the tables are built
   if (gwarp < ntiles) {
@@ -453,8 +499,14 @@ append_kernel(AppendParams p) {
 
   const int rl = lane % G::ROWS;           // row within the tile
   const int part = lane / G::ROWS;         // which 64 coordinates of the row
+  // this lane's part row in buffer 0, with its swizzle in bits 4-6
+  const uint32_t row0 = smem_u32(in_s) + (uint32_t)((part * G::ROWS + rl) * SM::PB) +
+                        (uint32_t)((rl & 7) << 4);
   int tb = 0;
-  for (int64_t tile = gwarp; tile < ntiles; tile += nwarps) {
+  uint32_t it = 0;                          // tiles done by this warp (mbarrier phase)
+  uint32_t staged[2] = {gwarp < ntiles ? 1u : 0u, 0u};   // tensor copies issued per kind
+  bool dead = false;
+  for (int64_t tile = gwarp; tile < ntiles && !dead; tile += nwarps, ++it) {
     const int nr = (int)imin64((int64_t)G::ROWS, npairs - tile * G::ROWS);
     const int64_t next = tile + nwarps;
 #pragma unroll 1
@@ -462,23 +514,36 @@ append_kernel(AppendParams p) {
       // prefetch one half-tile ahead: this tile's V rows, or the next tile's K rows
       if (kind == 0) {
         stage(tile, tb, 1);
+        ++staged[1];
       } else if (next < ntiles) {
         resolve(next, tb ^ 1);
         stage(next, tb ^ 1, 0);
+        ++staged[0];
       }
       cp_async_commit();
-      cp_async_wait<1>();
+      if (p.tma_in) {
+        const bool ok = mbar_wait(&bars[kind], it & 1u, kWaitMs);
+        if (!__all_sync(0xffffffffu, ok)) {     // the warp gives up together
+          if (lane == 0) report_error(p.err, TQ_DEVERR_TIMEOUT);
+          dead = true;
+          break;
+        }
+      } else {
+        cp_async_wait<1>();
+      }
       __syncwarp();
       const int bits = p.bits[kind];
       const int rwords = kind ? vwords : kwords;          // packed words + norm word
       uint64_t xp[32];
-      load_signed<Tin>(xp, in_s + kind * G::ROWS * SM::INPITCH + rl * SM::INPITCH +
-                               part * 64 * InType<Tin>::kBytes,
-                       smask + part * 64);
+      load_signed<Tin>(xp, row0 + (uint32_t)(kind * SM::KIND), smask + part * 64);
       float n;
       const float r = rotate_row<D>(xp, part, &n);
       const bool bad = !(fabsf(n) <= 3.402823466e38f);   // inf or NaN
-      uint32_t* orow = out_s + rl * out_pitch + (kind ? kwords : 0);
+      if (kind == 0 && p.bulk_out) {    // the previous tile's slots have been read out
+        bulk_wait_read_all();
+        __syncwarp();
+      }
+      uint32_t* orow = out_s + rl * swords + (kind ? kwords : 0);
       const EncodeTables* t = &tabs[kind];
       const int wpl = (rwords - 1) / G::TPR;               // words per lane
       uint32_t* mine = orow + part * wpl;
@@ -501,21 +566,41 @@ append_kernel(AppendParams p) {
       if (part == G::TPR - 1) orow[rwords - 1] = bad ? 0x7FC00000u : __float_as_uint(n);
       __syncwarp();
     }
-    // write back the tile's full slots: lanes run over (pair, word)
-    {
+    if (dead) break;
+    if (p.bulk_out) {
+      // one bulk store per token run of the tile (its heads' slots are contiguous)
+      fence_proxy_async_smem();
+      __syncwarp();
+      const int hr = p.run_heads;
+      if (lane * hr < nr) {
+        const int64_t off = dst_s[tb * G::ROWS + lane * hr];
+        if (off >= 0)
+          bulk_s2g(p.pages + off, out_s + lane * hr * swords, (uint32_t)(hr * swords * 4));
+        bulk_commit();
+      }
+    } else {
+      // write back the tile's full slots: lanes run over (pair, word)
       int rr = 0, w = lane;
       while (w >= swords) { w -= swords; ++rr; }
       for (; rr < nr;) {
         const int64_t off = dst_s[tb * G::ROWS + rr];
-        if (off >= 0) ((uint32_t*)(p.pages + off))[w] = out_s[rr * out_pitch + w];
+        if (off >= 0) ((uint32_t*)(p.pages + off))[w] = out_s[rr * swords + w];
         w += 32;
         while (w >= swords) { w -= swords; ++rr; }
       }
+      __syncwarp();
     }
-    __syncwarp();
     tb ^= 1;
   }
   cp_async_wait<0>();
+  if (p.tma_in && dead) {
+    // let the tensor copies still in flight land before the CTA's shared memory goes
+    // (each kind's copies complete in order; `it` of them were consumed or abandoned)
+    for (int kind = 0; kind < 2; ++kind)
+      for (uint32_t c = it; c < staged[kind]; ++c)
+        if (!mbar_wait(&bars[kind], c & 1u, kWaitMs)) break;
+  }
+  bulk_wait_all();
 }
 
 // Test export: the rotation of tq_quantize_append, written out as fp32 u and n.
@@ -523,30 +608,32 @@ template <int D, typename Tin>
 __global__ void __launch_bounds__(kAppendWarps * 32)
 rotate_unit_kernel(RotateParams p) {
   using G = AppendGeom<D>;
-  constexpr int RB = D * InType<Tin>::kBytes;
-  constexpr int INPITCH = RB + 16;
+  using SM = AppendSmem<D, Tin>;
   extern __shared__ __align__(16) uint8_t smem[];
   uint32_t* smask = (uint32_t*)smem;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint8_t* in_s = smem + 4 * D + warp * G::ROWS * INPITCH;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t in_off = ((sbase + 4 * D + 1023u) & ~1023u) - sbase;
+  uint8_t* in_s = smem + in_off + warp * SM::KIND;
   for (int j = threadIdx.x; j < D; j += blockDim.x) smask[j] = sign_mask_at(p.sign_seed, j);
   __syncthreads();
   const int rl = lane % G::ROWS, part = lane / G::ROWS;
+  const uint32_t row = smem_u32(in_s) + (uint32_t)((part * G::ROWS + rl) * SM::PB) +
+                       (uint32_t)((rl & 7) << 4);
   const int64_t ntiles = (p.rows + G::ROWS - 1) / G::ROWS;
   for (int64_t tile = (int64_t)blockIdx.x * kAppendWarps + warp; tile < ntiles;
        tile += (int64_t)gridDim.x * kAppendWarps) {
     const int64_t r0 = tile * G::ROWS;
     const int nr = (int)imin64((int64_t)G::ROWS, p.rows - r0);
     const Tin* base = (const Tin*)p.x;
-    stage_rows<RB>(in_s, INPITCH, nr,
-                   [&](int r) { return (const void*)(base + (r0 + r) * p.x_row_stride); },
-                   p.align_mode, lane);
+    stage_rows<SM::RB, SM::PB, G::ROWS>(
+        in_s, nr, [&](int r) { return (const void*)(base + (r0 + r) * p.x_row_stride); },
+        p.align_mode, lane);
     cp_async_commit();
     cp_async_wait<0>();
     __syncwarp();
     uint64_t xp[32];
-    load_signed<Tin>(xp, in_s + rl * INPITCH + part * 64 * InType<Tin>::kBytes,
-                     smask + part * 64);
+    load_signed<Tin>(xp, row, smask + part * 64);
     float n;
     const float r = rotate_row<D>(xp, part, &n);
     if (rl < nr) {

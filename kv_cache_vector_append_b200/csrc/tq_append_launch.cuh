@@ -7,7 +7,8 @@
 namespace tq {
 
 template <int D, typename Tin>
-tq_status launch_append_t(const AppendParams& p, const DeviceInfo& di, cudaStream_t st) {
+tq_status launch_append_t(const AppendParams& p, const AppendMaps& maps, const DeviceInfo& di,
+                          cudaStream_t st) {
   const size_t smem = AppendSmem<D, Tin>::bytes(p.bits[0], p.bits[1]);
   if ((int)smem > di.max_smem_optin) return TQ_ERR_UNSUPPORTED;
   auto kern = append_kernel<D, Tin>;
@@ -24,14 +25,14 @@ tq_status launch_append_t(const AppendParams& p, const DeviceInfo& di, cudaStrea
   const int64_t max_ctas = (int64_t)di.num_sms * per_sm;
   const int64_t want = (tiles + kAppendWarps - 1) / kAppendWarps;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, max_ctas));
-  kern<<<grid, kAppendWarps * 32, smem, st>>>(p);
+  kern<<<grid, kAppendWarps * 32, smem, st>>>(p, maps);
   return launch_status();
 }
 
 template <int D, typename Tin>
 tq_status launch_rotate_t(const RotateParams& p, const DeviceInfo& di, cudaStream_t st) {
   using G = AppendGeom<D>;
-  const size_t smem = 4 * D + kAppendWarps * G::ROWS * (D * InType<Tin>::kBytes + 16);
+  const size_t smem = 4 * D + 1024 + kAppendWarps * AppendSmem<D, Tin>::KIND;
   auto kern = rotate_unit_kernel<D, Tin>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
@@ -44,14 +45,14 @@ tq_status launch_rotate_t(const RotateParams& p, const DeviceInfo& di, cudaStrea
 }
 
 #define TQ_DECLARE_APPEND(D_, NAME_, T_)                                                  \
-  tq_status launch_append_d##D_##_##NAME_(const AppendParams& p, const DeviceInfo& di,   \
-                                          cudaStream_t st);                              \
+  tq_status launch_append_d##D_##_##NAME_(const AppendParams& p, const AppendMaps& maps, \
+                                          const DeviceInfo& di, cudaStream_t st);        \
   tq_status launch_rotate_d##D_##_##NAME_(const RotateParams& p, const DeviceInfo& di,   \
                                           cudaStream_t st);
 #define TQ_DEFINE_APPEND(D_, NAME_, T_)                                                   \
-  tq_status launch_append_d##D_##_##NAME_(const AppendParams& p, const DeviceInfo& di,   \
-                                          cudaStream_t st) {                             \
-    return launch_append_t<D_, T_>(p, di, st);                                          \
+  tq_status launch_append_d##D_##_##NAME_(const AppendParams& p, const AppendMaps& maps, \
+                                          const DeviceInfo& di, cudaStream_t st) {       \
+    return launch_append_t<D_, T_>(p, maps, di, st);                                    \
   }                                                                                      \
   tq_status launch_rotate_d##D_##_##NAME_(const RotateParams& p, const DeviceInfo& di,   \
                                           cudaStream_t st) {                             \

@@ -60,7 +60,6 @@ namespace tq {
 
 constexpr int kBlockSize = 16;        // tokens per page block
 constexpr int kMaxStages = 8;         // deepest stage ring
-constexpr uint32_t kWaitMs = 2000;    // a stage wait gives up after about 2 s
 constexpr float kLazyRescale = 8.0f;  // log2 units
 constexpr int kLutRow = 256;          // bytes per table entry (K half, V half)
 

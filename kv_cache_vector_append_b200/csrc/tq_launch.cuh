@@ -40,8 +40,8 @@ inline tq_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 
-tq_status launch_append_any(int dim, int dtype, const AppendParams& p, const DeviceInfo& di,
-                            cudaStream_t st);
+tq_status launch_append_any(int dim, int dtype, const AppendParams& p, const AppendMaps& maps,
+                            const DeviceInfo& di, cudaStream_t st);
 tq_status launch_rotate_any(int dim, int dtype, const RotateParams& p, const DeviceInfo& di,
                             cudaStream_t st);
 tq_status launch_decode_d64(int kb, int vb, const DecodeParams& p, const DecodePlan& plan,

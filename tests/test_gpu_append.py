@@ -77,6 +77,65 @@ def test_bit_exact_fp16_input():
     _bit_exact_case(tq, wl)
 
 
+# Tiles of 2048 / D consecutive (token, head) pairs are staged by tensor copies and
+# stored by one bulk copy per token when h_kv divides the tile (or the tile divides
+# h_kv) and the pool's slots are packed with 16-byte alignment; h_kv = 3 above takes
+# the cp.async staging and the per-word stores.  seq lengths leave ragged last tiles.
+@pytest.mark.parametrize("d,h_kv,dtype,kb,vb", [
+    (64, 8, "bfloat16", 4, 4), (128, 8, "bfloat16", 4, 4), (256, 8, "bfloat16", 3, 2),
+    (128, 32, "bfloat16", 4, 2), (128, 2, "bfloat16", 8, 1), (128, 1, "bfloat16", 4, 4),
+    (64, 16, "bfloat16", 2, 2), (256, 16, "bfloat16", 4, 4), (128, 8, "float32", 4, 4)])
+def test_bit_exact_tile_copy_modes(d, h_kv, dtype, kb, vb):
+    tq = _tq()
+    _bit_exact_case(tq, W.generate(_mini(d, kb, vb, dtype=dtype, h_kv=h_kv, batch=3, seq=41,
+                                         seed=h_kv + d)))
+
+
+def test_bit_exact_fp16_tile_copy():
+    tq = _tq()
+    wl = W.generate(_mini(128, 4, 4, dtype="float32", h_kv=8, batch=2, seq=33))
+    wl.k = wl.k.to(torch.float16)
+    wl.v = wl.v.to(torch.float16)
+    _bit_exact_case(tq, wl)
+
+
+def test_strided_inputs_match_contiguous():
+    """K and V as views into wider buffers (head stride 2D, token stride 2 h_kv D) give
+    the same pages as contiguous inputs."""
+    tq = _tq()
+    wl = W.generate(_mini(128, 4, 2, h_kv=8, batch=2, seq=45))
+    ref, cb = gpu_append(tq, wl)
+    t, h, d = wl.k.shape
+    wide_k = torch.zeros(t, h, 2 * d, dtype=wl.k.dtype)
+    wide_v = torch.zeros(t, h, 2 * d, dtype=wl.v.dtype)
+    wide_k[..., :d] = wl.k
+    wide_v[..., d:] = wl.v
+    k = wide_k.cuda()[..., :d]
+    v = wide_v.cuda()[..., d:]
+    pages = W.empty_pages(wl, device="cuda")
+    sm = torch.from_numpy(wl.slot_mapping.astype(np.int64)).cuda()
+    tq.quantize_append(pages, sm, k, v, cb, wl.spec.sign_seed)
+    torch.cuda.synchronize()
+    assert torch.equal(pages, ref)
+
+
+def test_skipped_tokens_with_token_stores():
+    """Tokens with slot -1 leave their slots untouched when slots are stored per token."""
+    tq = _tq()
+    wl = W.generate(_mini(128, 4, 4, h_kv=8, batch=2, seq=40))
+    sm = wl.slot_mapping.copy()
+    sm[1::3] = -1
+    pages, _ = gpu_append(tq, wl, fill=0xA5, slot_mapping=sm)
+    p = pages.cpu().numpy()
+    written = np.zeros(p.shape[:2], dtype=bool)
+    ok = sm >= 0
+    written[sm[ok] // 16, sm[ok] % 16] = True
+    assert np.all(p[~written] == 0xA5)
+    full, _ = gpu_append(tq, wl)
+    f = full.cpu().numpy()
+    assert np.array_equal(p[written], f[written])
+
+
 def _end_to_end(tq, wl, tokens=None, max_rows=None):
     """Oracle fp64 vs GPU: >= 99.99% identical codes, every mismatch within 1e-5 of a
     boundary; norms within 1e-6 relative."""
