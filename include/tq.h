@@ -139,6 +139,15 @@ TQ_API tq_status tq_slot_bytes(int32_t dim, int32_t k_bits, int32_t v_bits, int3
  *   sign_seed    SplitMix64 seed of the rotation signs.
  *   k_bits, v_bits  1..8.  D must be 64, 128 or 256.
  * Two tokens mapped to the same slot race (either row may win).
+ * Fast paths (same results, chosen per call on the host):
+ *   - k and v are staged by tensor copies when they are 16-bit, 16-byte aligned with
+ *     token and head strides that are multiples of 8 elements, and H_kv divides
+ *     2048/D or is a multiple of it;
+ *   - each token's slots are stored with one bulk copy when, in addition to that H_kv
+ *     rule, slot_stride == tq_slot_bytes(...), pages is 16-byte aligned with block and
+ *     row strides that are multiples of 16, and the token's run of slots is a
+ *     multiple of 16 bytes.
+ *   Other layouts take lane-wise copies.
  * Errors: TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED (nothing enqueued), TQ_ERR_CUDA. */
 TQ_API tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_tensor k,
                              tq_tensor v, const tq_codebooks* cb, uint64_t sign_seed,
