@@ -123,3 +123,41 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(ValueError):
         tq.quantize_append(cpu, torch.zeros(1, dtype=torch.int64), torch.zeros(1, 1, 128),
                            torch.zeros(1, 1, 128), None, 0)
+
+
+def test_host_limits_and_empty_inputs_on_cpu():
+    # Limits and empty inputs are settled by host validation alone (no GPU here).
+    tq, B, lib = _lib()
+    cbs = B.CodebooksDesc()
+    cbs.k = B.CodebookDesc(128, 4, 0x20000, 0x30000)
+    cbs.v = B.CodebookDesc(128, 4, 0x40000, 0x50000)
+
+    def app(pages, sm, k, v):
+        return lib.tq_quantize_append(pages, sm, k, v, ctypes.byref(cbs), 0, 4, 4, None)
+
+    # no tokens: nothing to do, success without touching the device
+    empty = _fake([0, 2, 128], B.BF16, strides=[256, 128, 1])
+    assert app(_fake([4, 16, 2, 136], B.U8), _fake([0], B.I64, strides=[1]), empty, empty) == B.OK
+    # 2^28 tokens x 8 heads reaches the 32-bit row-index limit
+    t = 1 << 28
+    big = _fake([t, 8, 128], B.BF16, strides=[1024, 128, 1])
+    assert app(_fake([4, 16, 8, 136], B.U8, strides=[17408, 1088, 136, 1]),
+               _fake([t], B.I64, strides=[1]), big, big) == B.ERR_UNSUPPORTED
+    # slot stride must be a multiple of 8 bytes
+    k = _fake([10, 2, 128], B.BF16)
+    assert app(_fake([4, 16, 2, 140], B.U8), _fake([10], B.I64), k, k) == B.ERR_INVALID_ARG
+
+    def dec(h_q, h_kv, d, cb):
+        q = _fake([2, h_q, d], B.BF16, strides=[h_q * d, d, 1])
+        pages = _fake([4, 16, h_kv, 136 if d == 128 else 264], B.U8,
+                      strides=[16 * h_kv * (136 if d == 128 else 264), h_kv * (136 if d == 128 else 264),
+                               136 if d == 128 else 264, 1])
+        return lib.tq_paged_decode(q, q, pages, _fake([2, 4], B.I32), _fake([2], B.I32),
+                                   ctypes.byref(cb), 0, 0.1, None)
+
+    # more KV heads than the decode kernel's warps: 32 at D=128, 16 at D=256
+    assert dec(32, 32, 128, cbs) == B.ERR_UNSUPPORTED
+    cb256 = B.CodebooksDesc()
+    cb256.k = B.CodebookDesc(256, 4, 0x20000, 0x30000)
+    cb256.v = B.CodebookDesc(256, 4, 0x40000, 0x50000)
+    assert dec(16, 16, 256, cb256) == B.ERR_UNSUPPORTED
