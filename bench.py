@@ -210,12 +210,14 @@ def oracle_sample_step(wl, tables, n_append=1024, n_decode_tokens=2048, seq=0):
     # the untimed part fills the decode range; the timed part re-appends n_app tokens
     pages = O.quantize_append(pages, slots, k, v, kt, vt, spec.sign_seed)
     t0 = time.perf_counter()
+    c0 = time.process_time()
     pages = O.quantize_append(pages, slots[:n_app], k[:n_app], v[:n_app], kt, vt,
                               spec.sign_seed)
     q = wl.q[seq:seq + 1].float().numpy().astype(np.float64)
     O.paged_decode(q, pages, wl.block_table[seq:seq + 1], np.array([n_dec], dtype=np.int32),
                    kt, vt, spec.sign_seed, spec.scale)
     dt = time.perf_counter() - t0
+    oracle_sample_step.cpu_seconds = time.process_time() - c0
     nbytes = append_bytes(spec, n_app) + decode_bytes(spec, [n_dec])[0]
     desc = (f"{n_app} tokens x {spec.num_kv_heads} KV heads appended + 1 sequence x {n_dec} "
             f"tokens x {spec.num_q_heads} q heads decoded")
@@ -226,17 +228,24 @@ def cpu_baseline(wl, tables, min_seconds=10.0, max_samples=64):
     """The oracle timed on host cores over repeated bounded samples (one per
     sequence, cycling) until at least min_seconds of oracle work has run."""
     oracle_sample_step(wl, tables, 256, 512)   # warm caches
-    total_t = total_b = 0.0
+    total_t = total_b = total_cpu = 0.0
     n = 0
     desc = ""
     while n < max_samples and (total_t < min_seconds or n == 0):
         dt, nb, desc = oracle_sample_step(wl, tables, seq=n)
         total_t += dt
         total_b += nb
+        total_cpu += oracle_sample_step.cpu_seconds
         n += 1
-    return {"value": total_b / total_t / 1e9, "unit": "GB/s", "cores": blas_threads(),
+    return {"value": total_b / total_t / 1e9, "unit": "GB/s",
+            "cores": effective_cores(total_cpu, total_t), "threads_available": blas_threads(),
             "kind": "oracle", "sample": f"{n} samples (sequences 0..{n - 1}, cycling) of: {desc}",
             "seconds": total_t}
+
+
+def effective_cores(cpu_seconds, wall_seconds):
+    """Host cores the oracle kept busy on average: process CPU time over wall time."""
+    return round(max(1.0, cpu_seconds / wall_seconds), 1) if wall_seconds > 0 else 1.0
 
 
 def oracle_tables(spec):
@@ -265,14 +274,15 @@ def run_reference(args):
     tables = oracle_tables(spec)
     for i in range(args.warmup):
         oracle_sample_step(wl, tables, seq=i)
-    total_t = total_b = 0.0
+    total_t = total_b = total_cpu = 0.0
     desc = ""
     for i in range(args.steps):
         dt, nb, desc = oracle_sample_step(wl, tables, seq=args.warmup + i)
         total_t += dt
         total_b += nb
+        total_cpu += oracle_sample_step.cpu_seconds
     value = total_b / total_t / 1e9
-    cores = blas_threads()
+    cores = effective_cores(total_cpu, total_t)
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
@@ -283,7 +293,8 @@ def run_reference(args):
                        "q_heads": spec.num_q_heads, "kv_heads": spec.num_kv_heads,
                        "k_bits": spec.k_bits, "v_bits": spec.v_bits,
                        "parallelism": "replicas" if args.gpus > 1 else "single"},
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores,
+                             "threads_available": blas_threads(), "kind": "oracle",
                              "sample": desc + " per step"},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
