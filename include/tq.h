@@ -171,6 +171,10 @@ TQ_API tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_
  *                TQ_DEVERR_SEQLEN_RANGE and the sequence gives 0.
  *   scale        softmax scale (typically 1/sqrt(D)).
  * H_q must be a multiple of H_kv with H_q / H_kv <= 16; block_size must be 16.
+ * H_kv is at most 16 (8 when D = 256 or H_q / H_kv > 8), and a staged block of all
+ * KV heads plus the code tables must fit in shared memory: with 8-bit tables that
+ * excludes 16 KV heads at D = 128 and 8 at D = 256 (TQ_ERR_UNSUPPORTED;
+ * tq_decode_plan_probe tells in advance).
  * One cooperative kernel launch: the CTAs that share a sequence wait for one another
  * (bounded; TQ_DEVERR_TIMEOUT) before merging its partial results.
  * Uses the per-device workspace (tq_set_workspace, or allocated by the library on
@@ -237,6 +241,20 @@ TQ_API tq_status tq_get_device_error(int32_t* out, void* stream);
  * reproduces the kernel's codes bit for bit). */
 TQ_API tq_status tq_rotate_unit(tq_tensor u, tq_tensor norm, tq_tensor x, uint64_t sign_seed,
                          void* stream);
+
+/* Test export of the decode kernel's shared-memory plan for one call geometry on a
+ * device described by num_sms, max_smem_optin (bytes one CTA may use) and
+ * dyn_smem_base (the shared-window address where dynamic shared memory starts).
+ * Host only: no device call.  out[14] receives, in order: wph, nst, row_pitch,
+ * stage_bytes, lut_win, lut_off, lut_bytes, stage_lo_off, stage_hi_off, n_low,
+ * misc_off, smem bytes, copy_mode (1: 2-D tensor box, 0: 1-D bulk copy), warps per CTA.
+ * Errors: TQ_ERR_INVALID_ARG for out == NULL or non-positive sizes; TQ_ERR_UNSUPPORTED
+ * when no layout fits. */
+TQ_API tq_status tq_decode_plan_probe(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                      int32_t head_dim, int32_t k_bits, int32_t v_bits,
+                                      int32_t slot_stride, int32_t max_blocks, int32_t num_sms,
+                                      int32_t max_smem_optin, uint32_t dyn_smem_base,
+                                      int64_t* out);
 
 /* Static description of a status code (never NULL). */
 TQ_API const char* tq_status_string(tq_status status);

@@ -27,7 +27,7 @@ DEVERR_LAYOUT = 0x20
 
 EXPORTED = ("tq_slot_bytes", "tq_quantize_append", "tq_paged_decode", "tq_paged_decode_noalloc",
             "tq_decode_workspace_size", "tq_set_workspace", "tq_get_device_error",
-            "tq_rotate_unit", "tq_status_string", "tq_version")
+            "tq_rotate_unit", "tq_decode_plan_probe", "tq_status_string", "tq_version")
 
 
 class TQError(RuntimeError):
@@ -78,6 +78,8 @@ def _load():
     lib.tq_set_workspace.argtypes = [ctypes.c_void_p, ctypes.c_size_t]
     lib.tq_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p]
     lib.tq_rotate_unit.argtypes = [T, T, T, ctypes.c_uint64, ctypes.c_void_p]
+    lib.tq_decode_plan_probe.argtypes = [ctypes.c_int32] * 10 + [ctypes.c_uint32,
+                                                                 ctypes.POINTER(ctypes.c_int64)]
     lib.tq_status_string.argtypes = [ctypes.c_int]
     lib.tq_status_string.restype = ctypes.c_char_p
     lib.tq_version.restype = ctypes.c_char_p
@@ -246,6 +248,23 @@ def rotate_unit(u, norm, x, sign_seed: int, stream=None) -> None:
     st = _stream_handle(stream, x.device)
     _check(_load().tq_rotate_unit(_desc(u), _desc(norm), _desc(x), ctypes.c_uint64(sign_seed), st),
            "tq_rotate_unit")
+
+
+DECODE_PLAN_FIELDS = ("wph", "nst", "row_pitch", "stage_bytes", "lut_win", "lut_off", "lut_bytes",
+                      "stage_lo_off", "stage_hi_off", "n_low", "misc_off", "smem", "copy_mode",
+                      "warps")
+
+
+def decode_plan_probe(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                      k_bits: int, v_bits: int, slot_stride: int, max_blocks: int,
+                      num_sms: int, max_smem_optin: int, dyn_smem_base: int):
+    """Host-only test export: the decode kernel's shared-memory plan as a dict, or the
+    status code when no plan is returned."""
+    out = (ctypes.c_int64 * len(DECODE_PLAN_FIELDS))()
+    s = _load().tq_decode_plan_probe(batch, num_q_heads, num_kv_heads, head_dim, k_bits, v_bits,
+                                     slot_stride, max_blocks, num_sms, max_smem_optin,
+                                     dyn_smem_base, out)
+    return dict(zip(DECODE_PLAN_FIELDS, list(out))) if s == OK else s
 
 
 def decode_workspace_size(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,

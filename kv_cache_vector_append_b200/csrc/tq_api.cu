@@ -525,6 +525,30 @@ tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_tensor 
   return launch_append_any(D, k.dtype, p, maps, ds->info, as_stream(stream));
 }
 
+tq_status tq_decode_plan_probe(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                               int32_t head_dim, int32_t k_bits, int32_t v_bits,
+                               int32_t slot_stride, int32_t max_blocks, int32_t num_sms,
+                               int32_t max_smem_optin, uint32_t dyn_smem_base, int64_t* out) {
+  if (out == nullptr || batch < 1 || num_q_heads < 1 || num_kv_heads < 1 || head_dim < 1 ||
+      slot_stride < 1 || max_blocks < 1 || num_sms < 1 || max_smem_optin < 1 ||
+      num_q_heads % num_kv_heads)
+    return TQ_ERR_INVALID_ARG;
+  DeviceInfo di;
+  di.num_sms = num_sms;
+  di.max_smem_optin = max_smem_optin;
+  di.dyn_smem_base = dyn_smem_base;
+  DecodePlan plan;
+  const tq_status s = plan_decode(batch, num_q_heads, num_kv_heads, head_dim, k_bits, v_bits,
+                                  slot_stride, max_blocks, true, di, &plan);
+  if (s != TQ_OK) return s;
+  const int64_t v[14] = {plan.wph,          plan.nst,          plan.row_pitch, plan.stage_bytes,
+                         plan.lut_win,      plan.lut_off,      plan.lut_bytes, plan.stage_lo_off,
+                         plan.stage_hi_off, plan.n_low,        plan.misc_off,  (int64_t)plan.smem,
+                         plan.copy_mode,    plan.maxw};
+  for (int i = 0; i < 14; ++i) out[i] = v[i];
+  return TQ_OK;
+}
+
 tq_status tq_rotate_unit(tq_tensor u, tq_tensor norm, tq_tensor x, uint64_t sign_seed,
                          void* stream) {
   if (!valid_tensor(x, 2) || !valid_tensor(u, 2) || !valid_tensor(norm, 1)) return TQ_ERR_INVALID_ARG;
