@@ -460,7 +460,14 @@ def encode_region(idx: np.ndarray, norm32: np.ndarray, bits: int) -> np.ndarray:
 
 
 def decode_region(region: np.ndarray, dim: int, bits: int):
-    """Split region bytes into (idx int64 (..., D), norm float32 (...))."""
+    """Split region bytes into (idx int64 (..., D), norm float32 (...)).
+
+    [TorbuQuant, "TQ4 page tensor": a K or V region is the packed indices, then
+    the fp32 norm].  The first ceil(D*bits/8) bytes are unpacked LSB-first
+    (``unpack_bits``); the next four bytes are the norm, little endian.  Pinned
+    against regions laid out by hand, bit by bit, with the norm written by
+    ``struct`` (tests/test_oracle_pack_encode.py).
+    """
     region = np.asarray(region, dtype=np.uint8)
     nb = (dim * bits + 7) // 8
     idx = unpack_bits(region[..., :nb], dim, bits)

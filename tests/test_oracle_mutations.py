@@ -114,3 +114,38 @@ def test_mutation_merge_missing_rescale(monkeypatch):
         return sum(p[2] for p in parts) / sum(p[1] for p in parts)
     monkeypatch.setattr(O, "merge_partials", bad)
     _fails(TA.test_rotated_domain_and_split_merge_equal_plain)
+
+
+def test_mutation_region_norm_offset(monkeypatch):
+    # the norm read four bytes early (from the last packed bytes)
+    def bad(region, dim, bits):
+        region = np.asarray(region, dtype=np.uint8)
+        nb = (dim * bits + 7) // 8
+        idx = O.unpack_bits(region[..., :nb], dim, bits)
+        norm = np.ascontiguousarray(region[..., nb - 4:nb]).view("<f4")[..., 0]
+        return idx, norm.astype(np.float32)
+    monkeypatch.setattr(O, "decode_region", bad)
+    _fails(TP.test_decode_region_reads_hand_built_regions, 4, 128)
+
+
+def test_mutation_region_norm_first(monkeypatch):
+    # the layout misread as [fp32 norm | packed codes]
+    def bad(region, dim, bits):
+        region = np.asarray(region, dtype=np.uint8)
+        nb = (dim * bits + 7) // 8
+        idx = O.unpack_bits(region[..., 4:4 + nb], dim, bits)
+        norm = np.ascontiguousarray(region[..., :4]).view("<f4")[..., 0]
+        return idx, norm.astype(np.float32)
+    monkeypatch.setattr(O, "decode_region", bad)
+    _fails(TP.test_decode_region_splits_a_padded_kv_slot, 128, 3, 2, 8)
+
+
+def test_mutation_region_big_endian_norm(monkeypatch):
+    def bad(region, dim, bits):
+        region = np.asarray(region, dtype=np.uint8)
+        nb = (dim * bits + 7) // 8
+        idx = O.unpack_bits(region[..., :nb], dim, bits)
+        norm = np.ascontiguousarray(region[..., nb:nb + 4]).view(">f4")[..., 0]
+        return idx, norm.astype(np.float32)
+    monkeypatch.setattr(O, "decode_region", bad)
+    _fails(TP.test_decode_region_reads_hand_built_regions, 2, 64)

@@ -1,6 +1,7 @@
 """Pins of the oracle's slot layout, bit packing, encode and slot writes."""
 import math
 import os
+import struct
 
 import numpy as np
 import pytest
@@ -165,3 +166,70 @@ def test_quantize_append_slot_placement():
             assert np.frombuffer(bytes(region[kb + vb - 4:kb + vb]), "<f4")[0] == vn
             assert np.all(region[kb + vb:] == 0xA5)   # padding untouched
     assert np.all(out[~written] == 0xA5)
+
+
+def _region_by_hand(idx, norm32, bits):
+    """Region bytes laid out by hand from the page diagram (TorbuQuant, "TQ4 page
+    tensor": packed indices, then the fp32 norm): code j occupies stream bits
+    [j*bits, (j+1)*bits), stream bit p is bit p % 8 of byte p // 8, and the norm
+    follows as four little-endian bytes (struct, not numpy)."""
+    nbytes = (len(idx) * bits + 7) // 8
+    out = bytearray(nbytes)
+    for j, code in enumerate(idx):
+        for k in range(bits):
+            if (int(code) >> k) & 1:
+                p = j * bits + k
+                out[p // 8] |= 1 << (p % 8)
+    return bytes(out) + struct.pack("<f", float(norm32))
+
+
+@pytest.mark.parametrize("bits", range(1, 9))
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_decode_region_reads_hand_built_regions(bits, d):
+    rng = np.random.default_rng(100 * d + bits)
+    for _ in range(3):
+        idx = rng.integers(0, 1 << bits, size=d)
+        # norms with four distinct bytes, so a shifted or reversed read shows
+        norm = np.float32(rng.uniform(0.5, 3000.0))
+        raw = _region_by_hand(idx, norm, bits)
+        assert len(raw) == O.region_bytes(d, bits)
+        got_idx, got_n = O.decode_region(np.frombuffer(raw, dtype=np.uint8), d, bits)
+        np.testing.assert_array_equal(got_idx, idx)
+        assert got_n.dtype == np.float32 and got_n == norm
+
+
+@pytest.mark.parametrize("d,kbits,vbits,pad", [(128, 4, 4, 0), (128, 3, 2, 8), (64, 8, 1, 16),
+                                               (256, 5, 7, 24)])
+def test_decode_region_splits_a_padded_kv_slot(d, kbits, vbits, pad):
+    # A whole slot: [K codes | K norm][V codes | V norm][padding], each region read
+    # back from its own byte range of the slot.
+    rng = np.random.default_rng(d + kbits + vbits + pad)
+    ki = rng.integers(0, 1 << kbits, size=(5, d))
+    vi = rng.integers(0, 1 << vbits, size=(5, d))
+    kn = rng.uniform(0.1, 50.0, size=5).astype(np.float32)
+    vn = rng.uniform(0.1, 50.0, size=5).astype(np.float32)
+    slots = np.array([np.frombuffer(_region_by_hand(ki[r], kn[r], kbits)
+                                    + _region_by_hand(vi[r], vn[r], vbits)
+                                    + b"\xa5" * pad, dtype=np.uint8) for r in range(5)])
+    kb, vb = O.region_bytes(d, kbits), O.region_bytes(d, vbits)
+    assert slots.shape == (5, kb + vb + pad)
+    gi, gn = O.decode_region(slots[:, :kb], d, kbits)
+    np.testing.assert_array_equal(gi, ki)
+    np.testing.assert_array_equal(gn, kn)
+    gi, gn = O.decode_region(slots[:, kb:kb + vb], d, vbits)
+    np.testing.assert_array_equal(gi, vi)
+    np.testing.assert_array_equal(gn, vn)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 8])
+def test_encode_region_matches_hand_layout_and_round_trips(bits):
+    d = 128
+    rng = np.random.default_rng(bits)
+    idx = rng.integers(0, 1 << bits, size=(4, d))
+    norm = rng.uniform(0.1, 9.0, size=4).astype(np.float32)
+    reg = O.encode_region(idx, norm, bits)
+    for r in range(4):
+        assert bytes(reg[r]) == _region_by_hand(idx[r], norm[r], bits)
+    gi, gn = O.decode_region(reg, d, bits)
+    np.testing.assert_array_equal(gi, idx)
+    np.testing.assert_array_equal(gn, norm)
