@@ -32,7 +32,8 @@
  *     sign_seed is set, else +1 (j = 0..D-1); the same signs serve K, V, q and
  *     every head; rotation y = (1/sqrt(D)) H (s * x), H the natural-order
  *     (Sylvester) Hadamard matrix;
- *   - norm: L2 norm of the input row, stored as fp32; unit coordinates u = y / n;
+ *   - norm: L2 norm of the input row, stored as fp32 (rows of any finite magnitude;
+ *     a norm beyond the fp32 range stores +inf); unit coordinates u = y / n;
  *   - code: idx = number of boundaries b_i with b_i < u (ties to the lower cell);
  *     a zero row stores norm 0 and codes idx(0); a row holding a non-finite value
  *     stores codes 0 and a quiet-NaN norm (0x7FC00000) and raises
@@ -170,13 +171,17 @@ TQ_API tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_
  *   seq_lens     i32 [B]; 0 <= seq_lens[b] <= max_blocks * block_size, otherwise
  *                TQ_DEVERR_SEQLEN_RANGE and the sequence gives 0.
  *   scale        softmax scale (typically 1/sqrt(D)).
+ * K and V code widths (cb->k.bits, cb->v.bits): each of 2, 3, 4 and 8, in any pair
+ * (TQ_ERR_UNSUPPORTED otherwise; tq_quantize_append takes 1..8).
  * H_q must be a multiple of H_kv with H_q / H_kv <= 16; block_size must be 16.
  * H_kv is at most 16 (8 when D = 256 or H_q / H_kv > 8), and a staged block of all
  * KV heads plus the code tables must fit in shared memory: with 8-bit tables that
  * excludes 16 KV heads at D = 128 and 8 at D = 256 (TQ_ERR_UNSUPPORTED;
  * tq_decode_plan_probe tells in advance).
  * One cooperative kernel launch: the CTAs that share a sequence wait for one another
- * (bounded; TQ_DEVERR_TIMEOUT) before merging its partial results.
+ * (bounded, about 2 s) before merging its partial results.  A wait that gives up raises
+ * TQ_DEVERR_TIMEOUT, leaves that sequence's output unwritten, and still returns the
+ * merge counters to zero, so the next call runs normally.
  * Uses the per-device workspace (tq_set_workspace, or allocated by the library on
  * the first call that needs more, and kept until process exit).
  * Errors: TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED / TQ_ERR_WORKSPACE (nothing
@@ -241,6 +246,17 @@ TQ_API tq_status tq_get_device_error(int32_t* out, void* stream);
  * reproduces the kernel's codes bit for bit). */
 TQ_API tq_status tq_rotate_unit(tq_tensor u, tq_tensor norm, tq_tensor x, uint64_t sign_seed,
                          void* stream);
+
+/* Test export for failure detection without a GPU fault (this library's own addition;
+ * the pages describe no counterpart).  The NEXT decode launch on the current device
+ * (tq_paged_decode or tq_paged_decode_noalloc) bounds its waits by `wait_ms`
+ * milliseconds instead of about 2 s, and its CTA number `withhold_cta` never announces
+ * its partial results.  So the CTAs that share a sequence with it give up waiting, raise
+ * TQ_DEVERR_TIMEOUT, and write no output for that sequence (a withheld CTA past the
+ * grid changes nothing).  One shot: later launches are normal.  Host only; nothing is
+ * enqueued.
+ * Errors: TQ_ERR_INVALID_ARG for withhold_cta < 0 or wait_ms outside 1..2000. */
+TQ_API tq_status tq_debug_inject_merge_stall(int32_t withhold_cta, int32_t wait_ms);
 
 /* Test export of the decode kernel's shared-memory plan for one call geometry on a
  * device described by num_sms, max_smem_optin (bytes one CTA may use) and

@@ -23,6 +23,8 @@ from ._binding import (  # noqa: F401
     DEVERR_NONFINITE,
     DEVERR_SEQLEN_RANGE,
     DEVERR_SLOT_RANGE,
+    DEVERR_TIMEOUT,
+    debug_inject_merge_stall,
     decode_workspace_size,
     get_device_error,
     library_path,

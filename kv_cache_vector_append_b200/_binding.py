@@ -27,7 +27,8 @@ DEVERR_LAYOUT = 0x20
 
 EXPORTED = ("tq_slot_bytes", "tq_quantize_append", "tq_paged_decode", "tq_paged_decode_noalloc",
             "tq_decode_workspace_size", "tq_set_workspace", "tq_get_device_error",
-            "tq_rotate_unit", "tq_decode_plan_probe", "tq_status_string", "tq_version")
+            "tq_rotate_unit", "tq_decode_plan_probe", "tq_debug_inject_merge_stall",
+            "tq_status_string", "tq_version")
 
 
 class TQError(RuntimeError):
@@ -80,6 +81,7 @@ def _load():
     lib.tq_rotate_unit.argtypes = [T, T, T, ctypes.c_uint64, ctypes.c_void_p]
     lib.tq_decode_plan_probe.argtypes = [ctypes.c_int32] * 10 + [ctypes.c_uint32,
                                                                  ctypes.POINTER(ctypes.c_int64)]
+    lib.tq_debug_inject_merge_stall.argtypes = [ctypes.c_int32, ctypes.c_int32]
     lib.tq_status_string.argtypes = [ctypes.c_int]
     lib.tq_status_string.restype = ctypes.c_char_p
     lib.tq_version.restype = ctypes.c_char_p
@@ -265,6 +267,14 @@ def decode_plan_probe(batch: int, num_q_heads: int, num_kv_heads: int, head_dim:
                                      slot_stride, max_blocks, num_sms, max_smem_optin,
                                      dyn_smem_base, out)
     return dict(zip(DECODE_PLAN_FIELDS, list(out))) if s == OK else s
+
+
+def debug_inject_merge_stall(withhold_cta: int, wait_ms: int) -> None:
+    """Test export: the next decode launch on the current device waits at most
+    ``wait_ms`` ms and its CTA ``withhold_cta`` never announces its partial results
+    (see include/tq.h)."""
+    _check(_load().tq_debug_inject_merge_stall(withhold_cta, wait_ms),
+           "tq_debug_inject_merge_stall")
 
 
 def decode_workspace_size(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -35,7 +36,9 @@ namespace {
 constexpr int kMaxDevices = 64;
 
 struct DeviceState {
-  unsigned int* err = nullptr;   // device address of g_tq_error_word
+  // device address of g_tq_error_word; published (release) last by the one-time set-up,
+  // so a non-null value means `info` is complete
+  std::atomic<unsigned int*> err{nullptr};
   void* user_ws = nullptr;
   size_t user_ws_bytes = 0;
   void* lib_ws = nullptr;
@@ -43,30 +46,42 @@ struct DeviceState {
   uint8_t* noalloc_scratch = nullptr;   // device address of g_tq_noalloc_scratch
   size_t counter_bytes = 0;             // largest merge-counter area a decode call used
   DeviceInfo info;
+  // one-shot test hook of the next decode launch (tq_debug_inject_merge_stall)
+  int32_t inject_withhold = -1;
+  uint32_t inject_wait_ms = 0;
 };
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 
+// The current device's state, set up on first use: the error word's address, the SM
+// count, the shared-memory limit and where dynamic shared memory starts.  The set-up
+// runs once per device under g_mu; other threads see the state only once it is whole.
 tq_status device_state(DeviceState** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TQ_ERR_CUDA;
   DeviceState& s = g_dev[dev];
-  if (s.err == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_tq_error_word) != cudaSuccess) return TQ_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&s.info.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return TQ_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&s.info.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
-        cudaSuccess)
-      return TQ_ERR_CUDA;
-    dyn_smem_base_probe<<<1, 1, 16>>>();
-    unsigned int base = 0;
-    if (cudaGetLastError() != cudaSuccess ||
-        cudaMemcpyFromSymbol(&base, g_tq_dyn_base, sizeof(base)) != cudaSuccess)
-      return TQ_ERR_CUDA;
-    s.info.dyn_smem_base = base;
-    s.err = (unsigned int*)p;
+  if (s.err.load(std::memory_order_acquire) == nullptr) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (s.err.load(std::memory_order_relaxed) == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_tq_error_word) != cudaSuccess) return TQ_ERR_CUDA;
+      DeviceInfo info;
+      if (cudaDeviceGetAttribute(&info.num_sms, cudaDevAttrMultiProcessorCount, dev) !=
+          cudaSuccess)
+        return TQ_ERR_CUDA;
+      if (cudaDeviceGetAttribute(&info.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                 dev) != cudaSuccess)
+        return TQ_ERR_CUDA;
+      dyn_smem_base_probe<<<1, 1, 16>>>();
+      unsigned int base = 0;
+      if (cudaGetLastError() != cudaSuccess ||
+          cudaMemcpyFromSymbol(&base, g_tq_dyn_base, sizeof(base)) != cudaSuccess)
+        return TQ_ERR_CUDA;
+      info.dyn_smem_base = base;
+      s.info = info;
+      s.err.store((unsigned int*)p, std::memory_order_release);
+    }
   }
   *out = &s;
   return TQ_OK;
@@ -391,19 +406,23 @@ tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tens
   p.smem_end = (int32_t)plan.smem;
   p.part = (float*)(ws + plan.part_off);
   p.counters = (unsigned int*)(ws + plan.counters_off);
+  p.wait_ms = kWaitMs;
+  p.withhold_cta = -1;
   {
     std::lock_guard<std::mutex> lock(g_mu);
     ds->counter_bytes = std::max(ds->counter_bytes, plan.part_off);
+    if (ds->inject_wait_ms > 0) {
+      p.wait_ms = ds->inject_wait_ms;
+      p.withhold_cta = ds->inject_withhold;
+      ds->inject_wait_ms = 0;
+      ds->inject_withhold = -1;
+    }
   }
-  p.err = ds->err;
+  p.err = ds->err.load(std::memory_order_relaxed);
 
   const int64_t steps_upper = (int64_t)B * ((max_blocks + plan.wph - 1) / plan.wph);
   cudaStream_t st = as_stream(stream);
-  switch (D) {
-    case 64: return launch_decode_d64(kbits, vbits, p, plan, tmap, steps_upper, st);
-    case 128: return launch_decode_d128(kbits, vbits, p, plan, tmap, steps_upper, st);
-    default: return launch_decode_d256(kbits, vbits, p, plan, tmap, steps_upper, st);
-  }
+  return launch_decode_any(D, kbits, vbits, p, plan, tmap, steps_upper, st);
 }
 
 }  // namespace
@@ -493,7 +512,7 @@ tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_tensor 
   p.region_off[0] = 0;
   p.region_off[1] = kb;
   p.sign_seed = sign_seed;
-  p.err = ds->err;
+  p.err = ds->err.load(std::memory_order_relaxed);
   const int es = dtype_size(k.dtype);
   p.align_mode = std::min(align_mode_of(k.data, es, {k.stride[0], k.stride[1]}),
                           align_mode_of(v.data, es, {v.stride[0], v.stride[1]}));
@@ -615,9 +634,10 @@ tq_status tq_get_device_error(int32_t* out, void* stream) {
   if (s != TQ_OK) return s;
   cudaStream_t st = as_stream(stream);
   unsigned int h = 0;
-  if (cudaMemcpyAsync(&h, ds->err, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+  unsigned int* err = ds->err.load(std::memory_order_relaxed);
+  if (cudaMemcpyAsync(&h, err, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess)
     return TQ_ERR_CUDA;
-  if (cudaMemsetAsync(ds->err, 0, sizeof(unsigned int), st) != cudaSuccess) return TQ_ERR_CUDA;
+  if (cudaMemsetAsync(err, 0, sizeof(unsigned int), st) != cudaSuccess) return TQ_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return TQ_ERR_CUDA;
   if (h != 0) {
     // a launch that reported an error may have stopped with merge counters raised:
@@ -636,6 +656,17 @@ tq_status tq_get_device_error(int32_t* out, void* stream) {
     }
   }
   *out = (int32_t)h;
+  return TQ_OK;
+}
+
+tq_status tq_debug_inject_merge_stall(int32_t withhold_cta, int32_t wait_ms) {
+  if (withhold_cta < 0 || wait_ms < 1 || wait_ms > (int32_t)kWaitMs) return TQ_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  tq_status s = device_state(&ds);
+  if (s != TQ_OK) return s;
+  std::lock_guard<std::mutex> lock(g_mu);
+  ds->inject_withhold = withhold_cta;
+  ds->inject_wait_ms = (uint32_t)wait_ms;
   return TQ_OK;
 }
 

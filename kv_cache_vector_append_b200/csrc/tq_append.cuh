@@ -259,20 +259,93 @@ __device__ __forceinline__ void load_signed(uint64_t (&xp)[32], uint32_t row,
   }
 }
 
-// The rotation shared by quantize-append and its test export.  On entry xp holds
-// this lane's 64 sign-flipped input elements (coordinates 64*part .. 64*part+63 of
-// the row) after the first butterfly stage (load_signed); on exit it holds the
-// unnormalised transform H (s * x) of those coordinates, and the function returns r
-// with u = x * r; *norm_out = ||x||_2.
-// Order of operations (fixed, so the export reproduces the kernel exactly):
-//   FWHT butterflies in stages h = 1 (in load_signed), 2, 4, ..., 32 in registers, then
-//   h = 64, 128 across the lanes of the row; ss = sum of squares of the transformed
-//   coordinates: even and odd coordinates accumulated separately by fused
-//   multiply-add in register order, added, then the lanes of a row add their sums
-//   pairwise (xor butterfly over the part bits); n = sqrt(ss / D) (IEEE);
-//   r = 1 / (n * sqrt(D)) (IEEE reciprocal), or 0 when n == 0.
+// 2^k as a float, for -126 <= k <= 127.
+__device__ __forceinline__ float pow2f(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
+
+// floor(log2 x) of the positive finite float with bit pattern b (normal or subnormal).
+__device__ __forceinline__ int exponent_of(uint32_t b) {
+  return b >= 0x00800000u ? (int)(b >> 23) - 127 : (31 - __clz((int)b)) - 149;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ uint32_t scale_bits(uint32_t w, float s1, float s2) {
+  return __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(w), s1), s2));
+}
+
+// Rare path of rotate_row.  Every lane of the warp takes part (the row maximum is
+// combined over the row's lanes).  For a row with `need` set that holds only finite
+// values, not all zero: e = floor(log2 max|x|), and this lane's 64 staged elements are
+// multiplied in place by 2^-e (two power-of-two factors, both normal floats; the
+// product is exact unless it leaves the normal range, and the 16-bit formats share
+// fp32's exponent range for bf16, while f16 rows never need it); returns e, else 0.
+// *bad = the row holds an infinity or NaN.
+template <int D, typename Tin>
+__device__ __noinline__ int rescale_staged_row(uint32_t row, bool need, bool* bad) {
+  using G = AppendGeom<D>;
+  constexpr int NCH = 64 * (int)sizeof(Tin) / 16;   // 16-byte chunks of the part row
+  uint32_t mx = 0u;                                  // |x| as fp32 bits (integer order)
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    const uint4 q = lds128(row ^ (uint32_t)(16 * c));
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if constexpr (sizeof(Tin) == 4) {
+        mx = max(mx, w[k] & 0x7fffffffu);
+      } else if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
+        mx = max(mx, (w[k] << 16) & 0x7fffffffu);
+        mx = max(mx, w[k] & 0x7fff0000u);
+      } else {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+        mx = max(mx, __float_as_uint(f.x) & 0x7fffffffu);
+        mx = max(mx, __float_as_uint(f.y) & 0x7fffffffu);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 1; m < G::TPR; m <<= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, G::ROWS * m));
+  *bad = mx >= 0x7f800000u;
+  if (!need || *bad || mx == 0u) return 0;
+  const int e = exponent_of(mx);
+  const float s1 = pow2f(-e / 2), s2 = pow2f(-e - (-e / 2));
+#pragma unroll 1
+  for (int c = 0; c < NCH; ++c) {
+    const uint32_t a = row ^ (uint32_t)(16 * c);
+    const uint4 q = lds128(a);
+    uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if constexpr (sizeof(Tin) == 4) {
+        w[k] = scale_bits(w[k], s1, s2);
+      } else if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
+        const uint32_t lo = scale_bits(w[k] << 16, s1, s2) >> 16;   // exact: low bits are 0
+        const uint32_t hi = scale_bits(w[k] & 0xffff0000u, s1, s2) & 0xffff0000u;
+        w[k] = hi | lo;
+      } else {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+        const __half2 h = __floats2half2_rn(__fmul_rn(__fmul_rn(f.x, s1), s2),
+                                            __fmul_rn(__fmul_rn(f.y, s1), s2));
+        w[k] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+    }
+    sts128(a, make_uint4(w[0], w[1], w[2], w[3]));
+  }
+  // these generic-proxy writes come before any later tensor copy into the buffer
+  fence_proxy_async_smem();
+  return e;
+}
+
+// FWHT stages h = 2, 4, ..., 32 in registers and h = 64, 128 across the lanes of the row
+// (stage h = 1 is done by load_signed), then the row's sum of squares of the transformed
+// coordinates: even and odd coordinates accumulated separately by fused multiply-add in
+// register order, added, then the lanes of a row add their sums pairwise (xor butterfly
+// over the part bits), so every lane of the row holds the same value.
 template <int D>
-__device__ __forceinline__ float rotate_row(uint64_t (&xp)[32], int part, float* norm_out) {
+__device__ __forceinline__ float fwht_ss(uint64_t (&xp)[32], int part) {
   using G = AppendGeom<D>;
 #pragma unroll
   for (int h = 1; h < 32; h <<= 1) {           // element stride 2h
@@ -304,9 +377,42 @@ __device__ __forceinline__ float rotate_row(uint64_t (&xp)[32], int part, float*
 #pragma unroll
   for (int m = 1; m < G::TPR; m <<= 1)
     ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, G::ROWS * m));
-  // ||H s x||^2 = D ||x||^2
+  return ss;
+}
+
+// The rotation shared by quantize-append and its test export.  Loads this lane's 64
+// input elements of the row from the staged tile (`row`, `m`: see load_signed) and
+// leaves in xp the unnormalised transform H (s * x') of those coordinates, where x' is
+// the row scaled by 2^-e; returns r with u = xp * r.  *norm_out = ||x||_2 in fp32,
+// *bad_out = the row holds an infinity or NaN.
+// The scale keeps fp32 in range whatever the row's magnitude: e = 0 unless the sum of
+// squares ss of the unscaled transform (= D ||x||^2) falls outside [2^-60, 2^100] (so
+// the squares would overflow, or lose precision as subnormals) or is not a number.
+// Then the warp's rows out of range are rescaled in place in the staged tile by
+// 2^-e, e = floor(log2 max|x|) (largest magnitude in [1, 2)), and every row of the warp
+// is transformed again; multiplying by a power of two is exact, so a row in range
+// comes out bit for bit the same.  Order of operations (fixed, so that the export
+// reproduces the kernel exactly): the FWHT and ss of fwht_ss; n' = sqrt(ss / D)
+// (IEEE); r = 1 / (n' sqrt(D)) (IEEE reciprocal), or 0 when n' == 0; norm = n' 2^e.
+template <int D, typename Tin>
+__device__ __forceinline__ float rotate_row(uint64_t (&xp)[32], uint32_t row, const uint32_t* m,
+                                            int part, float* norm_out, bool* bad_out) {
+  int e = 0;
+  bool bad = false;
+  float ss;
+#pragma unroll 1
+  for (int pass = 0;; ++pass) {
+    load_signed<Tin>(xp, row, m);
+    ss = fwht_ss<D>(xp, part);
+    const bool in_range = ss >= 0x1p-60f && ss <= 0x1p100f;
+    if (pass > 0 || !__any_sync(0xffffffffu, !in_range)) break;
+    e = rescale_staged_row<D, Tin>(row, !in_range, &bad);
+    __syncwarp();
+  }
+  // ||H s x'||^2 = D ||x'||^2
   const float n = sqrtf(__fmul_rn(ss, 1.0f / D));
-  *norm_out = n;
+  *norm_out = e == 0 ? n : __fmul_rn(__fmul_rn(n, pow2f(e / 2)), pow2f(e - e / 2));
+  *bad_out = bad;
   const float sqrt_d = D == 64 ? 8.0f : (D == 128 ? 11.313708498984761f : 16.0f);
   return n > 0.f ? __frcp_rn(__fmul_rn(n, sqrt_d)) : 0.f;
 }
@@ -535,10 +641,10 @@ append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
       const int bits = p.bits[kind];
       const int rwords = kind ? vwords : kwords;          // packed words + norm word
       uint64_t xp[32];
-      load_signed<Tin>(xp, row0 + (uint32_t)(kind * SM::KIND), smask + part * 64);
       float n;
-      const float r = rotate_row<D>(xp, part, &n);
-      const bool bad = !(fabsf(n) <= 3.402823466e38f);   // inf or NaN
+      bool bad;
+      const float r = rotate_row<D, Tin>(xp, row0 + (uint32_t)(kind * SM::KIND), smask + part * 64,
+                                         part, &n, &bad);
       if (kind == 0 && p.bulk_out) {    // the previous tile's slots have been read out
         bulk_wait_read_all();
         __syncwarp();
@@ -633,9 +739,9 @@ rotate_unit_kernel(RotateParams p) {
     cp_async_wait<0>();
     __syncwarp();
     uint64_t xp[32];
-    load_signed<Tin>(xp, row, smask + part * 64);
     float n;
-    const float r = rotate_row<D>(xp, part, &n);
+    bool bad;
+    const float r = rotate_row<D, Tin>(xp, row, smask + part * 64, part, &n, &bad);
     if (rl < nr) {
       float* u = p.u + (r0 + rl) * p.u_row_stride + part * 64;
       const uint64_t r2 = f2(r, r);
@@ -645,7 +751,7 @@ rotate_unit_kernel(RotateParams p) {
         u[2 * i] = f2lo(u2);
         u[2 * i + 1] = f2hi(u2);
       }
-      if (part == 0) p.norm[(r0 + rl) * p.norm_stride] = n;
+      if (part == 0) p.norm[(r0 + rl) * p.norm_stride] = bad ? __uint_as_float(0x7FC00000u) : n;
     }
     __syncwarp();
   }

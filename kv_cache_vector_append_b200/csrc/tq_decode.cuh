@@ -110,6 +110,8 @@ struct DecodeParams {
   unsigned int* counters;       // [2][B]: records written, merges done (per sequence);
                                 // zero between calls (the last user of a counter clears it)
   unsigned int* err;
+  uint32_t wait_ms;             // limit of every bounded wait (milliseconds)
+  int32_t withhold_cta;         // test hook: this CTA never announces its records (-1: none)
 };
 
 // Step range of CTA c out of C over S steps: [floor(c S / C), floor((c+1) S / C)).
@@ -394,6 +396,7 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   int32_t* ids = (int32_t*)(prefix + p.batch + 1);     // block ids of the range
   int* wsum = (int*)(ids + p.ids_cap);                 // [32] per-warp sums of the scan
   int* timed_out = wsum + 32;                          // a stage wait of this CTA gave up
+  int* merge_gave_up = timed_out + 1;                  // the current merge wait gave up
   float* scratch = (float*)(timed_out + 4);            // [warps][D + 2] merge partials
   int* rpos = (int*)(scratch + blockDim.x / 32 * (D + 2));  // [D] coordinate at a record position
 
@@ -733,32 +736,59 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     }
   };
 
+  // This CTA is done with sequence b (merged its share, or gave up): the last of the n
+  // covering CTAs to get here clears both of b's counters (ready for the next call).
+  // Every covering CTA has passed its wait by then, so none still reads them.
+  auto release_counters = [&](int b, int n) {
+    if (tid == 0 && atomicAdd(&merged[b], 1u) == (unsigned)n - 1) {
+      atomicExch(&arrived[b], 0u);
+      atomicExch(&merged[b], 0u);
+    }
+  };
+  // Covering CTAs of sequence b that have records (n) and this CTA's rank among them.
+  auto cover = [&](int b, int& n, int& rank) {
+    const int64_t c_lo = cta_of(prefix[b], S, Cn), c_hi = cta_of(prefix[b + 1] - 1, S, Cn);
+    n = 0;
+    rank = 0;
+    for (int64_t c = c_lo; c <= c_hi; ++c)
+      if (nonempty(c)) {
+        if (c < (int64_t)blockIdx.x) ++rank;
+        ++n;
+      }
+  };
+
   // End phase for sequence b: once every CTA covering b has written its records, this
   // CTA (rank k of the n covering CTAs) merges query heads k, k + n, ...: groups of g
   // warps take one head each, split its records, and the group's first warp combines
   // the g partials, divides by l and applies o = R^T O' (FWHT, 1/sqrt(D), sign flips).
   auto coop_merge = [&](int b) {
     const int64_t c_lo = cta_of(prefix[b], S, Cn), c_hi = cta_of(prefix[b + 1] - 1, S, Cn);
-    int n = 0, rank = 0;
-    for (int64_t c = c_lo; c <= c_hi; ++c)
-      if (nonempty(c)) {
-        if (c < (int64_t)blockIdx.x) ++rank;
-        ++n;
-      }
+    int n, rank;
+    cover(b, n, rank);
     const int R = (int)(c_hi - c_lo + 1) * wph;
     if (tid == 0) {
       // wait until all n covering CTAs have arrived (bounded)
       const uint64_t t0 = globaltimer_ns();
+      int gave_up = 0;
       while (*(volatile unsigned int*)&arrived[b] < (unsigned)n) {
-        if (globaltimer_ns() - t0 > (uint64_t)kWaitMs * 1000000ull) {
+        if (globaltimer_ns() - t0 > (uint64_t)p.wait_ms * 1000000ull) {
           report_error(p.err, TQ_DEVERR_TIMEOUT);
+          gave_up = 1;
           break;
         }
         __nanosleep(256);
       }
       __threadfence();
+      *merge_gave_up = gave_up;
     }
     __syncthreads();
+    if (*merge_gave_up) {
+      // some records never arrived: merge nothing, but still count this CTA as done with
+      // the sequence, so that the counters return to zero
+      release_counters(b, n);
+      __syncthreads();
+      return;
+    }
     const int nh = rank < p.h_q ? (p.h_q - rank + n - 1) / n : 0;   // heads of this CTA
     int g = 1;
     while (nh > 0 && 2 * g * min(nh, nwarps) <= nwarps) g *= 2;
@@ -809,11 +839,7 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
       }
       __syncthreads();
     }
-    // the last covering CTA to finish clears both counters (ready for a replay)
-    if (tid == 0 && atomicAdd(&merged[b], 1u) == (unsigned)n - 1) {
-      atomicExch(&arrived[b], 0u);
-      atomicExch(&merged[b], 0u);
-    }
+    release_counters(b, n);
   };
 
   // Outer loop: the segments (one per sequence) of this CTA's step range; inner loop:
@@ -832,7 +858,7 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     int rem = p.seq_lens[cur_b] - ((int)(s0 + r - prefix[cur_b]) * wph + sub) * kBlockSize;
     start(cur_b, cur_b == b_first);
     for (; r < seg_end; ++r, rem -= wph * kBlockSize) {
-      if (!dead && !mbar_wait(&full[x], phase, kWaitMs)) {
+      if (!dead && !mbar_wait(&full[x], phase, p.wait_ms)) {
         if (lane == 0) {
           report_error(p.err, TQ_DEVERR_TIMEOUT);
           *timed_out = 1;
@@ -1015,16 +1041,24 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   __syncthreads();
   if (tid == 0) {
     __threadfence();
-    for (int b = b_first; b <= cur_b; ++b)
-      if (prefix[b + 1] > prefix[b]) atomicAdd(&arrived[b], 1u);
+    if ((int)blockIdx.x != p.withhold_cta)
+      for (int b = b_first; b <= cur_b; ++b)
+        if (prefix[b + 1] > prefix[b]) atomicAdd(&arrived[b], 1u);
   }
   if (*timed_out) {
-    // copies may still be landing in the stages: give them time (bounded), skip the merge
+    // copies may still be landing in the stages: give them time (bounded), skip the
+    // merge, and count this CTA as done with its sequences (counters back to zero)
     if (tid == 0) {
       const uint64_t t0 = globaltimer_ns();
       while (globaltimer_ns() - t0 < 100000000ull) __nanosleep(1000);
     }
     __syncthreads();
+    for (int b = b_first; b <= cur_b; ++b)
+      if (prefix[b + 1] > prefix[b]) {
+        int n, rank;
+        cover(b, n, rank);
+        release_counters(b, n);
+      }
     return;
   }
   for (int b = b_first; b <= cur_b; ++b)

@@ -1,0 +1,6 @@
+// Decode kernels for head_dim 128 and 2-bit K codes (every V width).
+#include "tq_launch.cuh"
+
+namespace tq {
+TQ_DEFINE_DECODE(128, 2)
+}  // namespace tq

@@ -44,19 +44,10 @@ tq_status launch_append_any(int dim, int dtype, const AppendParams& p, const App
                             const DeviceInfo& di, cudaStream_t st);
 tq_status launch_rotate_any(int dim, int dtype, const RotateParams& p, const DeviceInfo& di,
                             cudaStream_t st);
-tq_status launch_decode_d64(int kb, int vb, const DecodeParams& p, const DecodePlan& plan,
-                            const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st);
-tq_status launch_decode_d128(int kb, int vb, const DecodeParams& p, const DecodePlan& plan,
-                             const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st);
-tq_status launch_decode_d256(int kb, int vb, const DecodeParams& p, const DecodePlan& plan,
-                             const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st);
-
-// (K bits, V bits) pairs with a compiled decode kernel.
+// Code widths with a compiled decode kernel: K and V independently in {2, 3, 4, 8}.
 inline bool decode_bits_supported(int kb, int vb) {
-  const int ok[][2] = {{2, 2}, {3, 3}, {4, 4}, {8, 8}, {4, 2}, {3, 2}, {8, 4}, {4, 3}};
-  for (auto& c : ok)
-    if (c[0] == kb && c[1] == vb) return true;
-  return false;
+  auto ok = [](int b) { return b == 2 || b == 3 || b == 4 || b == 8; };
+  return ok(kb) && ok(vb);
 }
 
 template <int D, int KB, int VB, int NH, int MAXW>
@@ -99,21 +90,44 @@ tq_status launch_decode_bits(const DecodeParams& p, const DecodePlan& plan,
   else return launch_decode_t<D, KB, VB, 1, 8>(p, plan, tmap, steps_upper, st);
 }
 
-template <int D>
-tq_status launch_decode_dim(int kb, int vb, const DecodeParams& p, const DecodePlan& plan,
-                            const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st) {
-#define TQ_BITS_CASE(KB_, VB_) \
-  if (kb == KB_ && vb == VB_)  \
-    return launch_decode_bits<D, KB_, VB_>(p, plan, tmap, steps_upper, st);
-  TQ_BITS_CASE(2, 2)
-  TQ_BITS_CASE(3, 3)
-  TQ_BITS_CASE(4, 4)
-  TQ_BITS_CASE(8, 8)
-  TQ_BITS_CASE(4, 2)
-  TQ_BITS_CASE(3, 2)
-  TQ_BITS_CASE(8, 4)
-  TQ_BITS_CASE(4, 3)
-#undef TQ_BITS_CASE
+// All V widths for one (head_dim, K width); instantiated in tq_decode_d<D>_k<KB>.cu so
+// that the kernels compile in parallel.
+template <int D, int KB>
+tq_status launch_decode_kbits(int vb, const DecodeParams& p, const DecodePlan& plan,
+                              const CUtensorMap& tmap, int64_t steps_upper, cudaStream_t st) {
+  switch (vb) {
+    case 2: return launch_decode_bits<D, KB, 2>(p, plan, tmap, steps_upper, st);
+    case 3: return launch_decode_bits<D, KB, 3>(p, plan, tmap, steps_upper, st);
+    case 4: return launch_decode_bits<D, KB, 4>(p, plan, tmap, steps_upper, st);
+    case 8: return launch_decode_bits<D, KB, 8>(p, plan, tmap, steps_upper, st);
+    default: return TQ_ERR_UNSUPPORTED;
+  }
+}
+
+#define TQ_FOR_EACH_DECODE(X) \
+  X(64, 2) X(64, 3) X(64, 4) X(64, 8) \
+  X(128, 2) X(128, 3) X(128, 4) X(128, 8) \
+  X(256, 2) X(256, 3) X(256, 4) X(256, 8)
+#define TQ_DECLARE_DECODE(D_, KB_)                                                          \
+  tq_status launch_decode_d##D_##_k##KB_(int vb, const DecodeParams& p, const DecodePlan& plan, \
+                                         const CUtensorMap& tmap, int64_t steps_upper,       \
+                                         cudaStream_t st);
+#define TQ_DEFINE_DECODE(D_, KB_)                                                           \
+  tq_status launch_decode_d##D_##_k##KB_(int vb, const DecodeParams& p, const DecodePlan& plan, \
+                                         const CUtensorMap& tmap, int64_t steps_upper,       \
+                                         cudaStream_t st) {                                  \
+    return launch_decode_kbits<D_, KB_>(vb, p, plan, tmap, steps_upper, st);                 \
+  }
+TQ_FOR_EACH_DECODE(TQ_DECLARE_DECODE)
+
+// Decode launch for any supported (head_dim, K width, V width).
+inline tq_status launch_decode_any(int dim, int kb, int vb, const DecodeParams& p,
+                                   const DecodePlan& plan, const CUtensorMap& tmap,
+                                   int64_t steps_upper, cudaStream_t st) {
+#define TQ_DECODE_CASE(D_, KB_) \
+  if (dim == D_ && kb == KB_) return launch_decode_d##D_##_k##KB_(vb, p, plan, tmap, steps_upper, st);
+  TQ_FOR_EACH_DECODE(TQ_DECODE_CASE)
+#undef TQ_DECODE_CASE
   return TQ_ERR_UNSUPPORTED;
 }
 

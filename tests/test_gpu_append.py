@@ -249,3 +249,45 @@ def test_zero_nonfinite_and_out_of_range_rows():
     i, n = O.decode_region(_regions(p, wl, np.array([6]), 0)[0, 1], 128, 4)
     assert np.isfinite(n) and n > 0
     assert tq.get_device_error() == 0   # read clears
+
+
+def _scale_tokens(wl, scales):
+    """Multiply token t's K and V rows by scales[t % len(scales)] (in fp32, then stored
+    in the workload's dtype), so that every warp tile mixes row magnitudes."""
+    f = torch.tensor([scales[t % len(scales)] for t in range(wl.k.shape[0])],
+                     dtype=torch.float64)[:, None, None]
+    wl.k = (wl.k.double() * f).to(wl.k.dtype)
+    wl.v = (wl.v.double() * f).to(wl.v.dtype)
+    return wl
+
+
+# The method is scale-free (u = y / n), so rows far from unit scale must encode like
+# unit-scale rows and keep their norm to 1e-6 relative: squares of 1e30 overflow fp32
+# and squares of 1e-20 are subnormal, so the kernel rescales such rows exactly.
+@pytest.mark.parametrize("dtype,scales", [
+    ("float32", [1.0, 1e-30, 1e30, 1e-20, 1e18, 1.0, 1e-37, 3e36]),
+    ("bfloat16", [1.0, 1e-35, 1e35, 1e-20, 1e18]),
+])
+def test_extreme_row_magnitudes(dtype, scales):
+    tq = _tq()
+    for d in (64, 128, 256):
+        wl = _scale_tokens(W.generate(_mini(d, 4, 3, dtype=dtype, h_kv=8, batch=2, seq=40,
+                                             seed=d)), scales)
+        _bit_exact_case(tq, wl)
+        _end_to_end(tq, wl)
+
+
+def test_norm_beyond_fp32_range_stores_inf():
+    # bf16 rows of 2e38 everywhere: ||x|| = 2e38 sqrt(D) exceeds fp32; the codes are
+    # still those of the unit row and the stored norm is +inf (the oracle's fp32 norm).
+    tq = _tq()
+    wl = W.generate(_mini(128, 4, 4, dtype="bfloat16", h_kv=2, batch=1, seq=8, seed=3))
+    wl.k[2] = 2e38
+    wl.v[5, 1] = -2e38
+    tq.get_device_error()
+    _end_to_end(tq, wl)
+    pages, _ = gpu_append(tq, wl)
+    p = pages.cpu().numpy()
+    _, n = O.decode_region(_regions(p, wl, np.array([2]), 0)[0], 128, 4)
+    assert np.all(np.isposinf(n))
+    assert tq.get_device_error() == 0    # a finite row is not an error

@@ -103,13 +103,83 @@ def test_block_table_out_of_range_flagged():
 @pytest.mark.parametrize("cfg", [1, 2, 3, 4])
 def test_full_size_configs_sampled(cfg):
     # Full-size append and decode in the bench's launch configuration; the oracle
-    # recomputes a seeded sample of sequences.
+    # recomputes a seeded sample of 8 sequences that always holds the shortest and the
+    # longest one (all of them when the batch is smaller).
     tq = _tq()
     wl = W.generate(W.CONFIGS[cfg])
     pages, cb = gpu_append(tq, wl)
     out = gpu_decode(tq, wl, pages, cb)
     rng = np.random.default_rng(cfg)
-    seqs = np.sort(rng.choice(wl.spec.batch, size=min(2, wl.spec.batch), replace=False))
+    bsz = wl.spec.batch
+    pick = {int(np.argmin(wl.seq_lens)), int(np.argmax(wl.seq_lens))}
+    rest = [b for b in rng.permutation(bsz) if b not in pick]
+    seqs = np.sort(np.array(sorted(pick) + rest[:max(0, min(8, bsz) - len(pick))]))
     ref = _oracle_decode(wl, pages.cpu().numpy(), seqs)
     err = decode_error(to_np_f64(out)[seqs], ref)
     assert err <= TOL, err
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("kb", [2, 3, 4, 8])
+@pytest.mark.parametrize("vb", [2, 3, 4, 8])
+def test_every_required_bit_pair(d, kb, vb):
+    tq = _tq()
+    lens = [200, 17, 33]
+    _case(tq, _with_lens(_spec(d, 8, 2, kb, vb, lens, seed=kb * 10 + vb), lens))
+
+
+@pytest.mark.parametrize("pad,h_kv", [(24, 2), (8, 1), (56, 4)])
+def test_padded_slot_stride(pad, h_kv):
+    # slot_stride > slot_bytes: the padding rides along in the staged blocks (a 2-D
+    # tensor box when a row of all heads is a multiple of 16 bytes, else a 1-D copy).
+    tq = _tq()
+    lens = [150, 16, 47]
+    wl = _with_lens(_spec(128, 4 * h_kv, h_kv, 4, 2, lens, seed=pad), lens)
+    pages, cb = gpu_append(tq, wl, slot_stride=wl.slot_bytes + pad, fill=0x77)
+    out = gpu_decode(tq, wl, pages, cb)
+    ref = _oracle_decode(wl, pages.cpu().numpy())
+    assert decode_error(to_np_f64(out), ref) <= TOL
+
+
+@pytest.mark.parametrize("q_dtype,out_dtype", [("float16", "float16"), ("float16", "float32"),
+                                               ("float32", "float32"), ("bfloat16", "float32")])
+def test_query_and_output_dtypes(q_dtype, out_dtype):
+    tq = _tq()
+    lens = [120, 40]
+    wl = _with_lens(_spec(128, 16, 4, 4, 4, lens, seed=4), lens)
+    wl.q = wl.q.float().to(getattr(torch, q_dtype))
+    _case(tq, wl, out_dtype=getattr(torch, out_dtype))
+
+
+def test_strided_query_and_output():
+    # q and out as views with head and batch strides wider than the dense layout.
+    tq = _tq()
+    lens = [90, 200, 5]
+    wl = _with_lens(_spec(64, 12, 3, 4, 3, lens, seed=8), lens)
+    pages, cb = gpu_append(tq, wl)
+    b, h, d = wl.q.shape
+    qbig = torch.zeros(b, h, 2 * d, dtype=wl.q.dtype, device="cuda")
+    qbig[..., d:] = wl.q.cuda()
+    q = qbig[..., d:]
+    obig = torch.full((b, 2 * h, d), float("nan"), dtype=torch.float32, device="cuda")
+    out = obig[:, 1::2]
+    assert q.stride(1) == 2 * d and out.stride(1) == 2 * d
+    tq.paged_decode(out, q, pages, torch.from_numpy(wl.block_table).cuda(),
+                    torch.from_numpy(wl.seq_lens).cuda(), cb, wl.spec.sign_seed, wl.spec.scale)
+    torch.cuda.synchronize()
+    assert torch.all(torch.isnan(obig[:, 0::2]))          # the other rows untouched
+    ref = _oracle_decode(wl, pages.cpu().numpy())
+    assert decode_error(to_np_f64(out), ref) <= TOL
+
+
+@pytest.mark.parametrize("k_scale,v_scale", [(1.0, 1e18), (1.0, 1e-20), (1e-20, 1.0),
+                                             (1e-12, 1e15)])
+def test_extreme_key_and_value_magnitudes(k_scale, v_scale):
+    # The decode reads norms from the slots: values of 1e18 or 1e-20 keep their weight
+    # through the lazy softmax reference, keys of 1e-20 give uniform attention.
+    tq = _tq()
+    lens = [300, 64]
+    wl = _with_lens(_spec(128, 8, 2, 4, 4, lens, dtype="float32", seed=12), lens)
+    wl.k = wl.k * k_scale
+    wl.v = wl.v * v_scale
+    _case(tq, wl)
