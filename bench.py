@@ -49,6 +49,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (smaller cases for profiling)")
+    ap.add_argument("--no-extra-configs", action="store_true",
+                    help="skip the configs[3] and configs[4] legs of the default run")
     return ap.parse_args(argv)
 
 
@@ -192,60 +194,129 @@ class ClockSampler:
 # CPU oracle (baseline and reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample_step(wl, tables, n_append=1024, n_decode_tokens=2048, seq=0):
-    """One bounded oracle step on the workload: quantize-append of n_append tokens
-    of sequence `seq` into a page pool, then a decode step of that sequence over
-    its first n_decode_tokens tokens.  Returns (seconds, algorithmic bytes, text)."""
-    from oracle import tq_oracle as O
+def oracle_sample_inputs(wl, seq, n_tokens=2048):
+    """Inputs of one bounded oracle sample of the workload: the first n_tokens tokens of
+    sequence `seq` (K, V, q as float arrays), appended into a compact page pool of their
+    own (block b of the sequence in pool block b) and then decoded.  Plain arrays, so
+    that they can go to a worker process."""
     spec = wl.spec
-    kt, vt = tables
     seq = int(seq) % max(1, spec.batch)
     start = int(wl.seq_lens[:seq].astype(np.int64).sum())
-    n_dec = int(min(n_decode_tokens, wl.seq_lens[seq]))
-    n_app = int(min(n_append, n_dec))
-    pages = np.zeros((wl.num_blocks, 16, spec.num_kv_heads, wl.slot_bytes), dtype=np.uint8)
-    slots = wl.slot_mapping[start:start + n_dec]
-    k = wl.k[start:start + n_dec].float().numpy()
-    v = wl.v[start:start + n_dec].float().numpy()
-    # the untimed part fills the decode range; the timed part re-appends n_app tokens
-    pages = O.quantize_append(pages, slots, k, v, kt, vt, spec.sign_seed)
+    n_dec = int(min(n_tokens, wl.seq_lens[seq]))
+    n_app = n_dec
+    return {"k": wl.k[start:start + n_dec].float().numpy(),
+            "v": wl.v[start:start + n_dec].float().numpy(),
+            "q": wl.q[seq:seq + 1].float().numpy().astype(np.float64),
+            "n_app": n_app, "n_dec": n_dec, "h_kv": spec.num_kv_heads,
+            "slot_bytes": wl.slot_bytes, "head_dim": spec.head_dim, "k_bits": spec.k_bits,
+            "v_bits": spec.v_bits, "sign_seed": spec.sign_seed, "scale": spec.scale,
+            "bytes": append_bytes(spec, n_app) + decode_bytes(spec, [n_dec])[0]}
+
+
+def oracle_sample_run(inp):
+    """Run one sample through the oracle as it stands, all of it timed: quantize-append
+    of the sample's tokens into an empty pool, then one decode step over them.
+    Returns (wall seconds, CPU seconds, algorithmic bytes)."""
+    from oracle import gen_codebooks as G
+    from oracle import tq_oracle as O
+    d = inp["head_dim"]
+    kt = G.read_table(os.path.join(G.DEFAULT_OUT, G.table_filename(d, inp["k_bits"])))
+    vt = G.read_table(os.path.join(G.DEFAULT_OUT, G.table_filename(d, inp["v_bits"])))
+    n_dec, n_app = inp["n_dec"], inp["n_app"]
+    nblk = (n_dec + 15) // 16
+    slots = np.arange(n_dec, dtype=np.int64)
     t0 = time.perf_counter()
     c0 = time.process_time()
-    pages = O.quantize_append(pages, slots[:n_app], k[:n_app], v[:n_app], kt, vt,
-                              spec.sign_seed)
-    q = wl.q[seq:seq + 1].float().numpy().astype(np.float64)
-    O.paged_decode(q, pages, wl.block_table[seq:seq + 1], np.array([n_dec], dtype=np.int32),
-                   kt, vt, spec.sign_seed, spec.scale)
-    dt = time.perf_counter() - t0
-    oracle_sample_step.cpu_seconds = time.process_time() - c0
-    nbytes = append_bytes(spec, n_app) + decode_bytes(spec, [n_dec])[0]
-    desc = (f"{n_app} tokens x {spec.num_kv_heads} KV heads appended + 1 sequence x {n_dec} "
-            f"tokens x {spec.num_q_heads} q heads decoded")
-    return dt, nbytes, desc
+    pages = np.zeros((nblk, 16, inp["h_kv"], inp["slot_bytes"]), dtype=np.uint8)
+    pages = O.quantize_append(pages, slots[:n_app], inp["k"][:n_app], inp["v"][:n_app], kt, vt,
+                              inp["sign_seed"])
+    O.paged_decode(inp["q"], pages, np.arange(nblk)[None], np.array([n_dec], dtype=np.int32),
+                   kt, vt, inp["sign_seed"], inp["scale"])
+    return time.perf_counter() - t0, time.process_time() - c0, inp["bytes"]
 
 
-def cpu_baseline(wl, tables, min_seconds=10.0, max_samples=64):
-    """The oracle timed on host cores over repeated bounded samples (one per
-    sequence, cycling) until at least min_seconds of oracle work has run."""
-    oracle_sample_step(wl, tables, 256, 512)   # warm caches
-    total_t = total_b = total_cpu = 0.0
+def _pool_worker(inp):
+    """One sample in a worker process, on one BLAS thread."""
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(1):
+            return oracle_sample_run(inp)
+    except ImportError:
+        return oracle_sample_run(inp)
+
+
+def sample_desc(wl, inp):
+    s = wl.spec
+    return (f"{inp['n_app']} tokens x {s.num_kv_heads} KV heads appended + 1 sequence x "
+            f"{inp['n_dec']} tokens x {s.num_q_heads} q heads decoded")
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+class OraclePool:
+    """The oracle on all host cores: one spawned worker process per core (spawn, so it
+    is safe after CUDA has been initialised), each on one BLAS thread, each running
+    whole samples."""
+
+    def __init__(self, cores=None):
+        import multiprocessing as mp
+        self.cores = cores or host_cores()
+        self.pool = mp.get_context("spawn").Pool(self.cores)
+
+    def run(self, inputs):
+        """Wall seconds, summed CPU seconds and bytes of running all inputs at once."""
+        t0 = time.perf_counter()
+        res = self.pool.map(_pool_worker, inputs, chunksize=1)
+        wall = time.perf_counter() - t0
+        return wall, sum(r[1] for r in res), sum(r[2] for r in res)
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+def cpu_baseline(wl, min_seconds=10.0, max_samples=64):
+    """The oracle timed on the host: on one core (samples one after another, one BLAS
+    thread, until min_seconds) and on all cores (a spawned worker per core, a batch of
+    samples per core, after a warm-up batch)."""
+    try:
+        from threadpoolctl import threadpool_limits
+        limit = threadpool_limits(1)
+    except ImportError:
+        limit = None
+    oracle_sample_run(oracle_sample_inputs(wl, 0, 256))     # warm caches
+    total_t = total_b = 0.0
     n = 0
     desc = ""
     while n < max_samples and (total_t < min_seconds or n == 0):
-        dt, nb, desc = oracle_sample_step(wl, tables, seq=n)
+        inp = oracle_sample_inputs(wl, n)
+        dt, _, nb = oracle_sample_run(inp)
+        desc = sample_desc(wl, inp)
         total_t += dt
         total_b += nb
-        total_cpu += oracle_sample_step.cpu_seconds
         n += 1
-    return {"value": total_b / total_t / 1e9, "unit": "GB/s",
-            "cores": effective_cores(total_cpu, total_t), "threads_available": blas_threads(),
-            "kind": "oracle", "sample": f"{n} samples (sequences 0..{n - 1}, cycling) of: {desc}",
-            "seconds": total_t}
-
-
-def effective_cores(cpu_seconds, wall_seconds):
-    """Host cores the oracle kept busy on average: process CPU time over wall time."""
-    return round(max(1.0, cpu_seconds / wall_seconds), 1) if wall_seconds > 0 else 1.0
+    if limit is not None:
+        limit.unregister()
+    single = {"value": total_b / total_t / 1e9, "cores": 1, "seconds": total_t,
+              "sample": f"{n} samples (sequences 0..{n - 1}, cycling) of: {desc}"}
+    pool = OraclePool()
+    try:
+        cores = pool.cores
+        pool.run([oracle_sample_inputs(wl, i, 256) for i in range(cores)])   # warm-up
+        per_core = max(1, int(round(min_seconds / max(total_t / n, 1e-3) / 2)))
+        inputs = [oracle_sample_inputs(wl, i) for i in range(cores * per_core)]
+        wall, cpu, nbytes = pool.run(inputs)
+    finally:
+        pool.close()
+    return {"value": nbytes / wall / 1e9, "unit": "GB/s", "cores": cores,
+            "cpu_seconds_per_wall_second": round(cpu / wall, 1), "kind": "oracle",
+            "sample": f"{len(inputs)} samples ({per_core} per core, sequences cycling) of: "
+                      f"{desc}", "seconds": wall, "single_core": single}
 
 
 def oracle_tables(spec):
@@ -255,47 +326,60 @@ def oracle_tables(spec):
     return kt, vt
 
 
-def blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info()]
-        return max(n) if n else 1
-    except Exception:
-        return 1
+def config_dict(spec, world, n_step_tokens, step_bytes):
+    """The `config` object of the JSON line (the same in both arms)."""
+    return {"workload": spec.name, "batch": spec.batch,
+            "seq_len": spec.seq_len or list(spec.seq_len_range),
+            "head_dim": spec.head_dim, "q_heads": spec.num_q_heads,
+            "kv_heads": spec.num_kv_heads, "k_bits": spec.k_bits, "v_bits": spec.v_bits,
+            "input_dtype": spec.dtype, "step_tokens_appended": int(n_step_tokens),
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": f"inputs larger than L2 ({step_bytes / 1e6:.0f} MB touched per step)"}
+
+
+def step_shape(wl):
+    """Tokens appended and algorithmic bytes of one full step of the workload."""
+    n_step = len(wl.step_tokens)
+    return n_step, append_bytes(wl.spec, n_step) + decode_bytes(wl.spec, wl.seq_lens)[0]
 
 
 def run_reference(args):
+    """The CPU oracle as it stands, on all host cores: each step is one batch of bounded
+    samples of the workload, one per core, run at once."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     from kv_cache_vector_append_b200 import workloads as W
     spec = W.CONFIGS[args.config]
     wl = W.generate(spec)
-    tables = oracle_tables(spec)
-    for i in range(args.warmup):
-        oracle_sample_step(wl, tables, seq=i)
-    total_t = total_b = total_cpu = 0.0
-    desc = ""
-    for i in range(args.steps):
-        dt, nb, desc = oracle_sample_step(wl, tables, seq=args.warmup + i)
-        total_t += dt
-        total_b += nb
-        total_cpu += oracle_sample_step.cpu_seconds
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    n_step, step_bytes = step_shape(wl)
+    pool = OraclePool()
+    try:
+        cores = pool.cores
+        for i in range(args.warmup):
+            pool.run([oracle_sample_inputs(wl, i * cores + j, 256) for j in range(cores)])
+        total_t = total_b = total_cpu = 0.0
+        inp = None
+        for i in range(args.steps):
+            inputs = [oracle_sample_inputs(wl, i * cores + j) for j in range(cores)]
+            inp = inputs[0]
+            wall, cpu, nb = pool.run(inputs)
+            total_t += wall
+            total_cpu += cpu
+            total_b += nb
+    finally:
+        pool.close()
     value = total_b / total_t / 1e9
-    cores = effective_cores(total_cpu, total_t)
+    desc = f"{cores} samples per step (one per core) of: {sample_desc(wl, inp)}"
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "impl": "reference",
-            "config": {"workload": spec.name, "batch": spec.batch, "seq_len":
-                       spec.seq_len or list(spec.seq_len_range), "head_dim": spec.head_dim,
-                       "q_heads": spec.num_q_heads, "kv_heads": spec.num_kv_heads,
-                       "k_bits": spec.k_bits, "v_bits": spec.v_bits,
-                       "parallelism": "replicas" if args.gpus > 1 else "single"},
+            "impl": "reference", "config": config_dict(spec, world, n_step, step_bytes),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores,
-                             "threads_available": blas_threads(), "kind": "oracle",
-                             "sample": desc + " per step"},
+                             "cpu_seconds_per_wall_second": round(total_cpu / total_t, 1),
+                             "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -306,6 +390,107 @@ def run_reference(args):
 # GPU arm
 # ---------------------------------------------------------------------------
 
+def device_inputs(wl, dev):
+    """The workload's step inputs, page pool (with the untimed setup tokens already
+    appended) and decode inputs on the device."""
+    import torch
+    import kv_cache_vector_append_b200 as tq
+    from kv_cache_vector_append_b200 import workloads as W
+    spec = wl.spec
+    step_idx = torch.from_numpy(wl.step_tokens)
+    setup_idx = torch.from_numpy(wl.setup_tokens)
+    cb = tq.load_codebooks(spec.head_dim, spec.k_bits, spec.v_bits, dev)
+    pages = W.empty_pages(wl, device=dev)
+    for s in range(0, len(wl.setup_tokens), 1 << 18):
+        ii = setup_idx[s:s + (1 << 18)]
+        tq.quantize_append(pages, torch.from_numpy(wl.slot_mapping[ii.numpy()]).to(dev),
+                           wl.k[ii].to(dev), wl.v[ii].to(dev), cb, spec.sign_seed)
+    return {"cb": cb, "pages": pages, "k": wl.k[step_idx].to(dev), "v": wl.v[step_idx].to(dev),
+            "sm": torch.from_numpy(wl.slot_mapping[wl.step_tokens]).to(dev),
+            "q": wl.q.to(dev), "out": torch.empty(wl.q.shape, dtype=wl.q.dtype, device=dev),
+            "bt": torch.from_numpy(wl.block_table).to(dev),
+            "sl": torch.from_numpy(wl.seq_lens).to(dev)}
+
+
+def time_legs(spec, x, steps, stream, flush=None):
+    """Mean ms of the append and of the decode over `steps` timed steps (CUDA events on
+    the launching stream).  With `flush` (a device buffer larger than L2) the buffer is
+    rewritten before every decode, outside its events."""
+    import torch
+    import kv_cache_vector_append_b200 as tq
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(steps):
+        ev[i][0].record(stream)
+        tq.quantize_append(x["pages"], x["sm"], x["k"], x["v"], x["cb"], spec.sign_seed, stream)
+        ev[i][1].record(stream)
+        if flush is not None:
+            flush.add_(1)
+        ev[i][2].record(stream)
+        tq.paged_decode(x["out"], x["q"], x["pages"], x["bt"], x["sl"], x["cb"], spec.sign_seed,
+                        spec.scale, stream)
+        ev[i][3].record(stream)
+    torch.cuda.synchronize()
+    return (float(np.mean([e[0].elapsed_time(e[1]) for e in ev])),
+            float(np.mean([e[2].elapsed_time(e[3]) for e in ev])))
+
+
+def leg_summary(wl, app_ms, dec_ms, peak):
+    spec = wl.spec
+    n_step = len(wl.step_tokens)
+    a_bytes = append_bytes(spec, n_step)
+    d_bytes, d_packed = decode_bytes(spec, wl.seq_lens)
+    rows = 2 * n_step * spec.num_kv_heads
+    return {"append": {"ms": app_ms, "mrows_per_s": rows / (app_ms * 1e-3) / 1e6,
+                       "gbs": a_bytes / (app_ms * 1e-3) / 1e9,
+                       "frac_of_peak": a_bytes / (app_ms * 1e-3) / 1e9 / peak, "rows": rows,
+                       "bytes": a_bytes},
+            "decode": {"ms": dec_ms, "packed_kv_gbs": d_packed / (dec_ms * 1e-3) / 1e9,
+                       "gbs": d_bytes / (dec_ms * 1e-3) / 1e9,
+                       "frac_of_peak": d_bytes / (dec_ms * 1e-3) / 1e9 / peak,
+                       "tokens_per_s": spec.batch / (dec_ms * 1e-3),
+                       "kv_tokens_scanned_per_s": float(np.sum(wl.seq_lens)) / (dec_ms * 1e-3),
+                       "bytes": d_bytes, "packed_bytes": d_packed}}
+
+
+def extra_config_legs(configs, dev, steps, warmup, peak):
+    """Append and decode of other workloads on this GPU (timed like the main step,
+    each in its own timed region): configs 3 and 4 by default.  configs[4]'s page pool
+    (92 MB) fits in L2, so its decode is also timed with L2 rewritten before each
+    launch."""
+    import torch
+    import kv_cache_vector_append_b200 as tq
+    from kv_cache_vector_append_b200 import workloads as W
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    for c in configs:
+        wl = W.generate(W.CONFIGS[c])
+        spec = wl.spec
+        x = device_inputs(wl, dev)
+        ws = tq.decode_workspace_size(spec.batch, spec.num_q_heads, spec.num_kv_heads,
+                                      spec.head_dim, wl.block_table.shape[1])
+        ws_t = torch.empty(ws, dtype=torch.uint8, device=dev)
+        tq.set_workspace(ws_t)
+        time_legs(spec, x, max(warmup, 3), stream)
+        app_ms, dec_ms = time_legs(spec, x, steps, stream)
+        leg = leg_summary(wl, app_ms, dec_ms, peak)
+        leg["step_tokens_appended"] = int(len(wl.step_tokens))
+        if c == 4:
+            flush = torch.zeros(4 * l2 // 4, dtype=torch.float32, device=dev)
+            time_legs(spec, x, max(warmup, 3), stream, flush)
+            _, dec_f = time_legs(spec, x, steps, stream, flush)
+            leg["decode_l2_flushed"] = leg_summary(wl, app_ms, dec_f, peak)["decode"]
+            leg["decode_l2_flushed"]["flush_bytes"] = int(flush.numel() * 4)
+            del flush
+        if tq.get_device_error(stream):
+            raise RuntimeError(f"device error during the {spec.name} leg")
+        tq.set_workspace(None)
+        res[spec.name] = leg
+        del x, ws_t
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -315,6 +500,8 @@ def run_gpu(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch one rank per GPU")
     if world > 1:
         torch.cuda.set_device(local)
         from datetime import timedelta
@@ -326,22 +513,9 @@ def run_gpu(args):
     if args.batch:
         spec = spec.scaled(batch=args.batch)
     wl = W.generate(spec)
-    step_idx = torch.from_numpy(wl.step_tokens)
-    setup_idx = torch.from_numpy(wl.setup_tokens)
-    cb = tq.load_codebooks(spec.head_dim, spec.k_bits, spec.v_bits, dev)
-    pages = W.empty_pages(wl, device=dev)
-    k_step = wl.k[step_idx].to(dev)
-    v_step = wl.v[step_idx].to(dev)
-    sm_step = torch.from_numpy(wl.slot_mapping[wl.step_tokens]).to(dev)
-    q = wl.q.to(dev)
-    out = torch.empty_like(q)
-    bt = torch.from_numpy(wl.block_table).to(dev)
-    sl = torch.from_numpy(wl.seq_lens).to(dev)
-    if len(wl.setup_tokens):
-        for s in range(0, len(wl.setup_tokens), 1 << 18):
-            ii = setup_idx[s:s + (1 << 18)]
-            tq.quantize_append(pages, torch.from_numpy(wl.slot_mapping[ii.numpy()]).to(dev),
-                               wl.k[ii].to(dev), wl.v[ii].to(dev), cb, spec.sign_seed)
+    x = device_inputs(wl, dev)
+    cb, pages, k_step, v_step, sm_step = x["cb"], x["pages"], x["k"], x["v"], x["sm"]
+    q, out, bt, sl = x["q"], x["out"], x["bt"], x["sl"]
     ws_bytes = tq.decode_workspace_size(spec.batch, spec.num_q_heads, spec.num_kv_heads,
                                         spec.head_dim, wl.block_table.shape[1])
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
@@ -349,11 +523,9 @@ def run_gpu(args):
     stream = torch.cuda.current_stream(dev)
     torch.cuda.synchronize(dev)
 
-    n_step = len(wl.step_tokens)
-    a_bytes = append_bytes(spec, n_step)
-    d_bytes, d_packed = decode_bytes(spec, wl.seq_lens)
-    step_bytes = a_bytes + d_bytes
-    rows = 2 * n_step * spec.num_kv_heads
+    n_step, step_bytes = step_shape(wl)
+    d_bytes, _ = decode_bytes(spec, wl.seq_lens)
+    step_bytes = append_bytes(spec, n_step) + d_bytes
 
     def step():
         tq.quantize_append(pages, sm_step, k_step, v_step, cb, spec.sign_seed, stream)
@@ -395,6 +567,7 @@ def run_gpu(args):
     # ---- end to end through the public API, host buffers ----
     e2e = None
     if not args.no_e2e:
+        step_idx = torch.from_numpy(wl.step_tokens)
         k_h = wl.k[step_idx].pin_memory()
         v_h = wl.v[step_idx].pin_memory()
         sm_h = torch.from_numpy(wl.slot_mapping[wl.step_tokens]).pin_memory()
@@ -432,56 +605,52 @@ def run_gpu(args):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms / args.steps}
 
+    peak, peak_kind = measured_peaks()
+    extra = None
+    if not args.no_extra_configs and args.config == 2 and not args.batch:
+        tq.set_workspace(None)
+        del x
+        extra = extra_config_legs((3, 4), dev, args.steps, args.warmup, peak)
+        tq.set_workspace(ws)
+
     if rank != 0:
         if world > 1:
             tq.set_workspace(None)
             dist.destroy_process_group()
         return 0
 
-    peak, peak_kind = measured_peaks()
     ms_per_step = total_ms / args.steps
     value = job_gbs(world, step_bytes, ms_per_step)
-    app_gbs = a_bytes / (app_ms * 1e-3) / 1e9
-    dec_gbs = d_bytes / (dec_ms * 1e-3) / 1e9
-    dec_packed_gbs = d_packed / (dec_ms * 1e-3) / 1e9
+    legs = leg_summary(wl, app_ms, dec_ms, peak)
     dominant = "append" if app_ms >= dec_ms else "decode"
     dom_kernel = "append_kernel" if dominant == "append" else "decode_kernel"
-    dom_gbs = app_gbs if dominant == "append" else dec_gbs
-    traffic = ncu_traffic(dom_kernel, spec.name)
+    dom_gbs = legs[dominant]["gbs"]
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "dtype_detail": "f32 rotate/norm/encode; decode contractions f16 x f16 -> f32",
+        "dtype": "f32+f16",
+        "dtype_detail": "append: f32 rotate/norm/encode; decode: f32 query rotation, softmax "
+                        "and merge, score and value contractions on f16 x f16 -> f32 mma",
         "data": "synthetic",
-        "config": {"workload": spec.name, "batch": spec.batch,
-                   "seq_len": spec.seq_len or list(spec.seq_len_range),
-                   "head_dim": spec.head_dim, "q_heads": spec.num_q_heads,
-                   "kv_heads": spec.num_kv_heads, "k_bits": spec.k_bits, "v_bits": spec.v_bits,
-                   "input_dtype": spec.dtype, "step_tokens_appended": n_step,
-                   "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": f"inputs larger than L2 ({step_bytes / 1e6:.0f} MB touched per step)"},
-        "append": {"ms": app_ms, "mrows_per_s": rows / (app_ms * 1e-3) / 1e6, "gbs": app_gbs,
-                   "frac_of_peak": app_gbs / peak, "rows": rows, "bytes": a_bytes},
-        "decode": {"ms": dec_ms, "packed_kv_gbs": dec_packed_gbs, "gbs": dec_gbs,
-                   "frac_of_peak": dec_gbs / peak,
-                   "tokens_per_s": spec.batch / (dec_ms * 1e-3),
-                   "kv_tokens_scanned_per_s": float(np.sum(wl.seq_lens)) / (dec_ms * 1e-3),
-                   "bytes": d_bytes, "packed_bytes": d_packed},
+        "config": config_dict(spec, world, n_step, step_bytes),
+        "append": legs["append"], "decode": legs["decode"],
         "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": dom_gbs, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": dom_gbs / peak,
-                     "traffic": traffic},
+                     "traffic": ncu_traffic(dom_kernel, spec.name)},
         "roofline_decode": {"bound": "hbm", "kernel": "decode_kernel",
-                            "achieved": dec_gbs, "peak": peak, "unit": "GB/s",
-                            "frac": dec_gbs / peak,
+                            "achieved": legs["decode"]["gbs"], "peak": peak, "unit": "GB/s",
+                            "frac": legs["decode"]["gbs"] / peak,
                             "traffic": ncu_traffic("decode_kernel", spec.name)},
         "gpu_launches": 2 * args.steps,   # append_kernel + decode_kernel
         "clocks": clk.summary(),
     }
+    if extra:
+        line["other_configs"] = extra
     if e2e is not None:
         line["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, oracle_tables(spec))
+        line["cpu_baseline"] = cpu_baseline(wl)
     print(json.dumps(line), flush=True)
     if world > 1:
         tq.set_workspace(None)
@@ -489,8 +658,23 @@ def run_gpu(args):
     return 0
 
 
+def launch_replicas(argv, n):
+    """`--gpus N` run directly (no launcher): start N ranks, one process per GPU on
+    this node, through torch.distributed.run, and return its exit code."""
+    import random
+    import subprocess
+    port = 20000 + random.randrange(20000)
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__)] + list(argv)
+    return subprocess.run(cmd, timeout=3600).returncode
+
+
 def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
     args = parse_args(argv)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return launch_replicas(argv, args.gpus)
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)

@@ -119,6 +119,18 @@ typedef struct {
   tq_codebook v;
 } tq_codebooks;
 
+/* The dense random rotation R (turboquant_serve 0.1.2, "Architecture" and "Rotation": a
+ * fixed random orthogonal matrix, seeded by head_dim; TorbuQuant, "Current Status": QR
+ * rotation) as two bf16 matrices: R = hi + lo, [dim][dim] row-major (row j gives output
+ * coordinate j), bf16 bit patterns in device memory, 16-byte aligned, owned by the caller.
+ * The library's data files rotations/qr_d<D>.tqrt hold them (hi = bf16 of the seeded
+ * Haar matrix, lo = bf16 of the remainder; R is exact in fp32 and orthogonal to ~1e-5). */
+typedef struct {
+  int32_t dim;
+  const uint16_t* hi;
+  const uint16_t* lo;
+} tq_rotation;
+
 /* Bytes of one slot before padding: (ceil(D*k_bits/8)+4) + (ceil(D*v_bits/8)+4)
  * (TorbuQuant, "TQ4 page tensor").  Host only; *out receives the value.
  * Errors: TQ_ERR_INVALID_ARG for dim < 1, bits outside 1..8 or out == NULL. */
@@ -140,6 +152,12 @@ TQ_API tq_status tq_slot_bytes(int32_t dim, int32_t k_bits, int32_t v_bits, int3
  *   sign_seed    SplitMix64 seed of the rotation signs.
  *   k_bits, v_bits  1..8.  D must be 64, 128 or 256.
  * Two tokens mapped to the same slot race (either row may win).
+ * Two launches: the fast path, then a redo that returns at once unless some row's sum
+ * of squares left the fast path's range (rows of magnitude beyond about 1e14 or below
+ * about 1e-10, zero rows, non-finite rows), in which case the whole call is done again
+ * with an exact power-of-two rescaling of those rows.  The two share a per-device flag:
+ * calls on one device whose kernels overlap on the GPU (unordered streams) must be
+ * ordered.
  * Fast paths (same results, chosen per call on the host):
  *   - k and v are staged by tensor copies when they are 16-bit, 16-byte aligned with
  *     token and head strides that are multiples of 8 elements, and H_kv divides
@@ -190,6 +208,31 @@ TQ_API tq_status tq_paged_decode(tq_tensor out, tq_tensor q, tq_tensor pages,
                           tq_tensor block_table, tq_tensor seq_lens,
                           const tq_codebooks* cb, uint64_t sign_seed, float scale,
                           void* stream);
+
+/* Paged decode with an uncompressed hot window (turboquant_pro 1.4.2, "Fused CUDA
+ * decode": the fp16 hot window is merged through the online softmax, and "Streaming
+ * cache"; tq-kv, "How It Works", "3-Fix for GGUF Models": sink tokens stay FP16, the
+ * current token is lossless).  Same as tq_paged_decode, except that sequence b also
+ * attends to hot tokens 0 .. hot_lens[b]-1 of hot_k / hot_v, inside the same softmax:
+ *   out[b, h] = sum_t softmax_t(scale * <q[b,h], key_t>) value_t over the seq_lens[b]
+ *               packed tokens (dequantized) and the hot tokens (read exactly).
+ *   hot_k, hot_v  [B, W, H_kv, D] in bf16, f16 or f32 (same dtype and strides); the
+ *                 last dim contiguous.  The caller keeps there whichever tokens stay
+ *                 uncompressed (the first few "sink" tokens, the most recent ones); their
+ *                 positions do not enter the result.  A token should be in the pages or
+ *                 in the window, not both.
+ *   hot_lens      i32 [B]; an entry outside [0, W] raises TQ_DEVERR_SEQLEN_RANGE and
+ *                 counts as 0.  A sequence with seq_lens[b] == 0 attends to its hot
+ *                 tokens alone; with no tokens at all it gives 0.
+ * The packed tokens are reduced as in tq_paged_decode; the CTA that finishes a query
+ * head computes the hot tokens' partial (fp32) and joins the two partials with one
+ * rescale before the division by the softmax sum.
+ * Errors: as tq_paged_decode, plus TQ_ERR_INVALID_ARG for mismatched hot tensors. */
+TQ_API tq_status tq_paged_decode_hot(tq_tensor out, tq_tensor q, tq_tensor pages,
+                                     tq_tensor block_table, tq_tensor seq_lens,
+                                     tq_tensor hot_k, tq_tensor hot_v, tq_tensor hot_lens,
+                                     const tq_codebooks* cb, uint64_t sign_seed, float scale,
+                                     void* stream);
 
 /* Allocation-free variant of tq_paged_decode (this library's own addition; the
  * pages describe no counterpart).  Same arguments, semantics and results as
@@ -246,6 +289,36 @@ TQ_API tq_status tq_get_device_error(int32_t* out, void* stream);
  * reproduces the kernel's codes bit for bit). */
 TQ_API tq_status tq_rotate_unit(tq_tensor u, tq_tensor norm, tq_tensor x, uint64_t sign_seed,
                          void* stream);
+
+/* Quantize-append with the dense rotation (turboquant_serve 0.1.2, "Architecture":
+ * rotate k, v = k @ R, then normalize, encode and pack; turboquant_pro 1.4.2, "Fused CUDA
+ * decode": rotation and quantization in one tiled GEMM).  Same slot layout, norm,
+ * encode and errors as tq_quantize_append, with y = R x in place of the randomized
+ * Hadamard transform: u = y / ||x||.  y is one tcgen05 GEMM per tile of 128 (token, head)
+ * rows (bf16 x bf16 -> fp32 in tensor memory, R as hi and lo).
+ *   rot   host pointer; rot->dim == D.
+ * Supported: D = 64 or 128; k, v bf16, 16-byte aligned with token and head strides that
+ * are multiples of 8 elements; H_kv a divisor or a multiple of 128 (TQ_ERR_UNSUPPORTED
+ * otherwise).  Rows whose sum of squares leaves [2^-60, 2^100] are rotated on the CUDA
+ * cores after an exact power-of-two rescaling. */
+TQ_API tq_status tq_quantize_append_dense(tq_tensor pages, tq_tensor slot_mapping, tq_tensor k,
+                                          tq_tensor v, const tq_codebooks* cb,
+                                          const tq_rotation* rot, int32_t k_bits, int32_t v_bits,
+                                          void* stream);
+
+/* Paged decode with the dense rotation: as tq_paged_decode (sign_seed unused), with
+ * q' = R q and o = R^T O' / l (fp32 on the CUDA cores, once per query head). */
+TQ_API tq_status tq_paged_decode_dense(tq_tensor out, tq_tensor q, tq_tensor pages,
+                                       tq_tensor block_table, tq_tensor seq_lens,
+                                       const tq_codebooks* cb, const tq_rotation* rot, float scale,
+                                       void* stream);
+
+/* Test export of the dense append's rotation: for each bf16 row x of `x` [N, D] writes
+ * u = R x / ||x|| (fp32, [N, D], unit stride) and fp32(||x||) to `norm` [N] with exactly
+ * the arithmetic of tq_quantize_append_dense (the same kernel), so that encoding these u
+ * on the host reproduces its codes bit for bit.  Same limits as that call. */
+TQ_API tq_status tq_rotate_unit_dense(tq_tensor u, tq_tensor norm, tq_tensor x,
+                                      const tq_rotation* rot, void* stream);
 
 /* Test export for failure detection without a GPU fault (this library's own addition;
  * the pages describe no counterpart).  The NEXT decode launch on the current device

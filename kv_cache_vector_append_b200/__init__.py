@@ -11,8 +11,14 @@ Public API (names follow the C entry points):
     load_codebooks(D, k_bits, v_bits, device) -> Codebooks
     quantize_append(pages, slot_mapping, k, v, codebooks, sign_seed, stream=None)
     paged_decode(out, q, pages, block_table, seq_lens, codebooks, sign_seed, scale, stream=None)
+    paged_decode_hot(out, q, pages, block_table, seq_lens, hot_k, hot_v, hot_lens, ...)
+                                # same, plus an uncompressed hot window (sinks, recent tokens)
     paged_decode_noalloc(...)   # same, with the library's fixed scratch (no allocation)
     rotate_unit(u, norm, x, sign_seed, stream=None)       # test export of the rotation
+    load_rotation(D, device) -> Rotation                  # dense (QR) rotation table
+    quantize_append_dense(pages, slot_mapping, k, v, codebooks, rotation, stream=None)
+    paged_decode_dense(out, q, pages, block_table, seq_lens, codebooks, rotation, scale, ...)
+    rotate_unit_dense(u, norm, x, rotation, stream=None)  # test export of the dense rotation
     decode_workspace_size(...), set_workspace(tensor), get_device_error(stream=None)
 """
 
@@ -30,7 +36,13 @@ from ._binding import (  # noqa: F401
     library_path,
     load_codebook_table,
     load_codebooks,
+    load_rotation,
+    Rotation,
+    quantize_append_dense,
+    paged_decode_dense,
+    rotate_unit_dense,
     paged_decode,
+    paged_decode_hot,
     paged_decode_noalloc,
     quantize_append,
     rotate_unit,

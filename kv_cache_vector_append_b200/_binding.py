@@ -25,9 +25,11 @@ DEVERR_SEQLEN_RANGE = 0x8
 DEVERR_TIMEOUT = 0x10
 DEVERR_LAYOUT = 0x20
 
-EXPORTED = ("tq_slot_bytes", "tq_quantize_append", "tq_paged_decode", "tq_paged_decode_noalloc",
+EXPORTED = ("tq_slot_bytes", "tq_quantize_append", "tq_paged_decode", "tq_paged_decode_hot",
+            "tq_paged_decode_noalloc",
             "tq_decode_workspace_size", "tq_set_workspace", "tq_get_device_error",
             "tq_rotate_unit", "tq_decode_plan_probe", "tq_debug_inject_merge_stall",
+            "tq_quantize_append_dense", "tq_paged_decode_dense", "tq_rotate_unit_dense",
             "tq_status_string", "tq_version")
 
 
@@ -49,6 +51,10 @@ class CodebookDesc(ctypes.Structure):
 
 class CodebooksDesc(ctypes.Structure):
     _fields_ = [("k", CodebookDesc), ("v", CodebookDesc)]
+
+
+class RotationDesc(ctypes.Structure):
+    _fields_ = [("dim", ctypes.c_int32), ("hi", ctypes.c_void_p), ("lo", ctypes.c_void_p)]
 
 
 _lib = None
@@ -75,6 +81,8 @@ def _load():
                                     ctypes.c_void_p]
     lib.tq_paged_decode_noalloc.argtypes = [T, T, T, T, T, CB, ctypes.c_uint64, ctypes.c_float,
                                             ctypes.c_void_p]
+    lib.tq_paged_decode_hot.argtypes = [T, T, T, T, T, T, T, T, CB, ctypes.c_uint64,
+                                        ctypes.c_float, ctypes.c_void_p]
     lib.tq_decode_workspace_size.argtypes = [ctypes.c_int32] * 6 + [ctypes.POINTER(ctypes.c_size_t)]
     lib.tq_set_workspace.argtypes = [ctypes.c_void_p, ctypes.c_size_t]
     lib.tq_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p]
@@ -82,6 +90,11 @@ def _load():
     lib.tq_decode_plan_probe.argtypes = [ctypes.c_int32] * 10 + [ctypes.c_uint32,
                                                                  ctypes.POINTER(ctypes.c_int64)]
     lib.tq_debug_inject_merge_stall.argtypes = [ctypes.c_int32, ctypes.c_int32]
+    RT = ctypes.POINTER(RotationDesc)
+    lib.tq_quantize_append_dense.argtypes = [T, T, T, T, CB, RT, ctypes.c_int32, ctypes.c_int32,
+                                             ctypes.c_void_p]
+    lib.tq_paged_decode_dense.argtypes = [T, T, T, T, T, CB, RT, ctypes.c_float, ctypes.c_void_p]
+    lib.tq_rotate_unit_dense.argtypes = [T, T, T, RT, ctypes.c_void_p]
     lib.tq_status_string.argtypes = [ctypes.c_int]
     lib.tq_status_string.restype = ctypes.c_char_p
     lib.tq_version.restype = ctypes.c_char_p
@@ -158,9 +171,16 @@ class CodebookTable:
     boundaries: np.ndarray
 
 
-def load_codebook_table(dim: int, bits: int) -> CodebookTable:
-    """Read ``codebooks/beta_d{dim}_b{bits}.tqcb`` (magic, 7 u32, L f32, L-1 f32)."""
-    path = os.path.join(_CODEBOOK_DIR, f"beta_d{dim}_b{bits}.tqcb")
+CODEBOOK_KINDS = ("beta", "gauss")
+
+
+def load_codebook_table(dim: int, bits: int, kind: str = "beta") -> CodebookTable:
+    """Read ``codebooks/{kind}_d{dim}_b{bits}.tqcb`` (magic, 7 u32, L f32, L-1 f32):
+    kind "beta" is the exact Beta-sphere table, "gauss" its Gaussian approximation
+    N(0, 1/D) (TorbuQuant, "Current Status")."""
+    if kind not in CODEBOOK_KINDS:
+        raise ValueError(f"codebook kind {kind!r}: one of {CODEBOOK_KINDS}")
+    path = os.path.join(_CODEBOOK_DIR, f"{kind}_d{dim}_b{bits}.tqcb")
     with open(path, "rb") as f:
         raw = f.read()
     if raw[:4] != b"TQCB":
@@ -177,11 +197,11 @@ def load_codebook_table(dim: int, bits: int) -> CodebookTable:
 class Codebooks:
     """Device-resident K and V tables plus the C descriptor that points at them."""
 
-    def __init__(self, dim: int, k_bits: int, v_bits: int, device="cuda"):
+    def __init__(self, dim: int, k_bits: int, v_bits: int, device="cuda", kind: str = "beta"):
         torch = _torch()
-        self.dim, self.k_bits, self.v_bits = dim, k_bits, v_bits
-        self.k_table = load_codebook_table(dim, k_bits)
-        self.v_table = load_codebook_table(dim, v_bits)
+        self.dim, self.k_bits, self.v_bits, self.kind = dim, k_bits, v_bits, kind
+        self.k_table = load_codebook_table(dim, k_bits, kind)
+        self.v_table = load_codebook_table(dim, v_bits, kind)
         self.k_centroids = torch.from_numpy(self.k_table.centroids).to(device)
         self.k_boundaries = torch.from_numpy(self.k_table.boundaries).to(device)
         if v_bits == k_bits:
@@ -196,8 +216,38 @@ class Codebooks:
                                    self.v_boundaries.data_ptr())
 
 
-def load_codebooks(dim: int, k_bits: int, v_bits: int, device="cuda") -> Codebooks:
-    return Codebooks(dim, k_bits, v_bits, device)
+_ROTATION_DIR = os.path.join(_PKG, "rotations")
+
+
+class Rotation:
+    """Device copy of the dense rotation table ``rotations/qr_d{dim}.tqrt`` (magic, 3 u32,
+    then hi and lo as D*D bf16 bit patterns each) and the C descriptor pointing at it."""
+
+    def __init__(self, dim: int, device="cuda"):
+        torch = _torch()
+        path = os.path.join(_ROTATION_DIR, f"qr_d{dim}.tqrt")
+        with open(path, "rb") as f:
+            raw = f.read()
+        if raw[:4] != b"TQRT":
+            raise ValueError(f"{path}: not a rotation table")
+        version_, d, self.seed = struct.unpack_from("<3I", raw, 4)
+        if version_ != 1 or d != dim:
+            raise ValueError(f"{path}: unexpected header")
+        words = np.frombuffer(raw, dtype="<u2", count=2 * dim * dim, offset=16).copy()
+        self.dim = dim
+        w = torch.from_numpy(words.view(np.int16)).to(device)
+        self.hi = w[:dim * dim].contiguous()
+        self.lo = w[dim * dim:].contiguous()
+        self.desc = RotationDesc(dim, self.hi.data_ptr(), self.lo.data_ptr())
+
+
+def load_rotation(dim: int, device="cuda") -> Rotation:
+    return Rotation(dim, device)
+
+
+def load_codebooks(dim: int, k_bits: int, v_bits: int, device="cuda",
+                   kind: str = "beta") -> Codebooks:
+    return Codebooks(dim, k_bits, v_bits, device, kind)
 
 
 # ---------------------------------------------------------------------------
@@ -230,6 +280,19 @@ def paged_decode(out, q, pages, block_table, seq_lens, codebooks: Codebooks, sig
            "tq_paged_decode")
 
 
+def paged_decode_hot(out, q, pages, block_table, seq_lens, hot_k, hot_v, hot_lens,
+                     codebooks: Codebooks, sign_seed: int, scale: float, stream=None) -> None:
+    """tq_paged_decode_hot: the decode over the packed pages plus an uncompressed hot
+    window hot_k/hot_v [B, W, H_kv, D] holding hot_lens[b] tokens of sequence b."""
+    _require_cuda(out, q, pages, block_table, seq_lens, hot_k, hot_v, hot_lens)
+    st = _stream_handle(stream, q.device)
+    _check(_load().tq_paged_decode_hot(_desc(out), _desc(q), _desc(pages), _desc(block_table),
+                                       _desc(seq_lens), _desc(hot_k), _desc(hot_v),
+                                       _desc(hot_lens), ctypes.byref(codebooks.desc),
+                                       ctypes.c_uint64(sign_seed), ctypes.c_float(scale), st),
+           "tq_paged_decode_hot")
+
+
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -243,6 +306,35 @@ def paged_decode_noalloc(out, q, pages, block_table, seq_lens, codebooks: Codebo
                                            _desc(seq_lens), ctypes.byref(codebooks.desc),
                                            ctypes.c_uint64(sign_seed), ctypes.c_float(scale), st),
            "tq_paged_decode_noalloc")
+
+
+def quantize_append_dense(pages, slot_mapping, k, v, codebooks: Codebooks, rotation: Rotation,
+                          stream=None) -> None:
+    _require_cuda(pages, slot_mapping, k, v)
+    st = _stream_handle(stream, pages.device)
+    _check(_load().tq_quantize_append_dense(_desc(pages), _desc(slot_mapping), _desc(k),
+                                            _desc(v), ctypes.byref(codebooks.desc),
+                                            ctypes.byref(rotation.desc), codebooks.k_bits,
+                                            codebooks.v_bits, st),
+           "tq_quantize_append_dense")
+
+
+def paged_decode_dense(out, q, pages, block_table, seq_lens, codebooks: Codebooks,
+                       rotation: Rotation, scale: float, stream=None) -> None:
+    _require_cuda(out, q, pages, block_table, seq_lens)
+    st = _stream_handle(stream, q.device)
+    _check(_load().tq_paged_decode_dense(_desc(out), _desc(q), _desc(pages), _desc(block_table),
+                                         _desc(seq_lens), ctypes.byref(codebooks.desc),
+                                         ctypes.byref(rotation.desc), ctypes.c_float(scale), st),
+           "tq_paged_decode_dense")
+
+
+def rotate_unit_dense(u, norm, x, rotation: Rotation, stream=None) -> None:
+    _require_cuda(u, norm, x)
+    st = _stream_handle(stream, x.device)
+    _check(_load().tq_rotate_unit_dense(_desc(u), _desc(norm), _desc(x),
+                                        ctypes.byref(rotation.desc), st),
+           "tq_rotate_unit_dense")
 
 
 def rotate_unit(u, norm, x, sign_seed: int, stream=None) -> None:

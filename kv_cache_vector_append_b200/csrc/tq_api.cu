@@ -16,6 +16,9 @@ namespace tq {
 
 __device__ unsigned int g_tq_error_word;
 
+// Flag and counter of quantize-append's redo (see append_kernel): zero between calls.
+__device__ unsigned int g_tq_append_redo[2];
+
 // Scratch of tq_paged_decode_noalloc: a fixed device array that every device which
 // loads the library holds until the process exits.  Host code never dereferences
 // this name (on the host it is only a stand-in); its device address is looked up
@@ -39,6 +42,7 @@ struct DeviceState {
   // device address of g_tq_error_word; published (release) last by the one-time set-up,
   // so a non-null value means `info` is complete
   std::atomic<unsigned int*> err{nullptr};
+  unsigned int* redo = nullptr;   // device address of g_tq_append_redo
   void* user_ws = nullptr;
   size_t user_ws_bytes = 0;
   void* lib_ws = nullptr;
@@ -65,7 +69,11 @@ tq_status device_state(DeviceState** out) {
     std::lock_guard<std::mutex> lock(g_mu);
     if (s.err.load(std::memory_order_relaxed) == nullptr) {
       void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_tq_error_word) != cudaSuccess) return TQ_ERR_CUDA;
+      void* r = nullptr;
+      if (cudaGetSymbolAddress(&p, g_tq_error_word) != cudaSuccess ||
+          cudaGetSymbolAddress(&r, g_tq_append_redo) != cudaSuccess)
+        return TQ_ERR_CUDA;
+      s.redo = (unsigned int*)r;
       DeviceInfo info;
       if (cudaDeviceGetAttribute(&info.num_sms, cudaDevAttrMultiProcessorCount, dev) !=
           cudaSuccess)
@@ -118,6 +126,25 @@ bool valid_codebook(const tq_codebook& c, int dim) {
 }
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool valid_rotation(const tq_rotation* r, int dim) {
+  return r != nullptr && r->dim == dim && r->hi != nullptr && r->lo != nullptr &&
+         (uintptr_t)r->hi % 16 == 0 && (uintptr_t)r->lo % 16 == 0;
+}
+
+// Heads per tensor box of the dense append (a tile is 128 pairs: box_h heads x
+// 128 / box_h tokens), or 0 when h_kv neither divides 128 nor is a multiple of it.
+int dense_box_heads(int h_kv) {
+  if (h_kv <= kDenseRows && kDenseRows % h_kv == 0) return h_kv;
+  if (h_kv % kDenseRows == 0) return kDenseRows;
+  return 0;
+}
+
+// A bf16 [T, H_kv, D] input the dense append reads by tensor copies.
+bool dense_input_ok(const tq_tensor& t) {
+  return t.dtype == TQ_BF16 && (uintptr_t)t.data % 16 == 0 && t.stride[0] % 8 == 0 &&
+         t.stride[1] % 8 == 0;
+}
 
 int align_mode_of(const void* data, int esize, std::initializer_list<int64_t> strides) {
   auto ok = [&](int a) {
@@ -344,11 +371,36 @@ tq_status decode_prepare(const tq_tensor& out, const tq_tensor& q, const tq_tens
   return TQ_OK;
 }
 
+// Optional uncompressed hot window of a decode call.
+struct HotWindow {
+  const tq_tensor* k = nullptr;
+  const tq_tensor* v = nullptr;
+  const tq_tensor* lens = nullptr;
+};
+
+// Validation of a hot window against a prepared call: k and v [B, W, H_kv, D] of one
+// float dtype with equal strides and a contiguous last dim, lens i32 [B] contiguous.
+tq_status hot_validate(const DecodeCall& call, const tq_tensor& q, const HotWindow& hw) {
+  const tq_tensor &k = *hw.k, &v = *hw.v, &n = *hw.lens;
+  if (!valid_tensor(k, 4) || !valid_tensor(v, 4) || !is_float_dtype(k.dtype) ||
+      k.dtype != v.dtype || k.stride[3] != 1)
+    return TQ_ERR_INVALID_ARG;
+  for (int i = 0; i < 4; ++i)
+    if (k.shape[i] != v.shape[i] || k.stride[i] != v.stride[i]) return TQ_ERR_INVALID_ARG;
+  if (k.shape[0] != q.shape[0] || k.shape[3] != q.shape[2] || k.shape[1] > 0x7fffffff)
+    return TQ_ERR_INVALID_ARG;
+  if (call.B > 0 && k.shape[2] != call.h_kv) return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(n, 1) || n.dtype != TQ_I32 || n.stride[0] != 1 || n.shape[0] != q.shape[0])
+    return TQ_ERR_INVALID_ARG;
+  return TQ_OK;
+}
+
 // Launch the decode kernels of a prepared call on workspace `ws` (plan.ws_bytes bytes).
 tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tensor& q,
                      const tq_tensor& pages, const tq_tensor& block_table,
                      const tq_tensor& seq_lens, const tq_codebooks* cb, uint64_t sign_seed,
-                     float scale, uint8_t* ws, void* stream) {
+                     float scale, uint8_t* ws, void* stream, const HotWindow& hw = HotWindow(),
+                     const tq_rotation* rot = nullptr) {
   const int B = call.B, h_q = call.h_q, h_kv = call.h_kv, D = call.D;
   const int kbits = call.kbits, vbits = call.vbits, kb = call.kb;
   const int64_t stride = call.stride;
@@ -408,6 +460,21 @@ tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tens
   p.counters = (unsigned int*)(ws + plan.counters_off);
   p.wait_ms = kWaitMs;
   p.withhold_cta = -1;
+  p.rot_hi = rot ? rot->hi : nullptr;
+  p.rot_lo = rot ? rot->lo : nullptr;
+  p.hot_k = nullptr;
+  p.hot_v = nullptr;
+  p.hot_lens = nullptr;
+  if (hw.k != nullptr) {
+    p.hot_k = hw.k->data;
+    p.hot_v = hw.v->data;
+    p.hot_bstride = hw.k->stride[0];
+    p.hot_tstride = hw.k->stride[1];
+    p.hot_hstride = hw.k->stride[2];
+    p.hot_dtype = hw.k->dtype;
+    p.hot_cap = (int32_t)hw.k->shape[1];
+    p.hot_lens = (const int32_t*)hw.lens->data;
+  }
   {
     std::lock_guard<std::mutex> lock(g_mu);
     ds->counter_bytes = std::max(ds->counter_bytes, plan.part_off);
@@ -423,6 +490,30 @@ tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tens
   const int64_t steps_upper = (int64_t)B * ((max_blocks + plan.wph - 1) / plan.wph);
   cudaStream_t st = as_stream(stream);
   return launch_decode_any(D, kbits, vbits, p, plan, tmap, steps_upper, st);
+}
+
+// The workspace of a decode call: the caller's (tq_set_workspace) or the library's own,
+// grown on demand.
+tq_status decode_workspace(const DecodeCall& call, uint8_t** ws) {
+  DeviceState* ds = call.ds;
+  const DecodePlan& plan = call.plan;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (ds->user_ws != nullptr) {
+    if (ds->user_ws_bytes < plan.ws_bytes) return TQ_ERR_WORKSPACE;
+    *ws = (uint8_t*)ds->user_ws;
+    return TQ_OK;
+  }
+  if (ds->lib_ws_bytes < plan.ws_bytes) {
+    if (ds->lib_ws) cudaFree(ds->lib_ws);
+    ds->lib_ws = nullptr;
+    ds->lib_ws_bytes = 0;
+    size_t want = std::max<size_t>(plan.ws_bytes, 1 << 20);
+    if (cudaMalloc(&ds->lib_ws, want) != cudaSuccess) return TQ_ERR_WORKSPACE;
+    if (cudaMemset(ds->lib_ws, 0, want) != cudaSuccess) return TQ_ERR_CUDA;
+    ds->lib_ws_bytes = want;
+  }
+  *ws = (uint8_t*)ds->lib_ws;
+  return TQ_OK;
 }
 
 }  // namespace
@@ -513,6 +604,7 @@ tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_tensor 
   p.region_off[1] = kb;
   p.sign_seed = sign_seed;
   p.err = ds->err.load(std::memory_order_relaxed);
+  p.redo = ds->redo;
   const int es = dtype_size(k.dtype);
   p.align_mode = std::min(align_mode_of(k.data, es, {k.stride[0], k.stride[1]}),
                           align_mode_of(v.data, es, {v.stride[0], v.stride[1]}));
@@ -542,6 +634,126 @@ tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_tensor 
                        rows / p.run_heads))
     p.tma_in = 1;
   return launch_append_any(D, k.dtype, p, maps, ds->info, as_stream(stream));
+}
+
+tq_status tq_quantize_append_dense(tq_tensor pages, tq_tensor slot_mapping, tq_tensor k,
+                                   tq_tensor v, const tq_codebooks* cb, const tq_rotation* rot,
+                                   int32_t k_bits, int32_t v_bits, void* stream) {
+  if (cb == nullptr) return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(pages, 4) || pages.dtype != TQ_U8 || pages.stride[3] != 1)
+    return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(slot_mapping, 1) || slot_mapping.dtype != TQ_I64) return TQ_ERR_INVALID_ARG;
+  if (!valid_tensor(k, 3) || !valid_tensor(v, 3) || !is_float_dtype(k.dtype) ||
+      k.dtype != v.dtype || k.stride[2] != 1 || v.stride[2] != 1)
+    return TQ_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (k.shape[i] != v.shape[i]) return TQ_ERR_INVALID_ARG;
+  const int64_t T = k.shape[0];
+  const int h_kv = (int)k.shape[1];
+  const int D = (int)k.shape[2];
+  if (slot_mapping.shape[0] != T || pages.shape[2] != h_kv) return TQ_ERR_INVALID_ARG;
+  if (k_bits < 1 || k_bits > 8 || v_bits < 1 || v_bits > 8) return TQ_ERR_INVALID_ARG;
+  if (!valid_codebook(cb->k, D) || !valid_codebook(cb->v, D) || cb->k.bits != k_bits ||
+      cb->v.bits != v_bits || !valid_rotation(rot, D))
+    return TQ_ERR_INVALID_ARG;
+  const int kb = region_bytes(D, k_bits), vb = region_bytes(D, v_bits);
+  if (pages.shape[3] < kb + vb || pages.shape[3] % 8 != 0) return TQ_ERR_INVALID_ARG;
+  if (pages.stride[0] % 4 || pages.stride[1] % 4 || pages.stride[2] % 4 ||
+      (uintptr_t)pages.data % 4)
+    return TQ_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return TQ_ERR_UNSUPPORTED;
+  if (T == 0 || h_kv == 0) return TQ_OK;
+  const int box_h = dense_box_heads(h_kv);
+  if (box_h == 0 || !dense_input_ok(k) || !dense_input_ok(v)) return TQ_ERR_UNSUPPORTED;
+  if (T * h_kv >= ((int64_t)1 << 31) - 256) return TQ_ERR_UNSUPPORTED;
+  DeviceState* ds = nullptr;
+  tq_status s = device_state(&ds);
+  if (s != TQ_OK) return s;
+  DenseAppendParams p{};
+  p.pages = (uint8_t*)pages.data;
+  p.num_slots = pages.shape[0] * pages.shape[1];
+  p.block_size = (int32_t)pages.shape[1];
+  p.bs_shift = -1;
+  for (int sh = 0; sh < 31; ++sh)
+    if ((int64_t)1 << sh == pages.shape[1]) p.bs_shift = sh;
+  p.h_kv = h_kv;
+  p.blk_stride = pages.stride[0];
+  p.row_stride = pages.stride[1];
+  p.head_stride = pages.stride[2];
+  p.slot_mapping = (const int64_t*)slot_mapping.data;
+  p.slot_map_stride = slot_mapping.stride[0];
+  p.num_tokens = T;
+  p.boundaries[0] = cb->k.boundaries;
+  p.boundaries[1] = cb->v.boundaries;
+  p.bits[0] = k_bits;
+  p.bits[1] = v_bits;
+  p.rot_hi = rot->hi;
+  p.rot_lo = rot->lo;
+  p.err = ds->err.load(std::memory_order_relaxed);
+  p.box_h = box_h;
+  p.wait_ms = kWaitMs;
+  DenseAppendMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  if (!encode_input_map(&maps.k, k.data, T, h_kv, D, k.stride[0], k.stride[1], box_h,
+                        kDenseRows / box_h) ||
+      !encode_input_map(&maps.v, v.data, T, h_kv, D, v.stride[0], v.stride[1], box_h,
+                        kDenseRows / box_h))
+    return TQ_ERR_UNSUPPORTED;
+  return launch_append_dense_any(D, p, maps, ds->info, as_stream(stream));
+}
+
+tq_status tq_rotate_unit_dense(tq_tensor u, tq_tensor norm, tq_tensor x, const tq_rotation* rot,
+                               void* stream) {
+  if (!valid_tensor(x, 2) || !valid_tensor(u, 2) || !valid_tensor(norm, 1)) return TQ_ERR_INVALID_ARG;
+  if (x.dtype != TQ_BF16 || u.dtype != TQ_F32 || norm.dtype != TQ_F32) return TQ_ERR_INVALID_ARG;
+  if (x.stride[1] != 1 || u.stride[1] != 1 || norm.stride[0] != 1 || u.shape[0] != x.shape[0] ||
+      u.shape[1] != x.shape[1] || norm.shape[0] != x.shape[0])
+    return TQ_ERR_INVALID_ARG;
+  const int D = (int)x.shape[1];
+  if (!valid_rotation(rot, D)) return TQ_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return TQ_ERR_UNSUPPORTED;
+  if (x.shape[0] == 0) return TQ_OK;
+  if ((uintptr_t)x.data % 16 || x.stride[0] % 8 || x.shape[0] >= ((int64_t)1 << 31) - 256)
+    return TQ_ERR_UNSUPPORTED;
+  DeviceState* ds = nullptr;
+  tq_status s = device_state(&ds);
+  if (s != TQ_OK) return s;
+  DenseAppendParams p{};
+  p.num_tokens = x.shape[0];
+  p.h_kv = 1;
+  p.bits[0] = p.bits[1] = 1;
+  p.boundaries[0] = p.boundaries[1] = nullptr;
+  p.rot_hi = rot->hi;
+  p.rot_lo = rot->lo;
+  p.err = ds->err.load(std::memory_order_relaxed);
+  p.box_h = 1;
+  p.wait_ms = kWaitMs;
+  p.export_mode = 1;
+  p.u_out = (float*)u.data;
+  p.u_stride = u.stride[0];
+  p.n_out = (float*)norm.data;
+  DenseAppendMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  if (!encode_input_map(&maps.k, x.data, x.shape[0], 1, D, x.stride[0], D, 1, kDenseRows))
+    return TQ_ERR_UNSUPPORTED;
+  maps.v = maps.k;
+  return launch_append_dense_any(D, p, maps, ds->info, as_stream(stream));
+}
+
+tq_status tq_paged_decode_dense(tq_tensor out, tq_tensor q, tq_tensor pages,
+                                tq_tensor block_table, tq_tensor seq_lens,
+                                const tq_codebooks* cb, const tq_rotation* rot, float scale,
+                                void* stream) {
+  DecodeCall call;
+  tq_status s = decode_prepare(out, q, pages, block_table, seq_lens, cb, scale, &call);
+  if (s != TQ_OK) return s;
+  if (!valid_rotation(rot, (int)q.shape[2])) return TQ_ERR_INVALID_ARG;
+  if (call.B == 0) return TQ_OK;
+  uint8_t* ws = nullptr;
+  s = decode_workspace(call, &ws);
+  if (s != TQ_OK) return s;
+  return decode_run(call, out, q, pages, block_table, seq_lens, cb, 0, scale, ws, stream,
+                    HotWindow(), rot);
 }
 
 tq_status tq_decode_plan_probe(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
@@ -676,29 +888,30 @@ tq_status tq_paged_decode(tq_tensor out, tq_tensor q, tq_tensor pages, tq_tensor
   DecodeCall call;
   tq_status s = decode_prepare(out, q, pages, block_table, seq_lens, cb, scale, &call);
   if (s != TQ_OK || call.B == 0) return s;
-  DeviceState* ds = call.ds;
-  const DecodePlan& plan = call.plan;
   uint8_t* ws = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (ds->user_ws != nullptr) {
-      if (ds->user_ws_bytes < plan.ws_bytes) return TQ_ERR_WORKSPACE;
-      ws = (uint8_t*)ds->user_ws;
-    } else {
-      if (ds->lib_ws_bytes < plan.ws_bytes) {
-        if (ds->lib_ws) cudaFree(ds->lib_ws);
-        ds->lib_ws = nullptr;
-        ds->lib_ws_bytes = 0;
-        size_t want = std::max<size_t>(plan.ws_bytes, 1 << 20);
-        if (cudaMalloc(&ds->lib_ws, want) != cudaSuccess) return TQ_ERR_WORKSPACE;
-        if (cudaMemset(ds->lib_ws, 0, want) != cudaSuccess) return TQ_ERR_CUDA;
-        ds->lib_ws_bytes = want;
-      }
-      ws = (uint8_t*)ds->lib_ws;
-    }
-  }
-
+  s = decode_workspace(call, &ws);
+  if (s != TQ_OK) return s;
   return decode_run(call, out, q, pages, block_table, seq_lens, cb, sign_seed, scale, ws, stream);
+}
+
+tq_status tq_paged_decode_hot(tq_tensor out, tq_tensor q, tq_tensor pages, tq_tensor block_table,
+                              tq_tensor seq_lens, tq_tensor hot_k, tq_tensor hot_v,
+                              tq_tensor hot_lens, const tq_codebooks* cb, uint64_t sign_seed,
+                              float scale, void* stream) {
+  DecodeCall call;
+  tq_status s = decode_prepare(out, q, pages, block_table, seq_lens, cb, scale, &call);
+  if (s != TQ_OK) return s;
+  HotWindow hw;
+  hw.k = &hot_k;
+  hw.v = &hot_v;
+  hw.lens = &hot_lens;
+  s = hot_validate(call, q, hw);
+  if (s != TQ_OK || call.B == 0) return s;
+  uint8_t* ws = nullptr;
+  s = decode_workspace(call, &ws);
+  if (s != TQ_OK) return s;
+  return decode_run(call, out, q, pages, block_table, seq_lens, cb, sign_seed, scale, ws, stream,
+                    hw);
 }
 
 tq_status tq_paged_decode_noalloc(tq_tensor out, tq_tensor q, tq_tensor pages,

@@ -56,6 +56,7 @@ struct AppendParams {
   int32_t run_heads;        // heads of one token in a tile (tiles token-aligned), else 0
   int32_t tma_in;           // 1: input rows staged by tensor copies (maps K, V)
   int32_t bulk_out;         // 1: slots stored by one bulk copy per token run
+  unsigned int* redo;       // [2]: a row left the fast path's range; CTAs of the redo done
 };
 
 // Tensor maps of K and V as (D, h_kv, tokens) 16-bit elements, boxes of
@@ -383,31 +384,36 @@ __device__ __forceinline__ float fwht_ss(uint64_t (&xp)[32], int part) {
 // The rotation shared by quantize-append and its test export.  Loads this lane's 64
 // input elements of the row from the staged tile (`row`, `m`: see load_signed) and
 // leaves in xp the unnormalised transform H (s * x') of those coordinates, where x' is
-// the row scaled by 2^-e; returns r with u = xp * r.  *norm_out = ||x||_2 in fp32,
-// *bad_out = the row holds an infinity or NaN.
-// The scale keeps fp32 in range whatever the row's magnitude: e = 0 unless the sum of
-// squares ss of the unscaled transform (= D ||x||^2) falls outside [2^-60, 2^100] (so
-// the squares would overflow, or lose precision as subnormals) or is not a number.
-// Then the warp's rows out of range are rescaled in place in the staged tile by
-// 2^-e, e = floor(log2 max|x|) (largest magnitude in [1, 2)), and every row of the warp
-// is transformed again; multiplying by a power of two is exact, so a row in range
-// comes out bit for bit the same.  Order of operations (fixed, so that the export
-// reproduces the kernel exactly): the FWHT and ss of fwht_ss; n' = sqrt(ss / D)
-// (IEEE); r = 1 / (n' sqrt(D)) (IEEE reciprocal), or 0 when n' == 0; norm = n' 2^e.
-template <int D, typename Tin>
+// the row scaled by 2^-e; returns r with u = xp * r.  *norm_out = ||x||_2 in fp32.
+// The fast path (SAFE = false) takes e = 0 and sets *out_of_range when the sum of
+// squares ss of the transform (= D ||x||^2) falls outside [2^-60, 2^100] (squares that
+// overflow fp32 or lose precision as subnormals, a zero row, a non-finite row); such a
+// call is then redone by the safe path.  The safe path (SAFE = true; also the test
+// export) rescales the warp's rows that are out of range in place in the staged tile
+// by 2^-e, e = floor(log2 max|x|) (largest magnitude in [1, 2)), and transforms every
+// row of the warp again; multiplying by a power of two is exact, so a row in range
+// comes out bit for bit as in the fast path.  *bad_out = the row holds an infinity or
+// NaN (safe path only).  Order of operations (fixed, so that the export reproduces the
+// kernel exactly): the FWHT and ss of fwht_ss; n' = sqrt(ss / D) (IEEE);
+// r = 1 / (n' sqrt(D)) (IEEE reciprocal), or 0 when n' == 0; norm = n' 2^e.
+template <int D, typename Tin, bool SAFE>
 __device__ __forceinline__ float rotate_row(uint64_t (&xp)[32], uint32_t row, const uint32_t* m,
-                                            int part, float* norm_out, bool* bad_out) {
+                                            int part, float* norm_out, bool* bad_out,
+                                            bool* out_of_range) {
   int e = 0;
   bool bad = false;
-  float ss;
-#pragma unroll 1
-  for (int pass = 0;; ++pass) {
-    load_signed<Tin>(xp, row, m);
-    ss = fwht_ss<D>(xp, part);
-    const bool in_range = ss >= 0x1p-60f && ss <= 0x1p100f;
-    if (pass > 0 || !__any_sync(0xffffffffu, !in_range)) break;
-    e = rescale_staged_row<D, Tin>(row, !in_range, &bad);
-    __syncwarp();
+  load_signed<Tin>(xp, row, m);
+  float ss = fwht_ss<D>(xp, part);
+  const bool in_range = ss >= 0x1p-60f && ss <= 0x1p100f;
+  if constexpr (SAFE) {
+    if (__any_sync(0xffffffffu, !in_range)) {
+      e = rescale_staged_row<D, Tin>(row, !in_range, &bad);
+      __syncwarp();
+      load_signed<Tin>(xp, row, m);
+      ss = fwht_ss<D>(xp, part);
+    }
+  } else {
+    *out_of_range = !in_range;
   }
   // ||H s x'||^2 = D ||x'||^2
   const float n = sqrtf(__fmul_rn(ss, 1.0f / D));
@@ -497,9 +503,17 @@ struct AppendSmem {
 // coordinates a lane), into the tile's slots staged in shared memory; then it stores
 // the full slots (whole-slot stores, so every DRAM sector of a slot is written by one
 // store pass).  Input rows are staged one half-tile ahead.
-template <int D, typename Tin>
+// SAFE = false: the fast path (rows of ordinary magnitude); when some row leaves its
+// range the kernel raises redo[0].  SAFE = true: launched right after it; every CTA
+// returns at once unless redo[0] is set, and otherwise the whole call is done again
+// with the rescaling rotation (identical results for the other rows); the last CTA
+// clears redo.
+template <int D, typename Tin, bool SAFE>
 __global__ void __launch_bounds__(kAppendWarps * 32, 2)
 append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
+  if constexpr (SAFE) {
+    if (*(volatile unsigned int*)&p.redo[0] == 0u) return;
+  }
   using G = AppendGeom<D>;
   using SM = AppendSmem<D, Tin>;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -609,6 +623,7 @@ append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
   const uint32_t row0 = smem_u32(in_s) + (uint32_t)((part * G::ROWS + rl) * SM::PB) +
                         (uint32_t)((rl & 7) << 4);
   int tb = 0;
+  bool redo_needed = false;                 // a row of this lane left the fast path's range
   uint32_t it = 0;                          // tiles done by this warp (mbarrier phase)
   uint32_t staged[2] = {gwarp < ntiles ? 1u : 0u, 0u};   // tensor copies issued per kind
   bool dead = false;
@@ -642,9 +657,10 @@ append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
       const int rwords = kind ? vwords : kwords;          // packed words + norm word
       uint64_t xp[32];
       float n;
-      bool bad;
-      const float r = rotate_row<D, Tin>(xp, row0 + (uint32_t)(kind * SM::KIND), smask + part * 64,
-                                         part, &n, &bad);
+      bool bad, oor;
+      const float r = rotate_row<D, Tin, SAFE>(xp, row0 + (uint32_t)(kind * SM::KIND),
+                                               smask + part * 64, part, &n, &bad, &oor);
+      if constexpr (!SAFE) redo_needed |= oor && rl < nr;
       if (kind == 0 && p.bulk_out) {    // the previous tile's slots have been read out
         bulk_wait_read_all();
         __syncwarp();
@@ -707,6 +723,16 @@ append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
         if (!mbar_wait(&bars[kind], c & 1u, kWaitMs)) break;
   }
   bulk_wait_all();
+  if constexpr (!SAFE) {
+    if (__any_sync(0xffffffffu, redo_needed) && lane == 0) atomicExch(&p.redo[0], 1u);
+  } else {
+    // the last CTA of the redo clears the flag (every CTA has read it by then)
+    __syncthreads();
+    if (threadIdx.x == 0 && atomicAdd(&p.redo[1], 1u) == gridDim.x - 1) {
+      atomicExch(&p.redo[0], 0u);
+      atomicExch(&p.redo[1], 0u);
+    }
+  }
 }
 
 // Test export: the rotation of tq_quantize_append, written out as fp32 u and n.
@@ -740,8 +766,8 @@ rotate_unit_kernel(RotateParams p) {
     __syncwarp();
     uint64_t xp[32];
     float n;
-    bool bad;
-    const float r = rotate_row<D, Tin>(xp, row, smask + part * 64, part, &n, &bad);
+    bool bad, oor;
+    const float r = rotate_row<D, Tin, true>(xp, row, smask + part * 64, part, &n, &bad, &oor);
     if (rl < nr) {
       float* u = p.u + (r0 + rl) * p.u_row_stride + part * 64;
       const uint64_t r2 = f2(r, r);

@@ -11,9 +11,12 @@ tq_status launch_append_t(const AppendParams& p, const AppendMaps& maps, const D
                           cudaStream_t st) {
   const size_t smem = AppendSmem<D, Tin>::bytes(p.bits[0], p.bits[1]);
   if ((int)smem > di.max_smem_optin) return TQ_ERR_UNSUPPORTED;
-  auto kern = append_kernel<D, Tin>;
+  auto kern = append_kernel<D, Tin, false>;
+  auto kern_safe = append_kernel<D, Tin, true>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
+          cudaSuccess ||
+      cudaFuncSetAttribute(kern_safe, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+          cudaSuccess)
     return TQ_ERR_CUDA;
   using G = AppendGeom<D>;
   const int64_t tiles = (p.num_tokens * p.h_kv + G::ROWS - 1) / G::ROWS;
@@ -25,7 +28,9 @@ tq_status launch_append_t(const AppendParams& p, const AppendMaps& maps, const D
   const int64_t max_ctas = (int64_t)di.num_sms * per_sm;
   const int64_t want = (tiles + kAppendWarps - 1) / kAppendWarps;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, max_ctas));
+  // the fast path, then the redo that runs only when a row left the fast path's range
   kern<<<grid, kAppendWarps * 32, smem, st>>>(p, maps);
+  kern_safe<<<grid, kAppendWarps * 32, smem, st>>>(p, maps);
   return launch_status();
 }
 

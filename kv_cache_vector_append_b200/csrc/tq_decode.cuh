@@ -112,7 +112,29 @@ struct DecodeParams {
   unsigned int* err;
   uint32_t wait_ms;             // limit of every bounded wait (milliseconds)
   int32_t withhold_cta;         // test hook: this CTA never announces its records (-1: none)
+  // Dense rotation R = hi + lo (bf16 bit patterns, [D][D] row-major) in place of the
+  // randomized Hadamard transform when rot_hi is not null: q' = R q, o = R^T O' / l.
+  const uint16_t* rot_hi;
+  const uint16_t* rot_lo;
+  // Uncompressed hot window (absent when hot_k is null): hot_k, hot_v [B, W, H_kv, D]
+  // with the last dim contiguous (strides in elements); sequence b also attends to its
+  // hot tokens 0 .. hot_lens[b]-1, inside the same softmax.
+  const void* hot_k;
+  const void* hot_v;
+  int64_t hot_bstride, hot_tstride, hot_hstride;
+  int32_t hot_dtype;
+  int32_t hot_cap;              // W
+  const int32_t* hot_lens;
 };
+
+// Attention partial of query head h of sequence b over its hot-window tokens, computed
+// by one warp in the original (unrotated) domain: lane l handles coordinates
+// l E .. l E + E - 1.  With s_t = scale log2(e) <q, k_t> (fp32): M = max_t s_t,
+// L = sum_t 2^(s_t - M), o = sum_t 2^(s_t - M) v_t (this lane's coordinates).  A
+// hot_lens entry outside [0, W] raises TQ_DEVERR_SEQLEN_RANGE and counts as 0 tokens.
+template <int D>
+__device__ __forceinline__ void hot_partial(const DecodeParams& p, int b, int h, int lane,
+                                            float& M, float& L, float (&o)[D / 32]);
 
 // Step range of CTA c out of C over S steps: [floor(c S / C), floor((c+1) S / C)).
 __host__ __device__ __forceinline__ int64_t cta_begin(int64_t c, int64_t S, int64_t C) {
@@ -213,8 +235,10 @@ struct Share {
 // Lookup tables.  Entry e of a table is row e (kLutRow bytes) of the table area at
 // the start of dynamic shared memory; lane l reads its copy of the K entry at byte
 // 4l of the row and its copy of the V entry at byte 128 + 4l.  For BITS <= 4 an entry
-// is a code pair: entry (x | y << BITS) = half2(c[x], c[y]); for BITS = 8 it is a
-// single code: entry x = half2(c[x], c[x]).
+// is a code pair: entry (x | y << BITS) = half2(c[x], c[y]); for BITS > 4 it is a
+// single code split in two halves: entry x = half2(hi, lo), hi = fp16(c[x]) and
+// lo = fp16(c[x] - hi), so that hi + lo carries c[x] to about 2^-22 (the K contraction
+// of 8-bit codes uses both).
 // ---------------------------------------------------------------------------
 __host__ __device__ constexpr int lut_entries(int bits) {
   return bits <= 4 ? 1 << (2 * bits) : 1 << bits;
@@ -227,8 +251,12 @@ __device__ __forceinline__ void lut_build(uint8_t* lut, const float* c, int tid,
   for (int i = tid; i < kEntries * 32; i += nt) {
     const int e = i >> 5, l = i & 31;
     uint32_t v;
-    if constexpr (BITS <= 4) v = pack_half2(c[e & ((1 << BITS) - 1)], c[e >> BITS]);
-    else v = pack_half2(c[e], c[e]);
+    if constexpr (BITS <= 4) {
+      v = pack_half2(c[e & ((1 << BITS) - 1)], c[e >> BITS]);
+    } else {
+      const float hi = __half2float(__float2half_rn(c[e]));
+      v = pack_half2(hi, c[e] - hi);
+    }
     *(uint32_t*)(lut + e * kLutRow + HALF * 128 + 4 * l) = v;
   }
 }
@@ -268,15 +296,18 @@ __device__ __forceinline__ uint32_t lut_ld(uint32_t addr) {
 }
 
 // half2 (c[x], c[y]) of the codes x, y of one thread's share (consecutive codes at
-// bit POS of the word array: one pair field, or two 8-bit fields).
+// bit POS of the word array: one pair field, or two single-code fields).  For BITS > 4
+// *rest receives half2 of the low parts (c[x] - hi[x], c[y] - hi[y]).
 template <int BITS, int POS, int NW>
-__device__ __forceinline__ uint32_t lut_pair(const uint32_t (&w)[NW], uint32_t off) {
+__device__ __forceinline__ uint32_t lut_pair(const uint32_t (&w)[NW], uint32_t off,
+                                             uint32_t* rest = nullptr) {
   if constexpr (BITS <= 4) {
     return lut_ld(lut_addr<POS, 2 * BITS>(w, off));
   } else {
-    const uint32_t lo = lut_ld(lut_addr<POS, BITS>(w, off));
-    const uint32_t hi = lut_ld(lut_addr<POS + BITS, BITS>(w, off));
-    return __byte_perm(lo, hi, 0x7610);   // low half of lo, high half of hi
+    const uint32_t ex = lut_ld(lut_addr<POS, BITS>(w, off));
+    const uint32_t ey = lut_ld(lut_addr<POS + BITS, BITS>(w, off));
+    if (rest) *rest = __byte_perm(ex, ey, 0x7632);   // high halves: the low parts
+    return __byte_perm(ex, ey, 0x5410);              // low halves: fp16(c)
   }
 }
 // half2 (c[x], c[y]) with x the code at bit POS of w0 and y the code at bit POS of w1.
@@ -287,9 +318,9 @@ __device__ __forceinline__ uint32_t lut_pair2(const uint32_t (&w0)[NW], const ui
     const uint32_t x = field<POS, BITS>(w0), y = field<POS, BITS>(w1);
     return lut_ld(((x | (y << BITS)) << 8) | off);
   } else {
-    const uint32_t lo = lut_ld(lut_addr<POS, BITS>(w0, off));
-    const uint32_t hi = lut_ld(lut_addr<POS, BITS>(w1, off));
-    return __byte_perm(lo, hi, 0x7610);
+    const uint32_t ex = lut_ld(lut_addr<POS, BITS>(w0, off));
+    const uint32_t ey = lut_ld(lut_addr<POS, BITS>(w1, off));
+    return __byte_perm(ex, ey, 0x5410);              // fp16(c[x]), fp16(c[y])
   }
 }
 
@@ -348,10 +379,108 @@ __device__ __forceinline__ void warp_fwht(float (&x)[E], int lane) {
     }
 }
 
+// R[r][lane E + i] for i < E (hi + lo, exact in fp32), E = D / 32 consecutive entries.
+template <int E>
+__device__ __forceinline__ void rot_row_part(const DecodeParams& p, int D, int r, int lane,
+                                             float (&v)[E]) {
+  const int64_t o = (int64_t)r * D + lane * E;
+#pragma unroll
+  for (int i = 0; i < E; ++i)
+    v[i] = __uint_as_float((uint32_t)p.rot_hi[o + i] << 16) +
+           __uint_as_float((uint32_t)p.rot_lo[o + i] << 16);
+}
+
+// y = R x for one warp: lane l holds x[l E + i] on entry and y[l E + i] on exit.  Output c
+// is the warp sum of the lanes' partial dot products with row c of R (fp32), kept in
+// `sc` (D floats of this warp's shared scratch).
+template <int E>
+__device__ __forceinline__ void dense_forward(const DecodeParams& p, float (&x)[E], int lane,
+                                              float* sc) {
+  constexpr int D = 32 * E;
+  for (int c = 0; c < D; ++c) {
+    float r[E];
+    rot_row_part<E>(p, D, c, lane, r);
+    float part = 0.f;
+#pragma unroll
+    for (int i = 0; i < E; ++i) part = fmaf(r[i], x[i], part);
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
+    if (lane == 0) sc[c] = part;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < E; ++i) x[i] = sc[lane * E + i];
+  __syncwarp();
+}
+
+// o = R^T a for one warp: lane l holds a[l E + i] on entry and o[l E + i] on exit;
+// o_c = sum_j R[j][c] a_j accumulated in fp32 over j = 0 .. D-1.
+template <int E>
+__device__ __forceinline__ void dense_inverse(const DecodeParams& p, float (&a)[E], int lane,
+                                              float* sc) {
+  constexpr int D = 32 * E;
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < E; ++i) sc[lane * E + i] = a[i];
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < E; ++i) a[i] = 0.f;
+  for (int j = 0; j < D; ++j) {
+    float r[E];
+    rot_row_part<E>(p, D, j, lane, r);
+    const float aj = sc[j];
+#pragma unroll
+    for (int i = 0; i < E; ++i) a[i] = fmaf(r[i], aj, a[i]);
+  }
+  __syncwarp();
+}
+
 __device__ __forceinline__ float load_as_f32(const void* base, int64_t i, int32_t dtype) {
   if (dtype == TQ_F32) return ((const float*)base)[i];
   if (dtype == TQ_BF16) return __bfloat162float(((const __nv_bfloat16*)base)[i]);
   return __half2float(((const __half*)base)[i]);
+}
+
+template <int D>
+__device__ __forceinline__ void hot_partial(const DecodeParams& p, int b, int h, int lane,
+                                            float& M, float& L, float (&o)[D / 32]) {
+  constexpr int E = D / 32;
+  M = -INFINITY;
+  L = 0.f;
+#pragma unroll
+  for (int i = 0; i < E; ++i) o[i] = 0.f;
+  int n = p.hot_lens[b];
+  if (n < 0 || n > p.hot_cap) {
+    if (lane == 0) report_error(p.err, TQ_DEVERR_SEQLEN_RANGE);
+    n = 0;
+  }
+  if (n == 0) return;
+  float qv[E];
+  const int64_t qo = (int64_t)b * p.q_bstride + (int64_t)h * p.q_hstride + lane * E;
+#pragma unroll
+  for (int i = 0; i < E; ++i) qv[i] = load_as_f32(p.q, qo + i, p.q_dtype);
+  const int64_t base = (int64_t)b * p.hot_bstride + (int64_t)(h / p.group) * p.hot_hstride +
+                       lane * E;
+  for (int t = 0; t < n; ++t) {
+    const int64_t off = base + (int64_t)t * p.hot_tstride;
+    float dot = 0.f;
+#pragma unroll
+    for (int i = 0; i < E; ++i) dot = fmaf(qv[i], load_as_f32(p.hot_k, off + i, p.hot_dtype), dot);
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, m);
+    const float sc = dot * p.scale_log2;
+    if (sc > M) {
+      const float f = M == -INFINITY ? 0.f : exp2f(M - sc);
+      L *= f;
+#pragma unroll
+      for (int i = 0; i < E; ++i) o[i] *= f;
+      M = sc;
+    }
+    const float w = exp2f(sc - M);
+    L += w;
+#pragma unroll
+    for (int i = 0; i < E; ++i) o[i] = fmaf(w, load_as_f32(p.hot_v, off + i, p.hot_dtype), o[i]);
+  }
 }
 
 __device__ __forceinline__ void store_from_f32(void* base, int64_t i, int32_t dtype, float v) {
@@ -455,12 +584,24 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     for (int b = lo; b < hi; ++b) { run += prefix[b + 1]; prefix[b + 1] = run; }
     __syncthreads();
   }
-  // sequences without steps (empty or rejected) give 0
+  // sequences without steps (empty or rejected) give 0, or attend to their hot window
+  // alone (one warp per query head)
   for (int b = blockIdx.x; b < B; b += gridDim.x) {
     if (prefix[b + 1] != prefix[b]) continue;
-    for (int i = tid; i < p.h_q * D; i += nthreads)
-      store_from_f32(p.out, (int64_t)b * p.o_bstride + (int64_t)(i / D) * p.o_hstride + i % D,
-                     p.out_dtype, 0.f);
+    if (p.hot_k == nullptr) {
+      for (int i = tid; i < p.h_q * D; i += nthreads)
+        store_from_f32(p.out, (int64_t)b * p.o_bstride + (int64_t)(i / D) * p.o_hstride + i % D,
+                       p.out_dtype, 0.f);
+    } else {
+      for (int h = warp; h < p.h_q; h += nwarps) {
+        float M, L, o[E];
+        hot_partial<D>(p, b, h, lane, M, L, o);
+        const float inv = L > 0.f ? 1.0f / L : 0.f;
+        const int64_t ob = (int64_t)b * p.o_bstride + (int64_t)h * p.o_hstride + lane * E;
+#pragma unroll
+        for (int i = 0; i < E; ++i) store_from_f32(p.out, ob + i, p.out_dtype, o[i] * inv);
+      }
+    }
   }
   const int64_t S = prefix[B];
   const int64_t Cn = gridDim.x;
@@ -581,15 +722,18 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
 #pragma unroll
     for (int i = 0; i < E; ++i) sg[i] = sign_mask_at(p.sign_seed, lane * E + i);
     auto rotate_head = [&](int h, float (&xq)[E]) {
+      if (p.rot_hi != nullptr) {
+        dense_forward<E>(p, xq, lane, scratch + warp * (D + 2));
+      } else {
 #pragma unroll
-      for (int i = 0; i < E; ++i) xq[i] = __uint_as_float(__float_as_uint(xq[i]) ^ sg[i]);
-      warp_fwht<E>(xq, lane);
+        for (int i = 0; i < E; ++i) xq[i] = __uint_as_float(__float_as_uint(xq[i]) ^ sg[i]);
+        warp_fwht<E>(xq, lane);
+#pragma unroll
+        for (int i = 0; i < E; ++i) xq[i] *= inv_sqrt_dim<D>();
+      }
       float ss = 0.f;
 #pragma unroll
-      for (int i = 0; i < E; ++i) {
-        xq[i] *= inv_sqrt_dim<D>();
-        ss = fmaf(xq[i], xq[i], ss);
-      }
+      for (int i = 0; i < E; ++i) ss = fmaf(xq[i], xq[i], ss);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       const float nrm = sqrtf(ss);
@@ -827,15 +971,41 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
             for (int i = 0; i < E; ++i) acc_o[i] = fmaf(f, sc[2 + lane * E + i], acc_o[i]);
           }
         }
-        const float inv = L > 0.f ? 1.0f / L : 0.f;
-#pragma unroll
-        for (int i = 0; i < E; ++i) acc_o[i] *= inv;
-        warp_fwht<E>(acc_o, lane);
         const int64_t ob = (int64_t)b * p.o_bstride + (int64_t)h * p.o_hstride + lane * E;
+        // o = R^T a: the dense rotation, or the FWHT, 1/sqrt(D) and the sign flips
+        auto inverse_rotate = [&](float (&a)[E]) {
+          if (p.rot_hi != nullptr) {
+            dense_inverse<E>(p, a, lane, scratch + warp * (D + 2));
+          } else {
+            warp_fwht<E>(a, lane);
 #pragma unroll
-        for (int i = 0; i < E; ++i)
-          store_from_f32(p.out, ob + i, p.out_dtype,
-                         __uint_as_float(__float_as_uint(acc_o[i] * inv_sqrt_dim<D>()) ^ sg[i]));
+            for (int i = 0; i < E; ++i)
+              a[i] = __uint_as_float(__float_as_uint(a[i] * inv_sqrt_dim<D>()) ^ sg[i]);
+          }
+        };
+        if (p.hot_k == nullptr) {
+          const float inv = L > 0.f ? 1.0f / L : 0.f;
+#pragma unroll
+          for (int i = 0; i < E; ++i) acc_o[i] *= inv;
+          inverse_rotate(acc_o);
+#pragma unroll
+          for (int i = 0; i < E; ++i) store_from_f32(p.out, ob + i, p.out_dtype, acc_o[i]);
+        } else {
+          // R^T O' of the packed tokens (not yet divided by L), then one softmax with
+          // the hot window's partial: rescale both to the larger reference and divide
+          // by the joint sum
+          inverse_rotate(acc_o);
+          float Mh, Lh, oh[E];
+          hot_partial<D>(p, b, h, lane, Mh, Lh, oh);
+          const float Mt = fmaxf(Mx, Mh);
+          const float f1 = Mx == -INFINITY ? 0.f : exp2f(Mx - Mt);
+          const float f2 = Mh == -INFINITY ? 0.f : exp2f(Mh - Mt);
+          const float Lt = f1 * L + f2 * Lh;
+          const float inv = Lt > 0.f ? 1.0f / Lt : 0.f;
+#pragma unroll
+          for (int i = 0; i < E; ++i)
+            store_from_f32(p.out, ob + i, p.out_dtype, (f1 * acc_o[i] + f2 * oh[i]) * inv);
+        }
       }
       __syncthreads();
     }
@@ -882,13 +1052,28 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
           KS::load(kw1, base + (gid + 8) * pitch, tig);
           static_for<C::KSTEPS>([&](auto KSI) {
             constexpr int ks = decltype(KSI)::value;
-            const uint32_t a0 = lut_pair<KB, KS::pos(4 * ks)>(kw0, lk_off);
-            const uint32_t a1 = lut_pair<KB, KS::pos(4 * ks)>(kw1, lk_off);
-            const uint32_t a2 = lut_pair<KB, KS::pos(4 * ks + 2)>(kw0, lk_off);
-            const uint32_t a3 = lut_pair<KB, KS::pos(4 * ks + 2)>(kw1, lk_off);
+            if constexpr (KB <= 4) {
+              const uint32_t a0 = lut_pair<KB, KS::pos(4 * ks)>(kw0, lk_off);
+              const uint32_t a1 = lut_pair<KB, KS::pos(4 * ks)>(kw1, lk_off);
+              const uint32_t a2 = lut_pair<KB, KS::pos(4 * ks + 2)>(kw0, lk_off);
+              const uint32_t a3 = lut_pair<KB, KS::pos(4 * ks + 2)>(kw1, lk_off);
   #pragma unroll
-            for (int hh = 0; hh < NH; ++hh)
-              mma_16816(sacc[hh], a0, a1, a2, a3, qb[ks][hh][0], qb[ks][hh][1]);
+              for (int hh = 0; hh < NH; ++hh)
+                mma_16816(sacc[hh], a0, a1, a2, a3, qb[ks][hh][0], qb[ks][hh][1]);
+            } else {
+              // wide codes: the fp16 centroids, then their low parts (c - fp16(c)), so that
+              // the scores carry the fp32 table to about 2^-22
+              uint32_t r0, r1, r2, r3;
+              const uint32_t a0 = lut_pair<KB, KS::pos(4 * ks)>(kw0, lk_off, &r0);
+              const uint32_t a1 = lut_pair<KB, KS::pos(4 * ks)>(kw1, lk_off, &r1);
+              const uint32_t a2 = lut_pair<KB, KS::pos(4 * ks + 2)>(kw0, lk_off, &r2);
+              const uint32_t a3 = lut_pair<KB, KS::pos(4 * ks + 2)>(kw1, lk_off, &r3);
+  #pragma unroll
+              for (int hh = 0; hh < NH; ++hh) {
+                mma_16816(sacc[hh], a0, a1, a2, a3, qb[ks][hh][0], qb[ks][hh][1]);
+                mma_16816(sacc[hh], r0, r1, r2, r3, qb[ks][hh][0], qb[ks][hh][1]);
+              }
+            }
           });
         }
         // this thread's tokens: r = 0, 1  <->  token gid + 8 r

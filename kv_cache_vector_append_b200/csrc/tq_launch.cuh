@@ -8,6 +8,7 @@
 
 #include "tq.h"
 #include "tq_append.cuh"
+#include "tq_append_dense.cuh"
 #include "tq_decode.cuh"
 
 namespace tq {
@@ -44,6 +45,8 @@ tq_status launch_append_any(int dim, int dtype, const AppendParams& p, const App
                             const DeviceInfo& di, cudaStream_t st);
 tq_status launch_rotate_any(int dim, int dtype, const RotateParams& p, const DeviceInfo& di,
                             cudaStream_t st);
+tq_status launch_append_dense_any(int dim, const DenseAppendParams& p, const DenseAppendMaps& maps,
+                                  const DeviceInfo& di, cudaStream_t st);
 // Code widths with a compiled decode kernel: K and V independently in {2, 3, 4, 8}.
 inline bool decode_bits_supported(int kb, int vb) {
   auto ok = [](int b) { return b == 2 || b == 3 || b == 4 || b == 8; };

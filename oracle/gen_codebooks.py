@@ -10,7 +10,7 @@ File format (little endian), one file per (D, bits):
     u32      version (1)
     u32      D
     u32      bits
-    u32      density id (0 = Beta-sphere, 1 = Gaussian)
+    u32      density id (0 = Beta-sphere, 1 = Gaussian approximation N(0, 1/D))
     u32      n_iter (iteration budget of Lloyd's iteration)
     u32      iterations actually run (< n_iter when a fixed point was reached)
     u32      reserved (0)
@@ -44,8 +44,15 @@ DEFAULT_OUT = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__fil
                            "kv_cache_vector_append_b200", "codebooks")
 
 
-def table_filename(dim: int, bits: int) -> str:
-    return f"beta_d{dim}_b{bits}.tqcb"
+KINDS = ("beta", "gauss")
+
+
+def table_filename(dim: int, bits: int, kind: str = "beta") -> str:
+    """beta_d<D>_b<bits>.tqcb: exact Beta-sphere density; gauss_d<D>_b<bits>.tqcb: its
+    Gaussian approximation N(0, 1/D)."""
+    if kind not in KINDS:
+        raise ValueError(kind)
+    return f"{kind}_d{dim}_b{bits}.tqcb"
 
 
 def write_table(path: str, t: O.CodebookTable) -> None:
@@ -74,29 +81,34 @@ def read_table(path: str) -> O.CodebookTable:
                            iterations_run=iters, centroids=c, boundaries=b.astype(np.float32))
 
 
-def build_table(dim: int, bits: int, n_iter: int = N_ITER) -> O.CodebookTable:
-    cb = O.lloyd_max_beta(dim, bits, n_iter)
-    return O.to_fp32_table(cb, dim, bits, O.BetaSphereDensity.density_id)
+def build_table(dim: int, bits: int, n_iter: int = N_ITER, kind: str = "beta") -> O.CodebookTable:
+    if kind == "beta":
+        cb = O.lloyd_max_beta(dim, bits, n_iter)
+        return O.to_fp32_table(cb, dim, bits, O.BetaSphereDensity.density_id)
+    cb = O.lloyd_max_gaussian_dim(dim, bits, n_iter)
+    return O.to_fp32_table(cb, dim, bits, O.GaussianDensity.density_id)
 
 
 def _job(args):
-    dim, bits, out = args
-    t = build_table(dim, bits)
-    write_table(os.path.join(out, table_filename(dim, bits)), t)
-    return dim, bits, t.iterations_run
+    dim, bits, out, kind = args
+    t = build_table(dim, bits, kind=kind)
+    write_table(os.path.join(out, table_filename(dim, bits, kind)), t)
+    return dim, bits, kind, t.iterations_run
 
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--out", default=DEFAULT_OUT)
     ap.add_argument("--jobs", type=int, default=os.cpu_count() or 1)
+    ap.add_argument("--kind", choices=KINDS + ("all",), default="all")
     args = ap.parse_args(argv)
     os.makedirs(args.out, exist_ok=True)
-    jobs = [(d, b, args.out) for b in sorted(BITS, reverse=True) for d in DIMS]
+    kinds = KINDS if args.kind == "all" else (args.kind,)
+    jobs = [(d, b, args.out, k) for k in kinds for b in sorted(BITS, reverse=True) for d in DIMS]
     ctx = mp.get_context("spawn")
     with ctx.Pool(args.jobs) as pool:
-        for dim, bits, iters in pool.imap_unordered(_job, jobs):
-            print(f"D={dim:4d} bits={bits}: {iters} iterations")
+        for dim, bits, kind, iters in pool.imap_unordered(_job, jobs):
+            print(f"{kind:5s} D={dim:4d} bits={bits}: {iters} iterations")
     return 0
 
 

@@ -154,6 +154,81 @@ def rht_matrix(dim: int, signs: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# Rotation: dense random orthogonal matrix (QR)
+# ---------------------------------------------------------------------------
+
+
+def haar_orthogonal(dim: int, seed: int) -> np.ndarray:
+    """Random orthogonal D x D matrix, Haar distributed, float64.
+
+    [turboquant_serve, "Architecture" / "Rotation": a fixed random orthogonal
+    matrix, seeded by head_dim]; [TorbuQuant, "Current Status": QR rotation].  The
+    pages name no generator: G is a D x D matrix of standard normals from numpy's
+    PCG64 generator seeded with ``seed``; with G = Q R its QR factorisation
+    (numpy.linalg.qr), the columns of Q are multiplied by the signs of diag(R), which
+    makes the factorisation unique and the result Haar distributed (Mezzadri, 2007).
+    """
+    g = np.random.default_rng(seed).standard_normal((dim, dim))
+    q, r = np.linalg.qr(g)
+    return q * np.sign(np.diag(r))[None, :]
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to bfloat16 (round to nearest even), returned as float64.
+    Through float32 (exact for the bf16 grid once the float32 value is rounded once)."""
+    f = np.asarray(x, dtype=np.float64).astype(np.float32)
+    b = f.view(np.uint32).astype(np.uint64)
+    lsb = (b >> np.uint64(16)) & np.uint64(1)
+    r = ((b + np.uint64(0x7FFF) + lsb) >> np.uint64(16)) << np.uint64(16)
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+@dataclass
+class DenseRotation:
+    """The dense rotation as both paths use it: R = hi + lo with hi = bf16(f) and
+    lo = bf16(f - hi), f = fp32(H) and H the float64 Haar matrix (f - hi is exact in
+    float32, so lo is a multiple of hi's float32 ulp and hi + lo is exact in float32).
+    R is within 2^-17 of H entry by entry (orthogonal to about 1e-5); the tensor-core
+    path multiplies by hi and by lo exactly."""
+
+    dim: int
+    seed: int
+    haar: np.ndarray    # float64 H
+    hi: np.ndarray      # float64 values on the bf16 grid
+    lo: np.ndarray
+
+    @property
+    def matrix(self) -> np.ndarray:
+        return self.hi + self.lo
+
+    def forward(self, x: np.ndarray) -> np.ndarray:
+        """y = R x along the last axis."""
+        return np.asarray(x, dtype=np.float64) @ self.matrix.T
+
+    def inverse(self, y: np.ndarray) -> np.ndarray:
+        """R^T y along the last axis (the transpose stands in for the inverse)."""
+        return np.asarray(y, dtype=np.float64) @ self.matrix
+
+
+def dense_rotation(dim: int, seed: int) -> DenseRotation:
+    h = haar_orthogonal(dim, seed)
+    f = h.astype(np.float32).astype(np.float64)
+    hi = bf16_round(f)
+    lo = bf16_round((f.astype(np.float32) - hi.astype(np.float32)).astype(np.float64))
+    return DenseRotation(dim=dim, seed=seed, haar=h, hi=hi, lo=lo)
+
+
+def rotate_forward(x: np.ndarray, rot) -> np.ndarray:
+    """R x with ``rot`` a DenseRotation, or the RHT when ``rot`` is its sign vector."""
+    return rot.forward(x) if isinstance(rot, DenseRotation) else rht_forward(x, rot)
+
+
+def rotate_inverse(y: np.ndarray, rot) -> np.ndarray:
+    """R^T y with ``rot`` a DenseRotation, or the RHT when ``rot`` is its sign vector."""
+    return rot.inverse(y) if isinstance(rot, DenseRotation) else rht_inverse(y, rot)
+
+
+# ---------------------------------------------------------------------------
 # Lloyd-Max codebooks
 # ---------------------------------------------------------------------------
 
@@ -290,6 +365,21 @@ def lloyd_max_beta(dim: int, bits: int, n_iter: int) -> Codebook:
 def lloyd_max_gaussian(bits: int, n_iter: int) -> Codebook:
     """Lloyd-Max codebook for N(0, 1)."""
     return lloyd_max(GaussianDensity(), bits, n_iter)
+
+
+def lloyd_max_gaussian_dim(dim: int, bits: int, n_iter: int) -> Codebook:
+    """Gaussian-approximation codebook of dimension D: the Lloyd-Max quantizer of
+    N(0, 1/D), the large-D limit of one coordinate of a uniform unit vector.
+
+    [TorbuQuant, "Current Status": Lloyd-Max codebooks, "exact Beta-sphere and
+    Gaussian approximation"].  The optimal quantizer of sigma X is sigma times that of
+    X (the two Lloyd-Max conditions are scale-equivariant), so this is the N(0, 1)
+    codebook with centroids and boundaries multiplied by 1/sqrt(D).
+    """
+    cb = lloyd_max_gaussian(bits, n_iter)
+    s = 1.0 / math.sqrt(dim)
+    return Codebook(centroids=cb.centroids * s, boundaries=cb.boundaries * s,
+                    iterations_run=cb.iterations_run, n_iter=cb.n_iter)
 
 
 def codebook_distortion(density, cb: Codebook) -> float:
@@ -429,6 +519,7 @@ def quantize_rows(x: np.ndarray, signs: np.ndarray, table: CodebookTable):
     [turboquant_pro, "How It Works": the L2 norm is preserved alongside the
     bits]:
       y = (1/sqrt(D)) H (s * x);  n = ||x||_2;  u = y / n;  idx = encode(u).
+    ``signs`` is the RHT sign vector, or a DenseRotation (then y = R x).
     A zero row stores n = 0 and encodes u = 0.  A row with a non-finite value
     stores all-zero indices and a quiet-NaN norm.
     """
@@ -438,7 +529,7 @@ def quantize_rows(x: np.ndarray, signs: np.ndarray, table: CodebookTable):
     rows = x.reshape(-1, d)
     nonfinite = ~np.all(np.isfinite(rows), axis=1)
     safe = np.where(nonfinite[:, None], 0.0, rows)
-    y = rht_forward(safe, signs)
+    y = rotate_forward(safe, signs)
     n = np.sqrt(np.sum(safe * safe, axis=1))
     u = np.where(n[:, None] > 0, y / np.where(n > 0, n, 1.0)[:, None], 0.0)
     idx = encode(u, table.boundaries)
@@ -482,7 +573,7 @@ def decode_region(region: np.ndarray, dim: int, bits: int):
 
 def quantize_append(pages: np.ndarray, slot_mapping: np.ndarray, k: np.ndarray,
                     v: np.ndarray, k_table: CodebookTable, v_table: CodebookTable,
-                    sign_seed: int) -> np.ndarray:
+                    sign_seed: int, rotation=None) -> np.ndarray:
     """Quantize every (token, KV head) row of K and V and store it in its slot.
 
     pages        uint8 [num_blocks, block_size, H_kv, slot_stride] (a copy is returned)
@@ -495,6 +586,7 @@ def quantize_append(pages: np.ndarray, slot_mapping: np.ndarray, k: np.ndarray,
     the "Store" stage]; [turboquant_serve, "Architecture": update() rotates,
     encodes and stores both k and v].  The same sign vector serves K and V and
     every head ([turboquant_serve, "Rotation": one fixed matrix per head_dim]).
+    ``rotation``: a DenseRotation to use instead of the RHT of ``sign_seed``.
     """
     pages = np.array(pages, dtype=np.uint8, copy=True)
     num_blocks, block_size, h_kv, stride = pages.shape
@@ -503,7 +595,7 @@ def quantize_append(pages: np.ndarray, slot_mapping: np.ndarray, k: np.ndarray,
     kb = region_bytes(d, k_table.bits)
     vb = region_bytes(d, v_table.bits)
     assert kb + vb <= stride
-    signs = rht_signs(d, sign_seed)
+    signs = rotation if rotation is not None else rht_signs(d, sign_seed)
     ki, kn, _, _ = quantize_rows(np.asarray(k, dtype=np.float64), signs, k_table)
     vi, vn, _, _ = quantize_rows(np.asarray(v, dtype=np.float64), signs, v_table)
     kreg = encode_region(ki, kn, k_table.bits)
@@ -527,14 +619,15 @@ def quantize_append(pages: np.ndarray, slot_mapping: np.ndarray, k: np.ndarray,
 
 def dequantize_rows(idx: np.ndarray, norm32: np.ndarray, table: CodebookTable,
                     signs: np.ndarray) -> np.ndarray:
-    """x_hat = norm * R^T c[idx] in float64 on the fp32 table values.
+    """x_hat = norm * R^T c[idx] in float64 on the fp32 table values (``signs``: the
+    RHT sign vector, or a DenseRotation).
 
     [turboquant_serve, "Architecture": unpack + Lloyd-Max decode -> restore
     magnitude -> multiply by R transposed]; [turboquant_pro, "How It Works":
     then invert].
     """
     c = np.asarray(table.centroids, dtype=np.float64)[np.asarray(idx)]
-    return np.asarray(norm32, dtype=np.float64)[..., None] * rht_inverse(c, signs)
+    return np.asarray(norm32, dtype=np.float64)[..., None] * rotate_inverse(c, signs)
 
 
 def gather_sequence(pages: np.ndarray, block_table_row: np.ndarray, seq_len: int):
@@ -551,7 +644,8 @@ def gather_sequence(pages: np.ndarray, block_table_row: np.ndarray, seq_len: int
 
 def paged_decode(q: np.ndarray, pages: np.ndarray, block_table: np.ndarray,
                  seq_lens: np.ndarray, k_table: CodebookTable,
-                 v_table: CodebookTable, sign_seed: int, scale: float) -> np.ndarray:
+                 v_table: CodebookTable, sign_seed: int, scale: float,
+                 rotation=None) -> np.ndarray:
     """One decode step over packed pages, by the plain definition.
 
     q [B, H_q, D]; returns o [B, H_q, D] float64.  For each sequence b and query
@@ -561,6 +655,7 @@ def paged_decode(q: np.ndarray, pages: np.ndarray, block_table: np.ndarray,
 
     [turboquant_serve, "Architecture": _decode then attention];
     [tq-kv, "Library API": scores from the compressed keys with a softmax scale].
+    ``rotation``: a DenseRotation to use instead of the RHT of ``sign_seed``.
     """
     q = np.asarray(q, dtype=np.float64)
     bsz, h_q, d = q.shape
@@ -568,7 +663,7 @@ def paged_decode(q: np.ndarray, pages: np.ndarray, block_table: np.ndarray,
     g = h_q // h_kv
     kb = region_bytes(d, k_table.bits)
     vb = region_bytes(d, v_table.bits)
-    signs = rht_signs(d, sign_seed)
+    signs = rotation if rotation is not None else rht_signs(d, sign_seed)
     out = np.zeros((bsz, h_q, d), dtype=np.float64)
     for b in range(bsz):
         n = int(seq_lens[b])
@@ -653,4 +748,61 @@ def paged_decode_rotated(q: np.ndarray, pages: np.ndarray, block_table: np.ndarr
                                             k_table, v_table, scale)
                      for s in range(0, n, step)]
             out[b, h] = rht_inverse(merge_partials(parts), signs)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Decode with an uncompressed hot window
+# ---------------------------------------------------------------------------
+
+
+def paged_decode_hot(q: np.ndarray, pages: np.ndarray, block_table: np.ndarray,
+                     seq_lens: np.ndarray, hot_k: np.ndarray, hot_v: np.ndarray,
+                     hot_lens: np.ndarray, k_table: CodebookTable, v_table: CodebookTable,
+                     sign_seed: int, scale: float, rotation=None) -> np.ndarray:
+    """One decode step over the packed pages plus an uncompressed hot window.
+
+    [turboquant_pro, "Fused CUDA decode": the fp16 hot window is merged with the
+    compressed tokens through the online softmax; "Streaming cache": recent tokens
+    stay uncompressed]; [tq-kv, "How It Works", "3-Fix for GGUF Models": the sink
+    tokens stay in FP16 and the current token is lossless].
+
+    q [B, H_q, D]; hot_k, hot_v [B, W, H_kv, D] (any real dtype, read exactly);
+    hot_lens [B]: sequence b attends to its seq_lens[b] packed tokens (dequantized
+    as in ``paged_decode``) and to hot tokens 0 .. hot_lens[b]-1, in one softmax over
+    all of them: s_t = scale <q, k_t>, o = sum_t softmax(s)_t v_t.  Which positions the
+    hot tokens held (the first few, the most recent) does not enter the result.  A
+    sequence with no tokens at all gives 0.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    bsz, h_q, d = q.shape
+    h_kv = pages.shape[2]
+    g = h_q // h_kv
+    kb = region_bytes(d, k_table.bits)
+    vb = region_bytes(d, v_table.bits)
+    signs = rht_signs(d, sign_seed)
+    if rotation is not None:
+        signs = rotation
+    hk = np.asarray(hot_k, dtype=np.float64)
+    hv = np.asarray(hot_v, dtype=np.float64)
+    out = np.zeros((bsz, h_q, d), dtype=np.float64)
+    for b in range(bsz):
+        n, w = int(seq_lens[b]), int(hot_lens[b])
+        if n + w == 0:
+            continue
+        keys = np.zeros((0, h_kv, d))
+        vals = np.zeros((0, h_kv, d))
+        if n > 0:
+            slots = gather_sequence(pages, block_table[b], n)
+            ki, kn = decode_region(slots[..., :kb], d, k_table.bits)
+            vi, vn = decode_region(slots[..., kb:kb + vb], d, v_table.bits)
+            keys = dequantize_rows(ki, kn, k_table, signs)
+            vals = dequantize_rows(vi, vn, v_table, signs)
+        keys = np.concatenate([keys, hk[b, :w]], axis=0)            # [n + w, H_kv, D]
+        vals = np.concatenate([vals, hv[b, :w]], axis=0)
+        for h in range(h_q):
+            kv = h // g
+            s = scale * (keys[:, kv, :] @ q[b, h])
+            p = np.exp(s - np.max(s))
+            out[b, h] = (p / np.sum(p)) @ vals[:, kv, :]
     return out

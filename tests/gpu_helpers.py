@@ -14,15 +14,16 @@ def require_gpu():
     import kv_cache_vector_append_b200 as tq  # noqa: F401  (fails loudly if the library is missing)
 
 
-def oracle_table(dim, bits):
-    return G.read_table(os.path.join(G.DEFAULT_OUT, G.table_filename(dim, bits)))
+def oracle_table(dim, bits, kind="beta"):
+    return G.read_table(os.path.join(G.DEFAULT_OUT, G.table_filename(dim, bits, kind)))
 
 
 def to_np_f64(t):
     return t.detach().to("cpu", torch.float32).numpy().astype(np.float64)
 
 
-def gpu_append(tq, wl, tokens=None, pages=None, slot_stride=None, fill=0, slot_mapping=None):
+def gpu_append(tq, wl, tokens=None, pages=None, slot_stride=None, fill=0, slot_mapping=None,
+               kind="beta"):
     """Run tq_quantize_append for `tokens` (indices into the workload) on cuda:0."""
     from kv_cache_vector_append_b200 import workloads as W
     dev = "cuda"
@@ -34,7 +35,7 @@ def gpu_append(tq, wl, tokens=None, pages=None, slot_stride=None, fill=0, slot_m
     v = wl.v[it].to(dev)
     sm = wl.slot_mapping[idx] if slot_mapping is None else slot_mapping
     sm = torch.from_numpy(np.ascontiguousarray(sm, dtype=np.int64)).to(dev)
-    cb = tq.load_codebooks(wl.spec.head_dim, wl.spec.k_bits, wl.spec.v_bits, dev)
+    cb = tq.load_codebooks(wl.spec.head_dim, wl.spec.k_bits, wl.spec.v_bits, dev, kind)
     tq.quantize_append(pages, sm, k, v, cb, wl.spec.sign_seed)
     torch.cuda.synchronize()
     return pages, cb

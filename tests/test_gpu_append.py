@@ -31,26 +31,26 @@ def _regions(pages_np, wl, tokens, kind):
     return rows[..., :kb] if kind == 0 else rows[..., kb:kb + vb]
 
 
-def _bit_exact_case(tq, wl, tokens=None):
+def _bit_exact_case(tq, wl, tokens=None, kind="beta"):
     """Packed bytes equal the oracle's packing of the GPU's own fp32 unit coords."""
-    pages, cb = gpu_append(tq, wl, tokens)
+    pages, cb = gpu_append(tq, wl, tokens, kind=kind)
     pages_np = pages.cpu().numpy()
     toks = np.arange(wl.k.shape[0]) if tokens is None else np.asarray(tokens)
     d = wl.spec.head_dim
-    for kind, (src, bits) in enumerate(((wl.k, wl.spec.k_bits), (wl.v, wl.spec.v_bits))):
+    for which, (src, bits) in enumerate(((wl.k, wl.spec.k_bits), (wl.v, wl.spec.v_bits))):
         x = src[torch.from_numpy(toks)].reshape(-1, d).cuda()
         u = torch.empty(x.shape, dtype=torch.float32, device="cuda")
         n = torch.empty(x.shape[0], dtype=torch.float32, device="cuda")
         tq.rotate_unit(u, n, x, wl.spec.sign_seed)
         u_np = u.cpu().numpy().astype(np.float64)
         n_np = n.cpu().numpy()
-        table = oracle_table(d, bits)
+        table = oracle_table(d, bits, kind)
         idx = O.encode(u_np, table.boundaries)
         expect = O.encode_region(idx, n_np, bits).reshape(len(toks), wl.spec.num_kv_heads, -1)
-        got = _regions(pages_np, wl, toks, kind)
+        got = _regions(pages_np, wl, toks, which)
         assert got.shape == expect.shape
         mism = np.nonzero(np.any(got != expect, axis=-1))
-        assert mism[0].size == 0, f"kind {kind}: {mism[0].size} rows differ, first {mism[0][:5]}"
+        assert mism[0].size == 0, f"region {which}: {mism[0].size} rows differ, first {mism[0][:5]}"
     return pages_np
 
 
@@ -136,20 +136,20 @@ def test_skipped_tokens_with_token_stores():
     assert np.array_equal(p[written], f[written])
 
 
-def _end_to_end(tq, wl, tokens=None, max_rows=None):
+def _end_to_end(tq, wl, tokens=None, max_rows=None, kind="beta"):
     """Oracle fp64 vs GPU: >= 99.99% identical codes, every mismatch within 1e-5 of a
     boundary; norms within 1e-6 relative."""
-    pages, _ = gpu_append(tq, wl, tokens)
+    pages, _ = gpu_append(tq, wl, tokens, kind=kind)
     pages_np = pages.cpu().numpy()
     toks = np.arange(wl.k.shape[0]) if tokens is None else np.asarray(tokens)
     d = wl.spec.head_dim
     signs = O.rht_signs(d, wl.spec.sign_seed)
     total = mism = 0
-    for kind, (src, bits) in enumerate(((wl.k, wl.spec.k_bits), (wl.v, wl.spec.v_bits))):
-        table = oracle_table(d, bits)
+    for which, (src, bits) in enumerate(((wl.k, wl.spec.k_bits), (wl.v, wl.spec.v_bits))):
+        table = oracle_table(d, bits, kind)
         x = to_np_f64(src[torch.from_numpy(toks)])
         ref_idx, ref_n, ref_u, _ = O.quantize_rows(x, signs, table)
-        got_idx, got_n = O.decode_region(_regions(pages_np, wl, toks, kind), d, bits)
+        got_idx, got_n = O.decode_region(_regions(pages_np, wl, toks, which), d, bits)
         np.testing.assert_allclose(got_n, ref_n, rtol=1e-6, atol=0)
         bad = got_idx != ref_idx
         total += bad.size
@@ -291,3 +291,12 @@ def test_norm_beyond_fp32_range_stores_inf():
     _, n = O.decode_region(_regions(p, wl, np.array([2]), 0)[0], 128, 4)
     assert np.all(np.isposinf(n))
     assert tq.get_device_error() == 0    # a finite row is not an error
+
+
+@pytest.mark.parametrize("d,kb,vb", [(128, 4, 2), (64, 3, 8), (256, 2, 4)])
+def test_gaussian_codebooks(d, kb, vb):
+    # The Gaussian-approximation tables (N(0, 1/D)) go through the same kernels.
+    tq = _tq()
+    wl = W.generate(_mini(d, kb, vb, h_kv=8, batch=2, seq=45, seed=d + 5))
+    _bit_exact_case(tq, wl, kind="gauss")
+    _end_to_end(tq, wl, kind="gauss")

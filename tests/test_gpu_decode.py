@@ -19,9 +19,9 @@ def _tq():
     return tq
 
 
-def _oracle_decode(wl, pages_np, seqs=None):
+def _oracle_decode(wl, pages_np, seqs=None, kind="beta"):
     d = wl.spec.head_dim
-    kt, vt = oracle_table(d, wl.spec.k_bits), oracle_table(d, wl.spec.v_bits)
+    kt, vt = oracle_table(d, wl.spec.k_bits, kind), oracle_table(d, wl.spec.v_bits, kind)
     seqs = np.arange(wl.spec.batch) if seqs is None else np.asarray(seqs)
     q = to_np_f64(wl.q)[seqs]
     return O.paged_decode(q, pages_np, wl.block_table[seqs], wl.seq_lens[seqs], kt, vt,
@@ -183,3 +183,75 @@ def test_extreme_key_and_value_magnitudes(k_scale, v_scale):
     wl.k = wl.k * k_scale
     wl.v = wl.v * v_scale
     _case(tq, wl)
+
+
+@pytest.mark.parametrize("kb,vb", [(4, 4), (3, 2), (8, 4)])
+def test_gaussian_codebooks(kb, vb):
+    tq = _tq()
+    lens = [260, 31]
+    wl = _with_lens(_spec(128, 16, 4, kb, vb, lens, seed=kb + vb), lens)
+    pages, cb = gpu_append(tq, wl, kind="gauss")
+    out = gpu_decode(tq, wl, pages, cb)
+    ref = _oracle_decode(wl, pages.cpu().numpy(), kind="gauss")
+    assert decode_error(to_np_f64(out), ref) <= TOL
+
+
+def _hot_case(tq, wl, w, hot_lens, hot_dtype, seed, k_scale=3.0):
+    """Append the workload, then decode with a hot window of w rows per sequence
+    (hot_lens[b] of them in use) and compare with the oracle's joint softmax."""
+    pages, cb = gpu_append(tq, wl)
+    b, h_kv, d = wl.spec.batch, wl.spec.num_kv_heads, wl.spec.head_dim
+    g = torch.Generator().manual_seed(seed)
+    dt = getattr(torch, hot_dtype)
+    hk = (torch.randn(b, w, h_kv, d, generator=g) * k_scale).to(dt)
+    hv = torch.randn(b, w, h_kv, d, generator=g).to(dt)
+    hl = np.asarray(hot_lens, dtype=np.int32)
+    q = wl.q.cuda()
+    out = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+    tq.paged_decode_hot(out, q, pages, torch.from_numpy(wl.block_table).cuda(),
+                        torch.from_numpy(wl.seq_lens).cuda(), hk.cuda(), hv.cuda(),
+                        torch.from_numpy(hl).cuda(), cb, wl.spec.sign_seed, wl.spec.scale)
+    torch.cuda.synchronize()
+    kt = oracle_table(d, wl.spec.k_bits)
+    vt = oracle_table(d, wl.spec.v_bits)
+    ref = O.paged_decode_hot(to_np_f64(wl.q), pages.cpu().numpy(), wl.block_table, wl.seq_lens,
+                             to_np_f64(hk), to_np_f64(hv), hl, kt, vt, wl.spec.sign_seed,
+                             wl.spec.scale)
+    return to_np_f64(out), ref
+
+
+@pytest.mark.parametrize("d,kb,vb,hot_dtype", [(128, 4, 4, "float16"), (64, 8, 2, "bfloat16"),
+                                               (128, 3, 2, "float32"), (256, 4, 2, "float16")])
+def test_hot_window_joins_the_softmax(d, kb, vb, hot_dtype):
+    # sequences: long packed + full window, packed-empty + window only, packed only,
+    # short packed + one hot token
+    tq = _tq()
+    lens = [300, 0, 17, 64]
+    wl = _with_lens(_spec(d, 8, 2, kb, vb, lens, seed=d + kb), lens)
+    got, ref = _hot_case(tq, wl, 24, [24, 5, 0, 1], hot_dtype, seed=kb)
+    assert np.all(np.isfinite(got))
+    assert decode_error(got, ref) <= TOL
+    assert tq.get_device_error() == 0
+
+
+def test_hot_window_dominant_and_long_split():
+    # hot keys with larger norms than the packed ones carry most of the weight; the
+    # packed part of the first sequence spans many CTAs
+    tq = _tq()
+    lens = [6000, 40, 0]
+    wl = _with_lens(_spec(128, 16, 4, 4, 2, lens, seed=77), lens)
+    got, ref = _hot_case(tq, wl, 64, [64, 64, 0], "float16", seed=5, k_scale=30.0)
+    assert decode_error(got, ref) <= TOL
+    assert np.all(got[2] == 0.0)                    # no tokens at all
+
+
+def test_hot_window_bad_length_flagged():
+    tq = _tq()
+    lens = [50, 50]
+    wl = _with_lens(_spec(128, 4, 1, 4, 4, lens, seed=3), lens)
+    tq.get_device_error()
+    got, _ = _hot_case(tq, wl, 8, [9, 3], "float16", seed=1)
+    assert tq.get_device_error() & tq.DEVERR_SEQLEN_RANGE
+    wl2 = _with_lens(_spec(128, 4, 1, 4, 4, lens, seed=3), lens)
+    got2, ref2 = _hot_case(tq, wl2, 8, [0, 3], "float16", seed=1)
+    assert decode_error(got[:1], ref2[:1]) <= TOL    # a bad length counts as 0 tokens

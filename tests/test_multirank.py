@@ -58,3 +58,29 @@ def test_reference_arm_other_ranks_print_nothing():
                        capture_output=True, text=True, env=env, timeout=300)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def test_gpus_flag_launches_one_rank_per_gpu():
+    # `bench.py --gpus 2` run directly starts two ranks through torch.distributed.run;
+    # in the reference arm rank 0 alone works and prints the one JSON line.
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--config", "0", "--steps", "1", "--warmup", "0"],
+                       capture_output=True, text=True, env=env, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    import json
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["n_gpus"] == 2
+    assert j["config"]["workload"] == "tiny-d128-k4v4"
+    assert j["cpu_baseline"]["cores"] >= 1
+
+
+def test_mismatched_world_size_is_refused():
+    import bench
+    env = dict(os.environ, WORLD_SIZE="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                        "--steps", "1"], capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode != 0

@@ -136,3 +136,89 @@ def test_gqa_grouping_is_contiguous():
         kv = h // g
         single = O.paged_decode(q[:, h:h + 1], pages[:, :, kv:kv + 1], bt, sl, kt, vt, 0, 0.125)
         np.testing.assert_allclose(out[:, h], single[:, 0], atol=1e-14)
+
+
+def _hot_window(bsz, w, h_kv, d, seed, dtype=np.float16):
+    rng = np.random.default_rng(seed)
+    hk = (rng.standard_normal((bsz, w, h_kv, d)) * 1.5).astype(dtype)
+    hv = rng.standard_normal((bsz, w, h_kv, d)).astype(dtype)
+    return hk, hv
+
+
+def test_hot_window_empty_equals_paged_decode():
+    d, h_kv, h_q = 64, 2, 6
+    lens = [40, 1, 0]
+    pages, bt, sl, kt, vt = _make_cache(d, h_kv, lens, 4, 2, seed=9)
+    q = np.random.default_rng(3).standard_normal((3, h_q, d))
+    hk, hv = _hot_window(3, 5, h_kv, d, 1)
+    got = O.paged_decode_hot(q, pages, bt, sl, hk, hv, np.zeros(3, int), kt, vt, 0, 0.125)
+    ref = O.paged_decode(q, pages, bt, sl, kt, vt, 0, 0.125)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-14)
+
+
+def test_hot_window_only_is_plain_attention():
+    # No packed tokens: textbook softmax attention over the fp16 rows, by loops.
+    d, h_kv, h_q, w = 64, 2, 4, 7
+    pages, bt, sl, kt, vt = _make_cache(d, h_kv, [0, 0], 4, 4, seed=2)
+    q = np.random.default_rng(5).standard_normal((2, h_q, d))
+    hk, hv = _hot_window(2, w, h_kv, d, 6)
+    hl = np.array([w, 3])
+    got = O.paged_decode_hot(q, pages, bt, sl, hk, hv, hl, kt, vt, 0, 0.125)
+    for b in range(2):
+        for h in range(h_q):
+            kv = h // (h_q // h_kv)
+            sc = [0.125 * sum(float(q[b, h, j]) * float(hk[b, t, kv, j]) for j in range(d))
+                  for t in range(hl[b])]
+            mx = max(sc)
+            e = [math.exp(x - mx) for x in sc]
+            ref = sum(ei * hv[b, t, kv].astype(np.float64) for t, ei in enumerate(e)) / sum(e)
+            np.testing.assert_allclose(got[b, h], ref, rtol=0, atol=1e-12)
+    assert np.all(O.paged_decode_hot(q, pages, bt, sl, hk, hv, np.zeros(2, int), kt, vt, 0,
+                                     0.125) == 0.0)
+
+
+def test_hot_window_joins_the_packed_softmax():
+    # One softmax over packed and hot tokens: brute force over the concatenated rows
+    # (packed rows dequantized through an explicit rotation matrix).
+    d, h_kv, h_q = 64, 1, 3
+    lens = [20, 33]
+    pages, bt, sl, kt, vt = _make_cache(d, h_kv, lens, 3, 2, seed=4)
+    q = np.random.default_rng(8).standard_normal((2, h_q, d)) * 2
+    hk, hv = _hot_window(2, 6, h_kv, d, 9)
+    hl = np.array([6, 2])
+    got = O.paged_decode_hot(q, pages, bt, sl, hk, hv, hl, kt, vt, 0, 0.125)
+    s = O.rht_signs(d, 0)
+    r = scipy.linalg.hadamard(d) * s[None, :] / math.sqrt(d)
+    kb, vb = O.region_bytes(d, 3), O.region_bytes(d, 2)
+    for b in range(2):
+        keys, vals = [], []
+        for t in range(lens[b]):
+            slot = pages[bt[b, t // 16], t % 16, 0]
+            ki, kn = O.decode_region(slot[:kb], d, 3)
+            vi, vn = O.decode_region(slot[kb:kb + vb], d, 2)
+            keys.append(float(kn) * (r.T @ kt.centroids.astype(np.float64)[ki]))
+            vals.append(float(vn) * (r.T @ vt.centroids.astype(np.float64)[vi]))
+        keys += [hk[b, t, 0].astype(np.float64) for t in range(hl[b])]
+        vals += [hv[b, t, 0].astype(np.float64) for t in range(hl[b])]
+        for h in range(h_q):
+            sc = [0.125 * float(np.dot(q[b, h], k_)) for k_ in keys]
+            mx = max(sc)
+            e = [math.exp(x - mx) for x in sc]
+            ref = sum(ei * v_ for ei, v_ in zip(e, vals)) / sum(e)
+            np.testing.assert_allclose(got[b, h], ref, rtol=0, atol=1e-12)
+    # and the split-KV merge of the packed part with the hot part equals it too
+    for b in range(2):
+        slots = O.gather_sequence(pages, bt[b], lens[b])
+        ki, kn = O.decode_region(slots[..., :kb], d, 3)
+        vi, vn = O.decode_region(slots[..., kb:kb + vb], d, 2)
+        for h in range(h_q):
+            qr = O.rht_forward(q[b, h], s)
+            m1, l1, o1 = O.rotated_domain_partial(qr, ki[:, 0], kn[:, 0], vi[:, 0], vn[:, 0], kt,
+                                                  vt, 0.125)
+            o1 = O.rht_inverse(o1, s)
+            sh = 0.125 * (hk[b, :hl[b], 0].astype(np.float64) @ q[b, h])
+            m2 = np.max(sh)
+            e2 = np.exp(sh - m2)
+            o2 = e2 @ hv[b, :hl[b], 0].astype(np.float64)
+            merged = O.merge_partials([(m1, l1, o1), (m2, np.sum(e2), o2)])
+            np.testing.assert_allclose(merged, got[b, h], rtol=0, atol=1e-12)

@@ -137,3 +137,42 @@ def test_stored_table_regenerates(d, bits):
     np.testing.assert_array_equal(t.centroids, r.centroids)
     np.testing.assert_array_equal(t.boundaries, r.boundaries)
     assert t.iterations_run == r.iterations_run
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_gaussian_tables_scale_to_max_1960(golden, d):
+    # sqrt(D) times the stored N(0, 1/D) table is the N(0, 1) Lloyd-Max quantizer: its
+    # distortion under N(0, 1) is Max's (1960) value.
+    dens = O.GaussianDensity()
+    for bits, value, tol in golden("gaussian_lloyd_max.txt"):
+        t = G.read_table(os.path.join(G.DEFAULT_OUT, G.table_filename(d, int(bits), "gauss")))
+        assert t.density_id == 1 and t.dim == d and t.bits == int(bits)
+        cb = O.Codebook(centroids=t.centroids.astype(np.float64) * math.sqrt(d),
+                        boundaries=t.boundaries.astype(np.float64) * math.sqrt(d),
+                        iterations_run=0, n_iter=0)
+        dist = O.codebook_distortion(dens, cb)
+        assert abs(dist - float(value)) <= float(tol) * float(value), (d, bits, dist)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_gaussian_approximation_approaches_beta_sphere(bits):
+    # One coordinate of a uniform unit vector tends to N(0, 1/D): the shipped Gaussian
+    # and exact tables, computed from two different densities, agree better as D grows.
+    gaps = []
+    for d in (64, 128, 256):
+        tb = G.read_table(os.path.join(G.DEFAULT_OUT, G.table_filename(d, bits, "beta")))
+        tg = G.read_table(os.path.join(G.DEFAULT_OUT, G.table_filename(d, bits, "gauss")))
+        c_b, c_g = tb.centroids.astype(np.float64), tg.centroids.astype(np.float64)
+        gaps.append(np.max(np.abs(c_b - c_g)) / np.max(np.abs(c_b)))
+        np.testing.assert_array_equal(tg.centroids, -tg.centroids[::-1])
+        assert np.all(np.diff(tg.boundaries) > 0)
+    assert gaps[0] > gaps[1] > gaps[2]
+    assert gaps[2] < 0.02
+
+
+@pytest.mark.parametrize("d,bits", [(128, 2), (64, 4)])
+def test_gaussian_table_is_the_fp32_of_the_oracle_codebook(d, bits):
+    t = G.read_table(os.path.join(G.DEFAULT_OUT, G.table_filename(d, bits, "gauss")))
+    cb = O.lloyd_max_gaussian_dim(d, bits, t.n_iter)
+    np.testing.assert_array_equal(t.centroids, cb.centroids.astype(np.float32))
+    np.testing.assert_array_equal(t.boundaries, cb.boundaries.astype(np.float32))

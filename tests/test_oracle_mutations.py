@@ -149,3 +149,23 @@ def test_mutation_region_big_endian_norm(monkeypatch):
         return idx, norm.astype(np.float32)
     monkeypatch.setattr(O, "decode_region", bad)
     _fails(TP.test_decode_region_reads_hand_built_regions, 2, 64)
+
+
+def test_mutation_hot_window_separate_softmax(monkeypatch):
+    # packed and hot tokens normalised separately, then averaged
+    orig = O.paged_decode_hot
+
+    def bad(q, pages, bt, sl, hk, hv, hl, kt, vt, seed, scale):
+        a = orig(q, pages, bt, sl, hk, hv, np.zeros_like(hl), kt, vt, seed, scale)
+        b = orig(q, pages, bt, np.zeros_like(sl), hk, hv, hl, kt, vt, seed, scale)
+        return 0.5 * (a + b)
+    monkeypatch.setattr(O, "paged_decode_hot", bad)
+    _fails(TA.test_hot_window_joins_the_packed_softmax)
+
+
+def test_mutation_haar_without_sign_fix(monkeypatch):
+    # numpy's QR factor used as it comes: the signs of R's diagonal left in R
+    def bad(dim, seed):
+        return np.linalg.qr(np.random.default_rng(seed).standard_normal((dim, dim)))[0]
+    monkeypatch.setattr(O, "haar_orthogonal", bad)
+    _fails(TR.test_haar_matrix_is_orthogonal_and_the_positive_diagonal_qr, 16)
