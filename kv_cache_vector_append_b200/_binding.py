@@ -74,33 +74,36 @@ def _load():
             "(there is no fallback implementation)")
     lib = ctypes.CDLL(_LIB_PATH)
     T, CB = TensorDesc, ctypes.POINTER(CodebooksDesc)
-    lib.tq_slot_bytes.argtypes = [ctypes.c_int32] * 3 + [ctypes.POINTER(ctypes.c_int32)]
-    lib.tq_quantize_append.argtypes = [T, T, T, T, CB, ctypes.c_uint64, ctypes.c_int32,
-                                       ctypes.c_int32, ctypes.c_void_p]
-    lib.tq_paged_decode.argtypes = [T, T, T, T, T, CB, ctypes.c_uint64, ctypes.c_float,
-                                    ctypes.c_void_p]
-    lib.tq_paged_decode_noalloc.argtypes = [T, T, T, T, T, CB, ctypes.c_uint64, ctypes.c_float,
-                                            ctypes.c_void_p]
-    lib.tq_paged_decode_hot.argtypes = [T, T, T, T, T, T, T, T, CB, ctypes.c_uint64,
-                                        ctypes.c_float, ctypes.c_void_p]
-    lib.tq_decode_workspace_size.argtypes = [ctypes.c_int32] * 6 + [ctypes.POINTER(ctypes.c_size_t)]
-    lib.tq_set_workspace.argtypes = [ctypes.c_void_p, ctypes.c_size_t]
-    lib.tq_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p]
-    lib.tq_rotate_unit.argtypes = [T, T, T, ctypes.c_uint64, ctypes.c_void_p]
-    lib.tq_decode_plan_probe.argtypes = [ctypes.c_int32] * 10 + [ctypes.c_uint32,
-                                                                 ctypes.POINTER(ctypes.c_int64)]
-    lib.tq_debug_inject_merge_stall.argtypes = [ctypes.c_int32, ctypes.c_int32]
     RT = ctypes.POINTER(RotationDesc)
-    lib.tq_quantize_append_dense.argtypes = [T, T, T, T, CB, RT, ctypes.c_int32, ctypes.c_int32,
-                                             ctypes.c_void_p]
-    lib.tq_paged_decode_dense.argtypes = [T, T, T, T, T, CB, RT, ctypes.c_float, ctypes.c_void_p]
-    lib.tq_rotate_unit_dense.argtypes = [T, T, T, RT, ctypes.c_void_p]
-    lib.tq_status_string.argtypes = [ctypes.c_int]
-    lib.tq_status_string.restype = ctypes.c_char_p
+    sig = {
+        "tq_slot_bytes": [ctypes.c_int32] * 3 + [ctypes.POINTER(ctypes.c_int32)],
+        "tq_quantize_append": [T, T, T, T, CB, ctypes.c_uint64, ctypes.c_int32, ctypes.c_int32,
+                               ctypes.c_void_p],
+        "tq_paged_decode": [T, T, T, T, T, CB, ctypes.c_uint64, ctypes.c_float, ctypes.c_void_p],
+        "tq_paged_decode_noalloc": [T, T, T, T, T, CB, ctypes.c_uint64, ctypes.c_float,
+                                    ctypes.c_void_p],
+        "tq_paged_decode_hot": [T, T, T, T, T, T, T, T, CB, ctypes.c_uint64, ctypes.c_float,
+                                ctypes.c_void_p],
+        "tq_decode_workspace_size": [ctypes.c_int32] * 6 + [ctypes.POINTER(ctypes.c_size_t)],
+        "tq_set_workspace": [ctypes.c_void_p, ctypes.c_size_t],
+        "tq_get_device_error": [ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p],
+        "tq_rotate_unit": [T, T, T, ctypes.c_uint64, ctypes.c_void_p],
+        "tq_decode_plan_probe": [ctypes.c_int32] * 10 + [ctypes.c_uint32,
+                                                         ctypes.POINTER(ctypes.c_int64)],
+        "tq_debug_inject_merge_stall": [ctypes.c_int32, ctypes.c_int32],
+        "tq_quantize_append_dense": [T, T, T, T, CB, RT, ctypes.c_int32, ctypes.c_int32,
+                                     ctypes.c_void_p],
+        "tq_paged_decode_dense": [T, T, T, T, T, CB, RT, ctypes.c_float, ctypes.c_void_p],
+        "tq_rotate_unit_dense": [T, T, T, RT, ctypes.c_void_p],
+        "tq_status_string": [ctypes.c_int],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name, None)     # every declared symbol is checked by the ABI test
+        if fn is None:
+            continue
+        fn.argtypes = args
+        fn.restype = ctypes.c_char_p if name == "tq_status_string" else ctypes.c_int
     lib.tq_version.restype = ctypes.c_char_p
-    for name in EXPORTED:
-        if name not in ("tq_status_string", "tq_version"):
-            getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
 

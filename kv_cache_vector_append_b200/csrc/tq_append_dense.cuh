@@ -374,6 +374,12 @@ append_dense_kernel(DenseAppendParams p, const __grid_constant__ DenseAppendMaps
       }
       dst_s[tid] = off;
     }
+    // the staged rows are read below: every thread waits for the tile's copies (thread 0
+    // has already waited for them before issuing the MMAs)
+    if (tid != 0 && !mbar_wait(&bars[b], full_parity, p.wait_ms)) {
+      report_error(p.err, TQ_DEVERR_TIMEOUT);
+      flags[2] = 1;
+    }
     // the row's norm from the staged input (plain fp32 sum of squares in k order)
     const bool active = !(p.export_mode && kind == 1);
     const uint8_t* xblk = st + kind * SM::KIND;

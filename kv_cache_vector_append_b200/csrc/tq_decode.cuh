@@ -127,14 +127,19 @@ struct DecodeParams {
   const int32_t* hot_lens;
 };
 
-// Attention partial of query head h of sequence b over its hot-window tokens, computed
-// by one warp in the original (unrotated) domain: lane l handles coordinates
-// l E .. l E + E - 1.  With s_t = scale log2(e) <q, k_t> (fp32): M = max_t s_t,
-// L = sum_t 2^(s_t - M), o = sum_t 2^(s_t - M) v_t (this lane's coordinates).  A
-// hot_lens entry outside [0, W] raises TQ_DEVERR_SEQLEN_RANGE and counts as 0 tokens.
-template <int D>
-__device__ __forceinline__ void hot_partial(const DecodeParams& p, int b, int h, int lane,
-                                            float& M, float& L, float (&o)[D / 32]);
+// Arguments of the hot-window partial (a copy of the fields it reads).
+struct HotArgs {
+  const void* hot_k;
+  const void* hot_v;
+  int64_t hot_bstride, hot_tstride, hot_hstride;
+  int32_t hot_dtype, hot_cap;
+  const int32_t* hot_lens;
+  const void* q;
+  int64_t q_bstride, q_hstride;
+  int32_t q_dtype, group;
+  float scale_log2;
+  unsigned int* err;
+};
 
 // Step range of CTA c out of C over S steps: [floor(c S / C), floor((c+1) S / C)).
 __host__ __device__ __forceinline__ int64_t cta_begin(int64_t c, int64_t S, int64_t C) {
@@ -381,25 +386,29 @@ __device__ __forceinline__ void warp_fwht(float (&x)[E], int lane) {
 
 // R[r][lane E + i] for i < E (hi + lo, exact in fp32), E = D / 32 consecutive entries.
 template <int E>
-__device__ __forceinline__ void rot_row_part(const DecodeParams& p, int D, int r, int lane,
-                                             float (&v)[E]) {
+__device__ __forceinline__ void rot_row_part(const uint16_t* hi, const uint16_t* lo, int r,
+                                             int lane, float (&v)[E]) {
+  constexpr int D = 32 * E;
   const int64_t o = (int64_t)r * D + lane * E;
 #pragma unroll
   for (int i = 0; i < E; ++i)
-    v[i] = __uint_as_float((uint32_t)p.rot_hi[o + i] << 16) +
-           __uint_as_float((uint32_t)p.rot_lo[o + i] << 16);
+    v[i] = __uint_as_float((uint32_t)hi[o + i] << 16) + __uint_as_float((uint32_t)lo[o + i] << 16);
 }
 
-// y = R x for one warp: lane l holds x[l E + i] on entry and y[l E + i] on exit.  Output c
-// is the warp sum of the lanes' partial dot products with row c of R (fp32), kept in
-// `sc` (D floats of this warp's shared scratch).
+// sc[0 .. D) <- R sc[0 .. D) for one warp (sc: this warp's shared scratch).  Output c is
+// the warp sum of the lanes' partial dot products with row c of R (fp32).  Out of line,
+// so that it leaves the register allocation of the caller's step loop alone.
 template <int E>
-__device__ __forceinline__ void dense_forward(const DecodeParams& p, float (&x)[E], int lane,
-                                              float* sc) {
+__device__ __noinline__ void dense_forward(const uint16_t* hi, const uint16_t* lo, float* sc,
+                                           int lane) {
   constexpr int D = 32 * E;
+  float x[E];
+#pragma unroll
+  for (int i = 0; i < E; ++i) x[i] = sc[lane * E + i];
+  __syncwarp();
   for (int c = 0; c < D; ++c) {
     float r[E];
-    rot_row_part<E>(p, D, c, lane, r);
+    rot_row_part<E>(hi, lo, c, lane, r);
     float part = 0.f;
 #pragma unroll
     for (int i = 0; i < E; ++i) part = fmaf(r[i], x[i], part);
@@ -408,30 +417,28 @@ __device__ __forceinline__ void dense_forward(const DecodeParams& p, float (&x)[
     if (lane == 0) sc[c] = part;
   }
   __syncwarp();
-#pragma unroll
-  for (int i = 0; i < E; ++i) x[i] = sc[lane * E + i];
-  __syncwarp();
 }
 
-// o = R^T a for one warp: lane l holds a[l E + i] on entry and o[l E + i] on exit;
-// o_c = sum_j R[j][c] a_j accumulated in fp32 over j = 0 .. D-1.
+// sc[0 .. D) <- R^T sc[0 .. D) for one warp: o_c = sum_j R[j][c] a_j in fp32 over
+// j = 0 .. D-1 (out of line, as dense_forward).
 template <int E>
-__device__ __forceinline__ void dense_inverse(const DecodeParams& p, float (&a)[E], int lane,
-                                              float* sc) {
+__device__ __noinline__ void dense_inverse(const uint16_t* hi, const uint16_t* lo, float* sc,
+                                           int lane) {
   constexpr int D = 32 * E;
-  __syncwarp();
-#pragma unroll
-  for (int i = 0; i < E; ++i) sc[lane * E + i] = a[i];
-  __syncwarp();
+  float a[E];
 #pragma unroll
   for (int i = 0; i < E; ++i) a[i] = 0.f;
+  __syncwarp();
   for (int j = 0; j < D; ++j) {
     float r[E];
-    rot_row_part<E>(p, D, j, lane, r);
+    rot_row_part<E>(hi, lo, j, lane, r);
     const float aj = sc[j];
 #pragma unroll
     for (int i = 0; i < E; ++i) a[i] = fmaf(r[i], aj, a[i]);
   }
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < E; ++i) sc[lane * E + i] = a[i];
   __syncwarp();
 }
 
@@ -441,46 +448,57 @@ __device__ __forceinline__ float load_as_f32(const void* base, int64_t i, int32_
   return __half2float(((const __half*)base)[i]);
 }
 
+// Attention partial of query head h of sequence b over its hot-window tokens, computed
+// by one warp in the original (unrotated) domain: lane l handles coordinates
+// l E .. l E + E - 1.  With s_t = scale log2(e) <q, k_t> (fp32): M = max_t s_t,
+// L = sum_t 2^(s_t - M), o = sum_t 2^(s_t - M) v_t, written to sc[0] = M, sc[1] = L,
+// sc[2 + c] = o_c (this warp's shared scratch).  A hot_lens entry outside [0, W] raises
+// TQ_DEVERR_SEQLEN_RANGE and counts as 0 tokens.  Out of line, as dense_forward.
 template <int D>
-__device__ __forceinline__ void hot_partial(const DecodeParams& p, int b, int h, int lane,
-                                            float& M, float& L, float (&o)[D / 32]) {
+__device__ __noinline__ void hot_partial(const HotArgs a, int b, int h, int lane, float* sc) {
   constexpr int E = D / 32;
-  M = -INFINITY;
-  L = 0.f;
+  float M = -INFINITY, L = 0.f, o[E];
 #pragma unroll
   for (int i = 0; i < E; ++i) o[i] = 0.f;
-  int n = p.hot_lens[b];
-  if (n < 0 || n > p.hot_cap) {
-    if (lane == 0) report_error(p.err, TQ_DEVERR_SEQLEN_RANGE);
+  int n = a.hot_lens[b];
+  if (n < 0 || n > a.hot_cap) {
+    if (lane == 0) report_error(a.err, TQ_DEVERR_SEQLEN_RANGE);
     n = 0;
   }
-  if (n == 0) return;
   float qv[E];
-  const int64_t qo = (int64_t)b * p.q_bstride + (int64_t)h * p.q_hstride + lane * E;
+  const int64_t qo = (int64_t)b * a.q_bstride + (int64_t)h * a.q_hstride + lane * E;
 #pragma unroll
-  for (int i = 0; i < E; ++i) qv[i] = load_as_f32(p.q, qo + i, p.q_dtype);
-  const int64_t base = (int64_t)b * p.hot_bstride + (int64_t)(h / p.group) * p.hot_hstride +
+  for (int i = 0; i < E; ++i) qv[i] = load_as_f32(a.q, qo + i, a.q_dtype);
+  const int64_t base = (int64_t)b * a.hot_bstride + (int64_t)(h / a.group) * a.hot_hstride +
                        lane * E;
   for (int t = 0; t < n; ++t) {
-    const int64_t off = base + (int64_t)t * p.hot_tstride;
+    const int64_t off = base + (int64_t)t * a.hot_tstride;
     float dot = 0.f;
 #pragma unroll
-    for (int i = 0; i < E; ++i) dot = fmaf(qv[i], load_as_f32(p.hot_k, off + i, p.hot_dtype), dot);
+    for (int i = 0; i < E; ++i) dot = fmaf(qv[i], load_as_f32(a.hot_k, off + i, a.hot_dtype), dot);
 #pragma unroll
     for (int m = 16; m > 0; m >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, m);
-    const float sc = dot * p.scale_log2;
-    if (sc > M) {
-      const float f = M == -INFINITY ? 0.f : exp2f(M - sc);
+    const float sc_t = dot * a.scale_log2;
+    if (sc_t > M) {
+      const float f = M == -INFINITY ? 0.f : exp2f(M - sc_t);
       L *= f;
 #pragma unroll
       for (int i = 0; i < E; ++i) o[i] *= f;
-      M = sc;
+      M = sc_t;
     }
-    const float w = exp2f(sc - M);
+    const float w = exp2f(sc_t - M);
     L += w;
 #pragma unroll
-    for (int i = 0; i < E; ++i) o[i] = fmaf(w, load_as_f32(p.hot_v, off + i, p.hot_dtype), o[i]);
+    for (int i = 0; i < E; ++i) o[i] = fmaf(w, load_as_f32(a.hot_v, off + i, a.hot_dtype), o[i]);
   }
+  __syncwarp();
+  if (lane == 0) {
+    sc[0] = M;
+    sc[1] = L;
+  }
+#pragma unroll
+  for (int i = 0; i < E; ++i) sc[2 + lane * E + i] = o[i];
+  __syncwarp();
 }
 
 __device__ __forceinline__ void store_from_f32(void* base, int64_t i, int32_t dtype, float v) {
@@ -493,7 +511,9 @@ __device__ __forceinline__ void store_from_f32(void* base, int64_t i, int32_t dt
 // area [full mbarriers | release counters | present masks | q' (H_q x D fp16) | |q'|
 // scales | step prefix sums | block ids | scan scratch | flag | merge partials |
 // record positions].
-template <int D, int KB, int VB, int NH, int MAXW>
+// EXT: the instantiation that also serves the hot window and the dense rotation (runtime
+// choices, both outside the step loop); the plain one carries none of their code.
+template <int D, int KB, int VB, int NH, int MAXW, bool EXT>
 __global__ void __launch_bounds__(MAXW * 32, 1)
 decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   using C = DecodeCfg<D, KB, VB>;
@@ -531,6 +551,25 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gid = lane >> 2, tig = lane & 3;
+  auto hot_args = [&]() {
+    HotArgs a;
+    a.hot_k = p.hot_k;
+    a.hot_v = p.hot_v;
+    a.hot_bstride = p.hot_bstride;
+    a.hot_tstride = p.hot_tstride;
+    a.hot_hstride = p.hot_hstride;
+    a.hot_dtype = p.hot_dtype;
+    a.hot_cap = p.hot_cap;
+    a.hot_lens = p.hot_lens;
+    a.q = p.q;
+    a.q_bstride = p.q_bstride;
+    a.q_hstride = p.q_hstride;
+    a.q_dtype = p.q_dtype;
+    a.group = p.group;
+    a.scale_log2 = p.scale_log2;
+    a.err = p.err;
+    return a;
+  };
   const int nthreads = blockDim.x;
   const int nwarps = nthreads >> 5;                    // = h_kv * wph
   const int wph = p.wph;                               // blocks per pipeline step
@@ -588,18 +627,21 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   // alone (one warp per query head)
   for (int b = blockIdx.x; b < B; b += gridDim.x) {
     if (prefix[b + 1] != prefix[b]) continue;
-    if (p.hot_k == nullptr) {
+    if (!EXT || p.hot_k == nullptr) {
       for (int i = tid; i < p.h_q * D; i += nthreads)
         store_from_f32(p.out, (int64_t)b * p.o_bstride + (int64_t)(i / D) * p.o_hstride + i % D,
                        p.out_dtype, 0.f);
     } else {
+      float* sc = scratch + warp * (D + 2);
       for (int h = warp; h < p.h_q; h += nwarps) {
-        float M, L, o[E];
-        hot_partial<D>(p, b, h, lane, M, L, o);
+        hot_partial<D>(hot_args(), b, h, lane, sc);
+        const float L = sc[1];
         const float inv = L > 0.f ? 1.0f / L : 0.f;
         const int64_t ob = (int64_t)b * p.o_bstride + (int64_t)h * p.o_hstride + lane * E;
 #pragma unroll
-        for (int i = 0; i < E; ++i) store_from_f32(p.out, ob + i, p.out_dtype, o[i] * inv);
+        for (int i = 0; i < E; ++i)
+          store_from_f32(p.out, ob + i, p.out_dtype, sc[2 + lane * E + i] * inv);
+        __syncwarp();
       }
     }
   }
@@ -722,8 +764,15 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
 #pragma unroll
     for (int i = 0; i < E; ++i) sg[i] = sign_mask_at(p.sign_seed, lane * E + i);
     auto rotate_head = [&](int h, float (&xq)[E]) {
-      if (p.rot_hi != nullptr) {
-        dense_forward<E>(p, xq, lane, scratch + warp * (D + 2));
+      if (EXT && p.rot_hi != nullptr) {
+        float* sc = scratch + warp * (D + 2);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < E; ++i) sc[lane * E + i] = xq[i];
+        dense_forward<E>(p.rot_hi, p.rot_lo, sc, lane);
+#pragma unroll
+        for (int i = 0; i < E; ++i) xq[i] = sc[lane * E + i];
+        __syncwarp();
       } else {
 #pragma unroll
         for (int i = 0; i < E; ++i) xq[i] = __uint_as_float(__float_as_uint(xq[i]) ^ sg[i]);
@@ -974,8 +1023,15 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
         const int64_t ob = (int64_t)b * p.o_bstride + (int64_t)h * p.o_hstride + lane * E;
         // o = R^T a: the dense rotation, or the FWHT, 1/sqrt(D) and the sign flips
         auto inverse_rotate = [&](float (&a)[E]) {
-          if (p.rot_hi != nullptr) {
-            dense_inverse<E>(p, a, lane, scratch + warp * (D + 2));
+          if (EXT && p.rot_hi != nullptr) {
+            float* sc = scratch + warp * (D + 2);
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < E; ++i) sc[lane * E + i] = a[i];
+            dense_inverse<E>(p.rot_hi, p.rot_lo, sc, lane);
+#pragma unroll
+            for (int i = 0; i < E; ++i) a[i] = sc[lane * E + i];
+            __syncwarp();
           } else {
             warp_fwht<E>(a, lane);
 #pragma unroll
@@ -983,7 +1039,7 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
               a[i] = __uint_as_float(__float_as_uint(a[i] * inv_sqrt_dim<D>()) ^ sg[i]);
           }
         };
-        if (p.hot_k == nullptr) {
+        if (!EXT || p.hot_k == nullptr) {
           const float inv = L > 0.f ? 1.0f / L : 0.f;
 #pragma unroll
           for (int i = 0; i < E; ++i) acc_o[i] *= inv;
@@ -995,8 +1051,13 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
           // the hot window's partial: rescale both to the larger reference and divide
           // by the joint sum
           inverse_rotate(acc_o);
-          float Mh, Lh, oh[E];
-          hot_partial<D>(p, b, h, lane, Mh, Lh, oh);
+          float* sc = scratch + warp * (D + 2);
+          hot_partial<D>(hot_args(), b, h, lane, sc);
+          const float Mh = sc[0], Lh = sc[1];
+          float oh[E];
+#pragma unroll
+          for (int i = 0; i < E; ++i) oh[i] = sc[2 + lane * E + i];
+          __syncwarp();
           const float Mt = fmaxf(Mx, Mh);
           const float f1 = Mx == -INFINITY ? 0.f : exp2f(Mx - Mt);
           const float f2 = Mh == -INFINITY ? 0.f : exp2f(Mh - Mt);
