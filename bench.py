@@ -491,6 +491,72 @@ def extra_config_legs(configs, dev, steps, warmup, peak):
     return res
 
 
+def variant_legs(wl, x, dev, steps, warmup, peak):
+    """The survey's next rows on the main workload, each in its own timed region:
+    quantize-append and decode with the dense (QR) rotation (tcgen05 GEMM), and the
+    decode with a 64-token uncompressed hot window per sequence (bf16)."""
+    import torch
+    import kv_cache_vector_append_b200 as tq
+    spec = wl.spec
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    ev = lambda: torch.cuda.Event(enable_timing=True)   # noqa: E731
+    if spec.head_dim in (64, 128):
+        rot = tq.load_rotation(spec.head_dim, dev)
+
+        def dense_step():
+            tq.quantize_append_dense(x["pages"], x["sm"], x["k"], x["v"], x["cb"], rot, stream)
+            tq.paged_decode_dense(x["out"], x["q"], x["pages"], x["bt"], x["sl"], x["cb"], rot,
+                                  spec.scale, stream)
+        for _ in range(max(warmup, 3)):
+            dense_step()
+        torch.cuda.synchronize(dev)
+        e = [[ev() for _ in range(3)] for _ in range(steps)]
+        for i in range(steps):
+            e[i][0].record(stream)
+            tq.quantize_append_dense(x["pages"], x["sm"], x["k"], x["v"], x["cb"], rot, stream)
+            e[i][1].record(stream)
+            tq.paged_decode_dense(x["out"], x["q"], x["pages"], x["bt"], x["sl"], x["cb"], rot,
+                                  spec.scale, stream)
+            e[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+        app = float(np.mean([a.elapsed_time(b) for a, b, _ in e]))
+        dec = float(np.mean([b.elapsed_time(c) for _, b, c in e]))
+        leg = leg_summary(wl, app, dec, peak)
+        n_rows = len(wl.step_tokens) * spec.num_kv_heads
+        leg["append"]["tensor_tflops"] = 2 * 2 * n_rows * 2 * spec.head_dim ** 2 / (app * 1e-3) / 1e12
+        res["dense_rotation"] = leg
+        # the RHT pages again for the rest of the run
+        tq.quantize_append(x["pages"], x["sm"], x["k"], x["v"], x["cb"], spec.sign_seed, stream)
+    w = 64
+    g = torch.Generator().manual_seed(7)
+    hk = torch.randn(spec.batch, w, spec.num_kv_heads, spec.head_dim, generator=g).to(
+        torch.bfloat16).to(dev)
+    hv = torch.randn(spec.batch, w, spec.num_kv_heads, spec.head_dim, generator=g).to(
+        torch.bfloat16).to(dev)
+    hl = torch.full((spec.batch,), w, dtype=torch.int32, device=dev)
+    for _ in range(max(warmup, 3)):
+        tq.paged_decode_hot(x["out"], x["q"], x["pages"], x["bt"], x["sl"], hk, hv, hl, x["cb"],
+                            spec.sign_seed, spec.scale, stream)
+    torch.cuda.synchronize(dev)
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for _ in range(steps):
+        tq.paged_decode_hot(x["out"], x["q"], x["pages"], x["bt"], x["sl"], hk, hv, hl, x["cb"],
+                            spec.sign_seed, spec.scale, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    dec = e0.elapsed_time(e1) / steps
+    d_bytes, d_packed = decode_bytes(spec, wl.seq_lens)
+    hot_bytes = 2 * spec.batch * w * spec.num_kv_heads * spec.head_dim * 2
+    res["hot_window"] = {"window_tokens": w, "ms": dec,
+                         "gbs": (d_bytes + hot_bytes) / (dec * 1e-3) / 1e9,
+                         "frac_of_peak": (d_bytes + hot_bytes) / (dec * 1e-3) / 1e9 / peak}
+    if tq.get_device_error(stream):
+        raise RuntimeError("device error during the variant legs")
+    return res
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -606,6 +672,9 @@ def run_gpu(args):
                "ms_per_step": e2e_ms / args.steps}
 
     peak, peak_kind = measured_peaks()
+    variants = None
+    if not args.no_extra_configs:
+        variants = variant_legs(wl, x, dev, args.steps, args.warmup, peak)
     extra = None
     if not args.no_extra_configs and args.config == 2 and not args.batch:
         tq.set_workspace(None)
@@ -642,9 +711,13 @@ def run_gpu(args):
                             "achieved": legs["decode"]["gbs"], "peak": peak, "unit": "GB/s",
                             "frac": legs["decode"]["gbs"] / peak,
                             "traffic": ncu_traffic("decode_kernel", spec.name)},
-        "gpu_launches": 2 * args.steps,   # append_kernel + decode_kernel
+        # append_kernel (fast path) + its redo launch (returns at once unless flagged) +
+        # decode_kernel, per step
+        "gpu_launches": 3 * args.steps,
         "clocks": clk.summary(),
     }
+    if variants:
+        line["variants"] = variants
     if extra:
         line["other_configs"] = extra
     if e2e is not None:

@@ -209,6 +209,30 @@ TQ_API tq_status tq_paged_decode(tq_tensor out, tq_tensor q, tq_tensor pages,
                           const tq_codebooks* cb, uint64_t sign_seed, float scale,
                           void* stream);
 
+/* The QJL residual sketch of the keys (tq-kv, "How It Works" step [5]: SRHT QJL error
+ * correction; TorbuQuant, "Current Status": QJL residual).  After the Lloyd-Max code,
+ * each K row also stores the 1-bit sketch of its rotated-domain residual r = u - c[idx]:
+ * z_j = [(S r)_j >= 0] with S = (1/sqrt(D)) H diag(s2), a second randomized Hadamard
+ * transform whose signs s2 come from SplitMix64 seeded with qjl_seed, and the fp32
+ * gamma = ||r||.  K region = [packed codes | fp32 norm | D sign bits, LSB-first | fp32
+ * gamma]; the V region follows unchanged.  Slot bytes: tq_slot_bytes_qjl (the pages'
+ * slot_stride is at least that and a multiple of 8, so it may need padding).
+ * Supported: D = 128 or 256 (the append), K widths 2, 3, 4 (the decode).  Same
+ * arguments, layouts and errors as tq_quantize_append / tq_paged_decode otherwise; a
+ * non-finite K row stores z = 0 and gamma = 0. */
+TQ_API tq_status tq_slot_bytes_qjl(int32_t dim, int32_t k_bits, int32_t v_bits, int32_t* out);
+TQ_API tq_status tq_quantize_append_qjl(tq_tensor pages, tq_tensor slot_mapping, tq_tensor k,
+                                        tq_tensor v, const tq_codebooks* cb, uint64_t sign_seed,
+                                        uint64_t qjl_seed, int32_t k_bits, int32_t v_bits,
+                                        void* stream);
+/* Decode over slots written by tq_quantize_append_qjl: each key is scored with its QJL
+ * correction, scale nK (<R q, c[idx]> + gamma sqrt(pi/2)/sqrt(D) <S R q, 2z - 1>), the
+ * second term as one more mma per k-step on +-1 fragments built from the sign bits. */
+TQ_API tq_status tq_paged_decode_qjl(tq_tensor out, tq_tensor q, tq_tensor pages,
+                                     tq_tensor block_table, tq_tensor seq_lens,
+                                     const tq_codebooks* cb, uint64_t sign_seed,
+                                     uint64_t qjl_seed, float scale, void* stream);
+
 /* Paged decode with an uncompressed hot window (turboquant_pro 1.4.2, "Fused CUDA
  * decode": the fp16 hot window is merged through the online softmax, and "Streaming
  * cache"; tq-kv, "How It Works", "3-Fix for GGUF Models": sink tokens stay FP16, the

@@ -13,6 +13,8 @@ Public API (names follow the C entry points):
     paged_decode(out, q, pages, block_table, seq_lens, codebooks, sign_seed, scale, stream=None)
     paged_decode_hot(out, q, pages, block_table, seq_lens, hot_k, hot_v, hot_lens, ...)
                                 # same, plus an uncompressed hot window (sinks, recent tokens)
+    quantize_append_qjl(...), paged_decode_qjl(...), slot_bytes_qjl(D, kb, vb)
+                                # keys with the QJL residual sketch
     paged_decode_noalloc(...)   # same, with the library's fixed scratch (no allocation)
     rotate_unit(u, norm, x, sign_seed, stream=None)       # test export of the rotation
     load_rotation(D, device) -> Rotation                  # dense (QR) rotation table
@@ -43,6 +45,9 @@ from ._binding import (  # noqa: F401
     rotate_unit_dense,
     paged_decode,
     paged_decode_hot,
+    paged_decode_qjl,
+    quantize_append_qjl,
+    slot_bytes_qjl,
     paged_decode_noalloc,
     quantize_append,
     rotate_unit,

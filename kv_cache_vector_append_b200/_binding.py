@@ -30,6 +30,7 @@ EXPORTED = ("tq_slot_bytes", "tq_quantize_append", "tq_paged_decode", "tq_paged_
             "tq_decode_workspace_size", "tq_set_workspace", "tq_get_device_error",
             "tq_rotate_unit", "tq_decode_plan_probe", "tq_debug_inject_merge_stall",
             "tq_quantize_append_dense", "tq_paged_decode_dense", "tq_rotate_unit_dense",
+            "tq_slot_bytes_qjl", "tq_quantize_append_qjl", "tq_paged_decode_qjl",
             "tq_status_string", "tq_version")
 
 
@@ -95,6 +96,11 @@ def _load():
                                      ctypes.c_void_p],
         "tq_paged_decode_dense": [T, T, T, T, T, CB, RT, ctypes.c_float, ctypes.c_void_p],
         "tq_rotate_unit_dense": [T, T, T, RT, ctypes.c_void_p],
+        "tq_slot_bytes_qjl": [ctypes.c_int32] * 3 + [ctypes.POINTER(ctypes.c_int32)],
+        "tq_quantize_append_qjl": [T, T, T, T, CB, ctypes.c_uint64, ctypes.c_uint64,
+                                   ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p],
+        "tq_paged_decode_qjl": [T, T, T, T, T, CB, ctypes.c_uint64, ctypes.c_uint64,
+                                ctypes.c_float, ctypes.c_void_p],
         "tq_status_string": [ctypes.c_int],
     }
     for name, args in sig.items():
@@ -338,6 +344,34 @@ def rotate_unit_dense(u, norm, x, rotation: Rotation, stream=None) -> None:
     _check(_load().tq_rotate_unit_dense(_desc(u), _desc(norm), _desc(x),
                                         ctypes.byref(rotation.desc), st),
            "tq_rotate_unit_dense")
+
+
+def slot_bytes_qjl(dim: int, k_bits: int, v_bits: int) -> int:
+    out = ctypes.c_int32()
+    _check(_load().tq_slot_bytes_qjl(dim, k_bits, v_bits, ctypes.byref(out)), "tq_slot_bytes_qjl")
+    return out.value
+
+
+def quantize_append_qjl(pages, slot_mapping, k, v, codebooks: Codebooks, sign_seed: int,
+                        qjl_seed: int, stream=None) -> None:
+    _require_cuda(pages, slot_mapping, k, v)
+    st = _stream_handle(stream, pages.device)
+    _check(_load().tq_quantize_append_qjl(_desc(pages), _desc(slot_mapping), _desc(k), _desc(v),
+                                          ctypes.byref(codebooks.desc), ctypes.c_uint64(sign_seed),
+                                          ctypes.c_uint64(qjl_seed), codebooks.k_bits,
+                                          codebooks.v_bits, st),
+           "tq_quantize_append_qjl")
+
+
+def paged_decode_qjl(out, q, pages, block_table, seq_lens, codebooks: Codebooks, sign_seed: int,
+                     qjl_seed: int, scale: float, stream=None) -> None:
+    _require_cuda(out, q, pages, block_table, seq_lens)
+    st = _stream_handle(stream, q.device)
+    _check(_load().tq_paged_decode_qjl(_desc(out), _desc(q), _desc(pages), _desc(block_table),
+                                       _desc(seq_lens), ctypes.byref(codebooks.desc),
+                                       ctypes.c_uint64(sign_seed), ctypes.c_uint64(qjl_seed),
+                                       ctypes.c_float(scale), st),
+           "tq_paged_decode_qjl")
 
 
 def rotate_unit(u, norm, x, sign_seed: int, stream=None) -> None:

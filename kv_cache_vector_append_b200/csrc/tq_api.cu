@@ -169,7 +169,7 @@ int pow2_floor(int x) {
 // Geometry of the decode kernel for one call (see tq_decode.cuh).
 tq_status plan_decode(int batch, int h_q, int h_kv, int dim, int kb, int vb, int slot_stride,
                       int max_blocks, bool allow_tensor_copy, const DeviceInfo& di,
-                      DecodePlan* plan) {
+                      DecodePlan* plan, bool qjl = false) {
   plan->maxw = decode_maxw(dim, h_q / h_kv);
   if (h_kv < 1 || h_kv > plan->maxw) return TQ_ERR_UNSUPPORTED;
   // A block is staged by one TMA copy.  When a row is a multiple of 16 bytes and the
@@ -208,7 +208,8 @@ tq_status plan_decode(int batch, int h_q, int h_kv, int dim, int kb, int vb, int
       for (int nst = kMaxStages; nst >= min_st; --nst) {
         const int64_t misc = 16 * nst + 2LL * h_q * dim + 4LL * h_q + 4LL * (batch + 1) +
                              4LL * ids_cap + 4 * 36 + (int64_t)plan->maxw * (dim + 2) * 4 +
-                             4LL * dim + 16;
+                             4LL * dim + 32 +
+                             (qjl ? ((int64_t)h_q * qjl_qz_stride(dim) + 15) / 16 * 16 : 0);
         for (int at_top = 0; at_top < 2; ++at_top) {
           const int64_t below = at_top ? low : low - misc;   // room for stages below
           if (below < 0) continue;
@@ -309,6 +310,7 @@ bool encode_input_map(CUtensorMap* map, const void* data, int64_t T, int h_kv, i
 
 struct DecodeCall {
   int B = 0, h_q = 0, h_kv = 0, D = 0, kbits = 0, vbits = 0, kb = 0, max_blocks = 0;
+  bool qjl = false;
   int64_t stride = 0;
   DeviceState* ds = nullptr;
   DecodePlan plan;
@@ -317,7 +319,8 @@ struct DecodeCall {
 // Validation and geometry of one decode call (shared by the decode entry points).
 tq_status decode_prepare(const tq_tensor& out, const tq_tensor& q, const tq_tensor& pages,
                          const tq_tensor& block_table, const tq_tensor& seq_lens,
-                         const tq_codebooks* cb, float scale, DecodeCall* call) {
+                         const tq_codebooks* cb, float scale, DecodeCall* call,
+                         bool qjl = false) {
   if (cb == nullptr || !std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
   if (!valid_tensor(q, 3) || !is_float_dtype(q.dtype) || q.stride[2] != 1) return TQ_ERR_INVALID_ARG;
   if (!valid_tensor(out, 3) || !is_float_dtype(out.dtype) || out.stride[2] != 1 ||
@@ -336,7 +339,7 @@ tq_status decode_prepare(const tq_tensor& out, const tq_tensor& q, const tq_tens
   if (h_kv < 1 || h_q % h_kv) return TQ_ERR_INVALID_ARG;
   if (!valid_codebook(cb->k, D) || !valid_codebook(cb->v, D)) return TQ_ERR_INVALID_ARG;
   const int kbits = cb->k.bits, vbits = cb->v.bits;
-  const int kb = region_bytes(D, kbits), vb = region_bytes(D, vbits);
+  const int kb = region_bytes(D, kbits) + (qjl ? D / 8 + 4 : 0), vb = region_bytes(D, vbits);
   const int64_t stride = pages.shape[3];
   if (stride < kb + vb || stride % 8) return TQ_ERR_INVALID_ARG;
   // contiguous page tensor: whole blocks are staged with 16-byte copies
@@ -347,6 +350,8 @@ tq_status decode_prepare(const tq_tensor& out, const tq_tensor& q, const tq_tens
   if (D != 64 && D != 128 && D != 256) return TQ_ERR_UNSUPPORTED;
   if (h_q / h_kv > 16 || h_kv > decode_maxw(D, h_q / h_kv)) return TQ_ERR_UNSUPPORTED;
   if (!decode_bits_supported(kbits, vbits)) return TQ_ERR_UNSUPPORTED;
+  if (qjl && (D == 64 || kbits > 4)) return TQ_ERR_UNSUPPORTED;
+  call->qjl = qjl;
   call->B = B;
   if (B == 0) return TQ_OK;
   DeviceState* ds = nullptr;
@@ -355,7 +360,7 @@ tq_status decode_prepare(const tq_tensor& out, const tq_tensor& q, const tq_tens
   const int max_blocks = (int)block_table.shape[1];
   DecodePlan plan;
   s = plan_decode(B, h_q, h_kv, D, kbits, vbits, (int)stride, std::max(max_blocks, 1), true,
-                  ds->info, &plan);
+                  ds->info, &plan, qjl);
   if (s != TQ_OK) return s;
   if ((h_kv * stride) % 8) return TQ_ERR_INVALID_ARG;
   call->h_q = h_q;
@@ -400,7 +405,7 @@ tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tens
                      const tq_tensor& pages, const tq_tensor& block_table,
                      const tq_tensor& seq_lens, const tq_codebooks* cb, uint64_t sign_seed,
                      float scale, uint8_t* ws, void* stream, const HotWindow& hw = HotWindow(),
-                     const tq_rotation* rot = nullptr) {
+                     const tq_rotation* rot = nullptr, uint64_t qjl_seed = 0) {
   const int B = call.B, h_q = call.h_q, h_kv = call.h_kv, D = call.D;
   const int kbits = call.kbits, vbits = call.vbits, kb = call.kb;
   const int64_t stride = call.stride;
@@ -413,7 +418,7 @@ tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tens
       !encode_page_map(&tmap, pages.data, pages.shape[0], h_kv * (int)stride, plan.row_pitch)) {
     // the 1-D bulk layout never needs more shared memory or workspace than the 2-D one
     const tq_status s = plan_decode(B, h_q, h_kv, D, kbits, vbits, (int)stride,
-                                    std::max(max_blocks, 1), false, ds->info, &plan);
+                                    std::max(max_blocks, 1), false, ds->info, &plan, call.qjl);
     if (s != TQ_OK) return s;
   }
   DecodeParams p{};
@@ -460,6 +465,8 @@ tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tens
   p.counters = (unsigned int*)(ws + plan.counters_off);
   p.wait_ms = kWaitMs;
   p.withhold_cta = -1;
+  p.qjl = call.qjl ? 1 : 0;
+  p.qjl_seed = qjl_seed;
   p.rot_hi = rot ? rot->hi : nullptr;
   p.rot_lo = rot ? rot->lo : nullptr;
   p.hot_k = nullptr;
@@ -544,9 +551,34 @@ tq_status tq_slot_bytes(int32_t dim, int32_t k_bits, int32_t v_bits, int32_t* ou
   return TQ_OK;
 }
 
+tq_status append_impl(tq_tensor pages, tq_tensor slot_mapping, tq_tensor k, tq_tensor v,
+                      const tq_codebooks* cb, uint64_t sign_seed, int32_t k_bits, int32_t v_bits,
+                      void* stream, bool qjl, uint64_t qjl_seed);
+
 tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_tensor k, tq_tensor v,
                              const tq_codebooks* cb, uint64_t sign_seed, int32_t k_bits,
                              int32_t v_bits, void* stream) {
+  return append_impl(pages, slot_mapping, k, v, cb, sign_seed, k_bits, v_bits, stream, false, 0);
+}
+
+tq_status tq_quantize_append_qjl(tq_tensor pages, tq_tensor slot_mapping, tq_tensor k,
+                                 tq_tensor v, const tq_codebooks* cb, uint64_t sign_seed,
+                                 uint64_t qjl_seed, int32_t k_bits, int32_t v_bits, void* stream) {
+  return append_impl(pages, slot_mapping, k, v, cb, sign_seed, k_bits, v_bits, stream, true,
+                     qjl_seed);
+}
+
+tq_status tq_slot_bytes_qjl(int32_t dim, int32_t k_bits, int32_t v_bits, int32_t* out) {
+  if (out == nullptr || dim < 8 || dim % 8 || k_bits < 1 || k_bits > 8 || v_bits < 1 ||
+      v_bits > 8)
+    return TQ_ERR_INVALID_ARG;
+  *out = region_bytes(dim, k_bits) + dim / 8 + 4 + region_bytes(dim, v_bits);
+  return TQ_OK;
+}
+
+tq_status append_impl(tq_tensor pages, tq_tensor slot_mapping, tq_tensor k, tq_tensor v,
+                      const tq_codebooks* cb, uint64_t sign_seed, int32_t k_bits, int32_t v_bits,
+                      void* stream, bool qjl, uint64_t qjl_seed) {
   if (cb == nullptr) return TQ_ERR_INVALID_ARG;
   if (!valid_tensor(pages, 4) || pages.dtype != TQ_U8 || pages.stride[3] != 1)
     return TQ_ERR_INVALID_ARG;
@@ -565,7 +597,8 @@ tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_tensor 
       cb->v.bits != v_bits)
     return TQ_ERR_INVALID_ARG;
   if (D != 64 && D != 128 && D != 256) return TQ_ERR_UNSUPPORTED;
-  const int kb = region_bytes(D, k_bits), vb = region_bytes(D, v_bits);
+  if (qjl && D == 64) return TQ_ERR_UNSUPPORTED;
+  const int kb = region_bytes(D, k_bits) + (qjl ? D / 8 + 4 : 0), vb = region_bytes(D, v_bits);
   if (pages.shape[3] < kb + vb || pages.shape[3] % 8 != 0) return TQ_ERR_INVALID_ARG;
   if (pages.stride[0] % 4 || pages.stride[1] % 4 || pages.stride[2] % 4 ||
       (uintptr_t)pages.data % 4)
@@ -603,6 +636,8 @@ tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_tensor 
   p.region_off[0] = 0;
   p.region_off[1] = kb;
   p.sign_seed = sign_seed;
+  p.kcent = qjl ? cb->k.centroids : nullptr;
+  p.qjl_seed = qjl_seed;
   p.err = ds->err.load(std::memory_order_relaxed);
   p.redo = ds->redo;
   const int es = dtype_size(k.dtype);
@@ -892,6 +927,19 @@ tq_status tq_paged_decode(tq_tensor out, tq_tensor q, tq_tensor pages, tq_tensor
   s = decode_workspace(call, &ws);
   if (s != TQ_OK) return s;
   return decode_run(call, out, q, pages, block_table, seq_lens, cb, sign_seed, scale, ws, stream);
+}
+
+tq_status tq_paged_decode_qjl(tq_tensor out, tq_tensor q, tq_tensor pages, tq_tensor block_table,
+                              tq_tensor seq_lens, const tq_codebooks* cb, uint64_t sign_seed,
+                              uint64_t qjl_seed, float scale, void* stream) {
+  DecodeCall call;
+  tq_status s = decode_prepare(out, q, pages, block_table, seq_lens, cb, scale, &call, true);
+  if (s != TQ_OK || call.B == 0) return s;
+  uint8_t* ws = nullptr;
+  s = decode_workspace(call, &ws);
+  if (s != TQ_OK) return s;
+  return decode_run(call, out, q, pages, block_table, seq_lens, cb, sign_seed, scale, ws, stream,
+                    HotWindow(), nullptr, qjl_seed);
 }
 
 tq_status tq_paged_decode_hot(tq_tensor out, tq_tensor q, tq_tensor pages, tq_tensor block_table,

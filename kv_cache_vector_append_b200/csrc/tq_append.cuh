@@ -57,6 +57,10 @@ struct AppendParams {
   int32_t tma_in;           // 1: input rows staged by tensor copies (maps K, V)
   int32_t bulk_out;         // 1: slots stored by one bulk copy per token run
   unsigned int* redo;       // [2]: a row left the fast path's range; CTAs of the redo done
+  // QJL residual sketch of the keys (append_kernel<..., QJL = true>): K centroids and the
+  // seed of the sketch's signs
+  const float* kcent;
+  uint64_t qjl_seed;
 };
 
 // Tensor maps of K and V as (D, h_kv, tokens) 16-bit elements, boxes of
@@ -423,10 +427,12 @@ __device__ __forceinline__ float rotate_row(uint64_t (&xp)[32], uint32_t row, co
   return n > 0.f ? __frcp_rn(__fmul_rn(n, sqrt_d)) : 0.f;
 }
 
-// Encode u = x * r and pack the 64 codes LSB-first into 2*BITS words.
-template <int BITS, bool FAST>
-__device__ __forceinline__ void encode_pack(const uint64_t (&xp)[32], float r,
-                                            const EncodeTables* t, uint32_t* words) {
+// Encode u = x * r and pack the 64 codes LSB-first into 2*BITS words.  RES: also leave
+// the residuals u - c[code] in xp (fp32 pairs), with `cent_win` the shared-window address
+// of the centroid table.
+template <int BITS, bool FAST, bool RES = false>
+__device__ __forceinline__ void encode_pack(uint64_t (&xp)[32], float r, const EncodeTables* t,
+                                            uint32_t* words, uint32_t cent_win = 0) {
   constexpr int W = 64 * BITS / 32;
   uint32_t acc[W];
 #pragma unroll
@@ -436,6 +442,7 @@ __device__ __forceinline__ void encode_pack(const uint64_t (&xp)[32], float r,
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     const uint64_t u2 = mul2(xp[i], r2);
+    float cv[2];
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       const float u = hf ? f2hi(u2) : f2lo(u2);
@@ -449,6 +456,7 @@ __device__ __forceinline__ void encode_pack(const uint64_t (&xp)[32], float r,
         if (o0 >= 2) acc[w0] += c4 << (o0 - 2);
         else acc[w0] += c4 >> (2 - o0);
         if (o0 + BITS > 32) acc[w0 + 1] += c4 >> (32 - o0 + 2);
+        if constexpr (RES) cv[hf] = lds_f32(cent_win + c4);
       } else {
         int e = 1;
 #pragma unroll
@@ -456,24 +464,83 @@ __device__ __forceinline__ void encode_pack(const uint64_t (&xp)[32], float r,
         const uint32_t code = (uint32_t)(e - (1 << BITS));
         acc[w0] += code << o0;
         if (o0 + BITS > 32) acc[w0 + 1] += code >> (32 - o0);
+        if constexpr (RES) cv[hf] = lds_f32(cent_win + 4 * code);
       }
     }
+    if constexpr (RES) xp[i] = sub2(u2, f2(cv[0], cv[1]));
   }
 #pragma unroll
   for (int w = 0; w < W; ++w) words[w] = acc[w];
 }
 
-template <int BITS>
-__device__ __forceinline__ void encode_pack_any(const uint64_t (&xp)[32], float r,
+template <int BITS, bool RES = false>
+__device__ __forceinline__ void encode_pack_any(uint64_t (&xp)[32], float r,
                                                 const EncodeTables* t, int fast,
-                                                uint32_t* words) {
+                                                uint32_t* words, uint32_t cent_win = 0) {
   if constexpr (BITS <= 4) {
     if (fast) {
-      encode_pack<BITS, true>(xp, r, t, words);
+      encode_pack<BITS, true, RES>(xp, r, t, words, cent_win);
       return;
     }
   }
-  encode_pack<BITS, false>(xp, r, t, words);
+  encode_pack<BITS, false, RES>(xp, r, t, words, cent_win);
+}
+
+template <bool RES>
+__device__ __forceinline__ void encode_pack_bits(int bits, uint64_t (&xp)[32], float r,
+                                                 const EncodeTables* t, int fast,
+                                                 uint32_t* words, uint32_t cent_win) {
+  switch (bits) {
+    case 1: encode_pack_any<1, RES>(xp, r, t, fast, words, cent_win); break;
+    case 2: encode_pack_any<2, RES>(xp, r, t, fast, words, cent_win); break;
+    case 3: encode_pack_any<3, RES>(xp, r, t, fast, words, cent_win); break;
+    case 4: encode_pack_any<4, RES>(xp, r, t, fast, words, cent_win); break;
+    case 5: encode_pack_any<5, RES>(xp, r, t, fast, words, cent_win); break;
+    case 6: encode_pack_any<6, RES>(xp, r, t, fast, words, cent_win); break;
+    case 7: encode_pack_any<7, RES>(xp, r, t, fast, words, cent_win); break;
+    default: encode_pack_any<8, RES>(xp, r, t, fast, words, cent_win); break;
+  }
+}
+
+// QJL sketch of this lane's 64 residuals r (in xp): the sketch's sign flips (`qm`, as in
+// load_signed), the FWHT (stage h = 1 here, then fwht_ss), and the sign bits
+// z_j = [ (S r)_j >= 0 ] of the lane's coordinates into two words (bit j of the lane's
+// 64).  Returns gamma = ||r||_2 of the row (the lanes of the row combined).
+template <int D>
+__device__ __forceinline__ float qjl_sketch_row(uint64_t (&xp)[32], const uint32_t* qm, int part,
+                                                uint32_t* z0, uint32_t* z1) {
+  using G = AppendGeom<D>;
+  uint64_t g2 = 0ull;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) g2 = fma2(xp[i], xp[i], g2);
+  float gg = __fadd_rn(f2lo(g2), f2hi(g2));
+#pragma unroll
+  for (int m = 1; m < G::TPR; m <<= 1)
+    gg = __fadd_rn(gg, __shfl_xor_sync(0xffffffffu, gg, G::ROWS * m));
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 s0 = *(const uint4*)(qm + 8 * c);
+    const uint4 s1 = *(const uint4*)(qm + 8 * c + 4);
+    const uint32_t sm[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float a = __uint_as_float(__float_as_uint(f2lo(xp[4 * c + k])) ^ sm[2 * k]);
+      const float b = __uint_as_float(__float_as_uint(f2hi(xp[4 * c + k])) ^ sm[2 * k + 1]);
+      xp[4 * c + k] = f2(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+  }
+  (void)fwht_ss<D>(xp, part);
+  uint32_t w0 = 0u, w1 = 0u;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    w0 |= (f2lo(xp[i]) >= 0.f ? 1u : 0u) << (2 * i);
+    w0 |= (f2hi(xp[i]) >= 0.f ? 1u : 0u) << (2 * i + 1);
+    w1 |= (f2lo(xp[16 + i]) >= 0.f ? 1u : 0u) << (2 * i);
+    w1 |= (f2hi(xp[16 + i]) >= 0.f ? 1u : 0u) << (2 * i + 1);
+  }
+  *z0 = w0;
+  *z1 = w1;
+  return sqrtf(gg);
 }
 
 // Shared memory: the K and V tables and sign masks; then (1024-byte aligned, as the
@@ -486,9 +553,11 @@ struct AppendSmem {
   static constexpr int RB = D * InType<Tin>::kBytes;    // bytes of one input row
   static constexpr int PB = 64 * InType<Tin>::kBytes;   // bytes of one lane's part of a row
   static constexpr int KIND = G::TPR * G::ROWS * PB;    // one kind's rows of a tile
-  static constexpr int TABLES = ((2 * (int)sizeof(EncodeTables) + 4 * D + 8) + 127) / 128 * 128;
+  // K and V tables, sign masks, flags[4], K centroids[256], QJL sign masks
+  static constexpr int TABLES =
+      ((2 * (int)sizeof(EncodeTables) + 4 * D + 16 + 1024 + 4 * D) + 127) / 128 * 128;
   static __host__ __device__ constexpr int slot_words(int kbits, int vbits) {
-    return (D * kbits / 8 + 4 + D * vbits / 8 + 4) / 4;
+    return (D * kbits / 8 + 4 + D * vbits / 8 + 4) / 4 + D / 32 + 1;   // room for a sketch
   }
   static __host__ __device__ constexpr int misc_per_warp(int swords) {
     return 16 + 2 * G::ROWS * 8 + 2 * 2 * G::ROWS * 8 + (G::ROWS * swords * 4 + 15) / 16 * 16;
@@ -508,7 +577,9 @@ struct AppendSmem {
 // returns at once unless redo[0] is set, and otherwise the whole call is done again
 // with the rescaling rotation (identical results for the other rows); the last CTA
 // clears redo.
-template <int D, typename Tin, bool SAFE>
+// QJL: the K rows also store the QJL sketch of their residual (K region: codes, norm,
+// D sign bits, residual norm).
+template <int D, typename Tin, bool SAFE, bool QJL>
 __global__ void __launch_bounds__(kAppendWarps * 32, 2)
 append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
   if constexpr (SAFE) {
@@ -520,8 +591,10 @@ append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
   EncodeTables* tabs = (EncodeTables*)smem;                       // [2]: K, V
   uint32_t* smask = (uint32_t*)(smem + 2 * sizeof(EncodeTables));  // D sign masks
   int* fast = (int*)(smask + D);                                    // [2] bucket encode valid
+  float* kcent_s = (float*)(fast + 4);                              // [256] K centroids (QJL)
+  uint32_t* qmask = (uint32_t*)(kcent_s + 256);                     // [D] QJL sketch signs
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kwords = (D * p.bits[0] + 7) / 8 / 4 + 1;             // K region words
+  const int kwords = (D * p.bits[0] + 7) / 8 / 4 + 1 + (QJL ? D / 32 + 1 : 0);   // K region
   const int vwords = (D * p.bits[1] + 7) / 8 / 4 + 1;
   const int swords = kwords + vwords;                              // slot words written
   const uint32_t sbase = smem_u32(smem);
@@ -612,6 +685,10 @@ append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
   build_tables(&tabs[0], p.boundaries[0], p.bits[0], threadIdx.x, blockDim.x, &fast[0]);
   build_tables(&tabs[1], p.boundaries[1], p.bits[1], threadIdx.x, blockDim.x, &fast[1]);
   for (int j = threadIdx.x; j < D; j += blockDim.x) smask[j] = sign_mask_at(p.sign_seed, j);
+  if constexpr (QJL) {
+    for (int j = threadIdx.x; j < D; j += blockDim.x) qmask[j] = sign_mask_at(p.qjl_seed, j);
+    for (int j = threadIdx.x; j < (1 << p.bits[0]); j += blockDim.x) kcent_s[j] = p.kcent[j];
+  }
   __syncthreads();
   build_bucket_table(&tabs[0], p.bits[0], threadIdx.x, blockDim.x);
   build_bucket_table(&tabs[1], p.bits[1], threadIdx.x, blockDim.x);
@@ -654,7 +731,6 @@ append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
       }
       __syncwarp();
       const int bits = p.bits[kind];
-      const int rwords = kind ? vwords : kwords;          // packed words + norm word
       uint64_t xp[32];
       float n;
       bool bad, oor;
@@ -667,25 +743,32 @@ append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
       }
       uint32_t* orow = out_s + rl * swords + (kind ? kwords : 0);
       const EncodeTables* t = &tabs[kind];
-      const int wpl = (rwords - 1) / G::TPR;               // words per lane
+      const int cw = D * bits / 32;                        // code words of the region
+      const int wpl = cw / G::TPR;                         // code words per lane
       uint32_t* mine = orow + part * wpl;
+      const bool sketch = QJL && kind == 0;
       if (!bad) {
         const int use_fast = fast[kind];
-        switch (bits) {
-          case 1: encode_pack_any<1>(xp, r, t, use_fast, mine); break;
-          case 2: encode_pack_any<2>(xp, r, t, use_fast, mine); break;
-          case 3: encode_pack_any<3>(xp, r, t, use_fast, mine); break;
-          case 4: encode_pack_any<4>(xp, r, t, use_fast, mine); break;
-          case 5: encode_pack_any<5>(xp, r, t, use_fast, mine); break;
-          case 6: encode_pack_any<6>(xp, r, t, use_fast, mine); break;
-          case 7: encode_pack_any<7>(xp, r, t, use_fast, mine); break;
-          default: encode_pack_any<8>(xp, r, t, use_fast, mine); break;
+        if (sketch) {
+          encode_pack_bits<true>(bits, xp, r, t, use_fast, mine, smem_u32(kcent_s));
+          uint32_t z0, z1;
+          const float gamma = qjl_sketch_row<D>(xp, qmask + part * 64, part, &z0, &z1);
+          orow[cw + 1 + 2 * part] = z0;
+          orow[cw + 2 + 2 * part] = z1;
+          if (part == G::TPR - 1) orow[cw + 1 + D / 32] = __float_as_uint(gamma);
+        } else {
+          encode_pack_bits<false>(bits, xp, r, t, use_fast, mine, 0u);
         }
       } else {
         for (int w = 0; w < wpl; ++w) mine[w] = 0u;
+        if (sketch) {
+          orow[cw + 1 + 2 * part] = 0u;
+          orow[cw + 2 + 2 * part] = 0u;
+          if (part == G::TPR - 1) orow[cw + 1 + D / 32] = 0u;
+        }
         if (part == 0 && rl < nr) report_error(p.err, TQ_DEVERR_NONFINITE);
       }
-      if (part == G::TPR - 1) orow[rwords - 1] = bad ? 0x7FC00000u : __float_as_uint(n);
+      if (part == G::TPR - 1) orow[cw] = bad ? 0x7FC00000u : __float_as_uint(n);
       __syncwarp();
     }
     if (dead) break;

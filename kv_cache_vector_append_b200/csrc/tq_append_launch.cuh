@@ -6,13 +6,13 @@
 
 namespace tq {
 
-template <int D, typename Tin>
-tq_status launch_append_t(const AppendParams& p, const AppendMaps& maps, const DeviceInfo& di,
+template <int D, typename Tin, bool QJL>
+tq_status launch_append_q(const AppendParams& p, const AppendMaps& maps, const DeviceInfo& di,
                           cudaStream_t st) {
   const size_t smem = AppendSmem<D, Tin>::bytes(p.bits[0], p.bits[1]);
   if ((int)smem > di.max_smem_optin) return TQ_ERR_UNSUPPORTED;
-  auto kern = append_kernel<D, Tin, false>;
-  auto kern_safe = append_kernel<D, Tin, true>;
+  auto kern = append_kernel<D, Tin, false, QJL>;
+  auto kern_safe = append_kernel<D, Tin, true, QJL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
           cudaSuccess ||
       cudaFuncSetAttribute(kern_safe, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -32,6 +32,16 @@ tq_status launch_append_t(const AppendParams& p, const AppendMaps& maps, const D
   kern<<<grid, kAppendWarps * 32, smem, st>>>(p, maps);
   kern_safe<<<grid, kAppendWarps * 32, smem, st>>>(p, maps);
   return launch_status();
+}
+
+// The plain append, or (p.kcent set) the one that also stores the keys' QJL sketch
+// (built for head_dim 128 and 256).
+template <int D, typename Tin>
+tq_status launch_append_t(const AppendParams& p, const AppendMaps& maps, const DeviceInfo& di,
+                          cudaStream_t st) {
+  if (p.kcent == nullptr) return launch_append_q<D, Tin, false>(p, maps, di, st);
+  if constexpr (D >= 128) return launch_append_q<D, Tin, true>(p, maps, di, st);
+  return TQ_ERR_UNSUPPORTED;
 }
 
 template <int D, typename Tin>

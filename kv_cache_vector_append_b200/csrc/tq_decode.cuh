@@ -125,7 +125,16 @@ struct DecodeParams {
   int32_t hot_dtype;
   int32_t hot_cap;              // W
   const int32_t* hot_lens;
+  // QJL residual sketch of the keys (decode_kernel MODE 2): K region = [codes | norm |
+  // D sign bits | residual norm gamma]; the sketch's signs come from qjl_seed
+  int32_t qjl;
+  uint64_t qjl_seed;
 };
+
+// Bytes per query head of the QJL mode's sketched-query fragments: (b0, b1) half2 pairs
+// for every (k-step, tig), padded by 8 bytes so that the 8 heads of a warp's B
+// fragments fall in different banks.
+__host__ __device__ constexpr int qjl_qz_stride(int d) { return d / 16 * 32 + 8; }
 
 // Arguments of the hot-window partial (a copy of the fields it reads).
 struct HotArgs {
@@ -389,10 +398,24 @@ template <int E>
 __device__ __forceinline__ void rot_row_part(const uint16_t* hi, const uint16_t* lo, int r,
                                              int lane, float (&v)[E]) {
   constexpr int D = 32 * E;
-  const int64_t o = (int64_t)r * D + lane * E;
+  const int64_t o = (int64_t)r * D + lane * E;   // E consecutive entries, 2E-byte aligned
+  uint32_t h[E / 2], l[E / 2];
+  if constexpr (E == 2) {
+    h[0] = *(const uint32_t*)(hi + o);
+    l[0] = *(const uint32_t*)(lo + o);
+  } else if constexpr (E == 4) {
+    const uint2 a = *(const uint2*)(hi + o), b = *(const uint2*)(lo + o);
+    h[0] = a.x; h[1] = a.y; l[0] = b.x; l[1] = b.y;
+  } else {
+    const uint4 a = *(const uint4*)(hi + o), b = *(const uint4*)(lo + o);
+    h[0] = a.x; h[1] = a.y; h[2] = a.z; h[3] = a.w;
+    l[0] = b.x; l[1] = b.y; l[2] = b.z; l[3] = b.w;
+  }
 #pragma unroll
-  for (int i = 0; i < E; ++i)
-    v[i] = __uint_as_float((uint32_t)hi[o + i] << 16) + __uint_as_float((uint32_t)lo[o + i] << 16);
+  for (int i = 0; i < E / 2; ++i) {
+    v[2 * i] = __uint_as_float(h[i] << 16) + __uint_as_float(l[i] << 16);
+    v[2 * i + 1] = __uint_as_float(h[i] & 0xffff0000u) + __uint_as_float(l[i] & 0xffff0000u);
+  }
 }
 
 // sc[0 .. D) <- R sc[0 .. D) for one warp (sc: this warp's shared scratch).  Output c is
@@ -406,15 +429,24 @@ __device__ __noinline__ void dense_forward(const uint16_t* hi, const uint16_t* l
 #pragma unroll
   for (int i = 0; i < E; ++i) x[i] = sc[lane * E + i];
   __syncwarp();
-  for (int c = 0; c < D; ++c) {
-    float r[E];
-    rot_row_part<E>(hi, lo, c, lane, r);
-    float part = 0.f;
+  for (int c = 0; c < D; c += 4) {            // four independent reductions at a time
+    float part[4];
 #pragma unroll
-    for (int i = 0; i < E; ++i) part = fmaf(r[i], x[i], part);
+    for (int j = 0; j < 4; ++j) {
+      float r[E];
+      rot_row_part<E>(hi, lo, c + j, lane, r);
+      part[j] = 0.f;
 #pragma unroll
-    for (int m = 16; m > 0; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
-    if (lane == 0) sc[c] = part;
+      for (int i = 0; i < E; ++i) part[j] = fmaf(r[i], x[i], part[j]);
+    }
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) part[j] += __shfl_xor_sync(0xffffffffu, part[j], m);
+    if (lane == 0) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sc[c + j] = part[j];
+    }
   }
   __syncwarp();
 }
@@ -454,8 +486,15 @@ __device__ __forceinline__ float load_as_f32(const void* base, int64_t i, int32_
 // L = sum_t 2^(s_t - M), o = sum_t 2^(s_t - M) v_t, written to sc[0] = M, sc[1] = L,
 // sc[2 + c] = o_c (this warp's shared scratch).  A hot_lens entry outside [0, W] raises
 // TQ_DEVERR_SEQLEN_RANGE and counts as 0 tokens.  Out of line, as dense_forward.
-template <int D>
-__device__ __noinline__ void hot_partial(const HotArgs a, int b, int h, int lane, float* sc) {
+template <typename T>
+__device__ __forceinline__ float as_f32(T x) {
+  if constexpr (std::is_same<T, float>::value) return x;
+  else return to_f32(x);
+}
+
+template <int D, typename T>
+__device__ __forceinline__ void hot_partial_t(const HotArgs& a, int b, int h, int lane,
+                                              float* sc) {
   constexpr int E = D / 32;
   float M = -INFINITY, L = 0.f, o[E];
 #pragma unroll
@@ -469,27 +508,48 @@ __device__ __noinline__ void hot_partial(const HotArgs a, int b, int h, int lane
   const int64_t qo = (int64_t)b * a.q_bstride + (int64_t)h * a.q_hstride + lane * E;
 #pragma unroll
   for (int i = 0; i < E; ++i) qv[i] = load_as_f32(a.q, qo + i, a.q_dtype);
+  const T* hk = (const T*)a.hot_k;
+  const T* hv = (const T*)a.hot_v;
   const int64_t base = (int64_t)b * a.hot_bstride + (int64_t)(h / a.group) * a.hot_hstride +
                        lane * E;
-  for (int t = 0; t < n; ++t) {
-    const int64_t off = base + (int64_t)t * a.hot_tstride;
-    float dot = 0.f;
+  for (int t0 = 0; t0 < n; t0 += 4) {          // four tokens: independent reductions
+    float dot[4];
 #pragma unroll
-    for (int i = 0; i < E; ++i) dot = fmaf(qv[i], load_as_f32(a.hot_k, off + i, a.hot_dtype), dot);
+    for (int j = 0; j < 4; ++j) {
+      dot[j] = 0.f;
+      if (t0 + j < n) {
+        const int64_t off = base + (int64_t)(t0 + j) * a.hot_tstride;
 #pragma unroll
-    for (int m = 16; m > 0; m >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, m);
-    const float sc_t = dot * a.scale_log2;
-    if (sc_t > M) {
-      const float f = M == -INFINITY ? 0.f : exp2f(M - sc_t);
+        for (int i = 0; i < E; ++i) dot[j] = fmaf(qv[i], as_f32(hk[off + i]), dot[j]);
+      }
+    }
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dot[j] += __shfl_xor_sync(0xffffffffu, dot[j], m);
+    float mx = M;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      dot[j] = t0 + j < n ? dot[j] * a.scale_log2 : -INFINITY;
+      mx = fmaxf(mx, dot[j]);
+    }
+    if (mx > M) {
+      const float f = M == -INFINITY ? 0.f : exp2f(M - mx);
       L *= f;
 #pragma unroll
       for (int i = 0; i < E; ++i) o[i] *= f;
-      M = sc_t;
+      M = mx;
     }
-    const float w = exp2f(sc_t - M);
-    L += w;
 #pragma unroll
-    for (int i = 0; i < E; ++i) o[i] = fmaf(w, load_as_f32(a.hot_v, off + i, a.hot_dtype), o[i]);
+    for (int j = 0; j < 4; ++j) {
+      if (t0 + j < n) {
+        const float w = exp2f(dot[j] - M);
+        const int64_t off = base + (int64_t)(t0 + j) * a.hot_tstride;
+        L += w;
+#pragma unroll
+        for (int i = 0; i < E; ++i) o[i] = fmaf(w, as_f32(hv[off + i]), o[i]);
+      }
+    }
   }
   __syncwarp();
   if (lane == 0) {
@@ -499,6 +559,19 @@ __device__ __noinline__ void hot_partial(const HotArgs a, int b, int h, int lane
 #pragma unroll
   for (int i = 0; i < E; ++i) sc[2 + lane * E + i] = o[i];
   __syncwarp();
+}
+
+// Attention partial of query head h of sequence b over its hot-window tokens, computed
+// by one warp in the original (unrotated) domain: lane l handles coordinates
+// l E .. l E + E - 1.  With s_t = scale log2(e) <q, k_t> (fp32): M = max_t s_t,
+// L = sum_t 2^(s_t - M), o = sum_t 2^(s_t - M) v_t, written to sc[0] = M, sc[1] = L,
+// sc[2 + c] = o_c (this warp's shared scratch).  A hot_lens entry outside [0, W] raises
+// TQ_DEVERR_SEQLEN_RANGE and counts as 0 tokens.  Out of line, as dense_forward.
+template <int D>
+__device__ __noinline__ void hot_partial(const HotArgs a, int b, int h, int lane, float* sc) {
+  if (a.hot_dtype == TQ_F32) hot_partial_t<D, float>(a, b, h, lane, sc);
+  else if (a.hot_dtype == TQ_BF16) hot_partial_t<D, __nv_bfloat16>(a, b, h, lane, sc);
+  else hot_partial_t<D, __half>(a, b, h, lane, sc);
 }
 
 __device__ __forceinline__ void store_from_f32(void* base, int64_t i, int32_t dtype, float v) {
@@ -511,11 +584,18 @@ __device__ __forceinline__ void store_from_f32(void* base, int64_t i, int32_t dt
 // area [full mbarriers | release counters | present masks | q' (H_q x D fp16) | |q'|
 // scales | step prefix sums | block ids | scan scratch | flag | merge partials |
 // record positions].
-// EXT: the instantiation that also serves the hot window and the dense rotation (runtime
-// choices, both outside the step loop); the plain one carries none of their code.
-template <int D, int KB, int VB, int NH, int MAXW, bool EXT>
+// MODE 0: the plain kernel.  MODE 1 (EXT): also serves the hot window and the dense
+// rotation (runtime choices, both outside the step loop).  MODE 2 (QJL): keys carry the
+// QJL sketch of their residual, scored as
+//   s = scale nK (<q', c[idx]> + gamma sqrt(pi/2)/sqrt(D) <S q', 2z - 1>)
+// with S the sketch's randomized Hadamard transform (a second mma per k-step on +-1
+// fragments built from the sign bits).
+template <int D, int KB, int VB, int NH, int MAXW, int MODE>
 __global__ void __launch_bounds__(MAXW * 32, 1)
 decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
+  constexpr bool EXT = MODE == 1;
+  constexpr bool QJL = MODE == 2;
+  constexpr int QZS = qjl_qz_stride(D);
   using C = DecodeCfg<D, KB, VB>;
   using KS = typename C::KS;
   using VS = typename C::VS;
@@ -541,7 +621,9 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   uint32_t* present = (uint32_t*)(released + nst);     // per stage: bit k = block k staged
   __half* qh = (__half*)(present + nst);               // unit q' of the current sequence
   float* qsc = (float*)(qh + p.h_q * D);               // |q'| * scale * log2 e
-  int32_t* prefix = (int32_t*)(qsc + p.h_q);
+  // QJL: S q' / |q'| of every query head in mma B-fragment order (QZS bytes a head)
+  uint8_t* qz = (uint8_t*)(((uintptr_t)(qsc + p.h_q) + 15) & ~(uintptr_t)15);
+  int32_t* prefix = (int32_t*)(qz + (QJL ? (p.h_q * QZS + 15) / 16 * 16 : 0));
   int32_t* ids = (int32_t*)(prefix + p.batch + 1);     // block ids of the range
   int* wsum = (int*)(ids + p.ids_cap);                 // [32] per-warp sums of the scan
   int* timed_out = wsum + 32;                          // a stage wait of this CTA gave up
@@ -790,6 +872,24 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
 #pragma unroll
       for (int i = 0; i < E; ++i) qh[h * D + lane * E + i] = __float2half_rn(xq[i] * inv);
       if (lane == 0) qsc[h] = nrm * p.scale_log2;
+      if constexpr (QJL) {
+        // S q'/|q'| = (1/sqrt(D)) H (s2 * q'/|q'|), stored where the B fragments of the
+        // sketch product read it: coordinate c = 32 w + i of word w (bit i of the key's
+        // sign word w) goes to k-step 8 (w / 4) + (i % 16) / 2, thread w % 4, pair i % 2,
+        // half i / 16
+        float zq[E];
+#pragma unroll
+        for (int i = 0; i < E; ++i)
+          zq[i] = __uint_as_float(__float_as_uint(xq[i] * inv) ^ sign_mask_at(p.qjl_seed, lane * E + i));
+        warp_fwht<E>(zq, lane);
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          const int c = lane * E + i, w = c >> 5, bi = c & 31;
+          const int ks = 8 * (w >> 2) + ((bi & 15) >> 1);
+          const int off = h * QZS + (ks * 4 + (w & 3)) * 8 + (bi & 1) * 4 + (bi >> 4) * 2;
+          *(__half*)(qz + off) = __float2half_rn(zq[i] * inv_sqrt_dim<D>());
+        }
+      }
     };
     auto load_head = [&](int h, float (&xq)[E]) {
       const int64_t off = (int64_t)b * p.q_bstride + (int64_t)h * p.q_hstride + lane * E;
@@ -1137,6 +1237,43 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
             }
           });
         }
+        // QJL: the sketch product Z~ . (S Qhat)^T on +-1 fragments: bit i of the thread's
+        // sign word w gives the low half, bit i + 16 the high half (shifted into the fp16
+        // sign bit of +1 / -1)
+        float saccz[NH][4];
+        float kq[2];
+        if constexpr (QJL) {
+          constexpr int NWZ = D / 128;               // sign words a thread reads per row
+#pragma unroll
+          for (int hh = 0; hh < NH; ++hh)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) saccz[hh][k] = 0.f;
+          uint32_t zw0[NWZ], zw1[NWZ];
+#pragma unroll
+          for (int w = 0; w < NWZ; ++w) {
+            zw0[w] = *(const uint32_t*)(base + gid * pitch + C::KPACK + 4 + 4 * (tig + 4 * w));
+            zw1[w] = *(const uint32_t*)(base + (gid + 8) * pitch + C::KPACK + 4 + 4 * (tig + 4 * w));
+          }
+#pragma unroll
+          for (int r = 0; r < 2; ++r)
+            kq[r] = *(const float*)(base + (gid + 8 * r) * pitch + C::KPACK + 4 + D / 8) *
+                    (1.2533141373155003f * inv_sqrt_dim<D>());   // gamma sqrt(pi/2)/sqrt(D)
+          static_for<C::KSTEPS>([&](auto KSI) {
+            constexpr int ks = decltype(KSI)::value;
+            constexpr int w = ks / 8, i = 2 * (ks % 8);
+            const uint32_t a0 = ((zw0[w] << (15 - i)) & 0x80008000u) ^ 0xBC00BC00u;
+            const uint32_t a1 = ((zw1[w] << (15 - i)) & 0x80008000u) ^ 0xBC00BC00u;
+            const uint32_t a2 = ((zw0[w] << (14 - i)) & 0x80008000u) ^ 0xBC00BC00u;
+            const uint32_t a3 = ((zw1[w] << (14 - i)) & 0x80008000u) ^ 0xBC00BC00u;
+  #pragma unroll
+            for (int hh = 0; hh < NH; ++hh) {
+              const int g = 8 * hh + gid;
+              uint2 bz = make_uint2(0u, 0u);
+              if (g < G) bz = *(const uint2*)(qz + (kvh * G + g) * QZS + (ks * 4 + tig) * 8);
+              mma_16816(saccz[hh], a0, a1, a2, a3, bz.x, bz.y);
+            }
+          });
+        }
         // this thread's tokens: r = 0, 1  <->  token gid + 8 r
         float nK[2], nV[2], eV[2];
         bool ok[2];
@@ -1162,7 +1299,8 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
             zloc[e] = -INFINITY;
   #pragma unroll
             for (int r = 0; r < 2; ++r) {
-              const float a = sacc[hh][2 * r + e];
+              float a = sacc[hh][2 * r + e];
+              if constexpr (QJL) a = fmaf(kq[r], saccz[hh][2 * r + e], a);
               sv[e][r] = ok[r] ? a * nK[r] * qscale[hh][e] : -INFINITY;
               zloc[e] = fmaxf(zloc[e], sv[e][r] + eV[r]);
             }

@@ -56,8 +56,13 @@ inline bool decode_bits_supported(int kb, int vb) {
 template <int D, int KB, int VB, int NH, int MAXW>
 tq_status launch_decode_t(const DecodeParams& p, const DecodePlan& plan, const CUtensorMap& tmap,
                           int64_t steps_upper, cudaStream_t st) {
-  auto kern = (p.hot_k != nullptr || p.rot_hi != nullptr) ? decode_kernel<D, KB, VB, NH, MAXW, true>
-                                                          : decode_kernel<D, KB, VB, NH, MAXW, false>;
+  auto kern = decode_kernel<D, KB, VB, NH, MAXW, 0>;
+  if (p.qjl) {
+    if constexpr (D >= 128 && KB <= 4) kern = decode_kernel<D, KB, VB, NH, MAXW, 2>;
+    else return TQ_ERR_UNSUPPORTED;
+  } else if (p.hot_k != nullptr || p.rot_hi != nullptr) {
+    kern = decode_kernel<D, KB, VB, NH, MAXW, 1>;
+  }
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem) !=
       cudaSuccess)
     return TQ_ERR_CUDA;

@@ -806,3 +806,138 @@ def paged_decode_hot(q: np.ndarray, pages: np.ndarray, block_table: np.ndarray,
             p = np.exp(s - np.max(s))
             out[b, h] = (p / np.sum(p)) @ vals[:, kv, :]
     return out
+
+
+# ---------------------------------------------------------------------------
+# QJL residual sketch of the keys
+# ---------------------------------------------------------------------------
+
+QJL_CONST = math.sqrt(math.pi / 2.0)
+
+
+def qjl_region_bytes(dim: int) -> int:
+    """Bytes the QJL sketch adds to a K region: D sign bits, then the fp32 residual norm."""
+    return dim // 8 + 4
+
+
+def k_region_bytes(dim: int, bits: int, qjl: bool) -> int:
+    return region_bytes(dim, bits) + (qjl_region_bytes(dim) if qjl else 0)
+
+
+def qjl_sketch(r: np.ndarray, qjl_signs: np.ndarray):
+    """1-bit sketch of the residual r (..., D): z = [S r >= 0] with S = (1/sqrt(D)) H
+    diag(s'), a second randomized Hadamard transform with its own seeded signs
+    (tq-kv, "How It Works" step [5]: SRHT QJL error correction; TorbuQuant, "Current
+    Status": QJL residual).  Returns (z int64 (..., D) in {0, 1}, gamma = ||r||_2)."""
+    r = np.asarray(r, dtype=np.float64)
+    z = (rht_forward(r, qjl_signs) >= 0.0).astype(np.int64)
+    return z, np.sqrt(np.sum(r * r, axis=-1))
+
+
+def qjl_correction(z: np.ndarray, gamma: np.ndarray, qjl_signs: np.ndarray) -> np.ndarray:
+    """The residual estimate gamma sqrt(pi/2) / sqrt(D) S^T (2z - 1), in the rotated
+    domain: its inner product with a rotated query y is the QJL estimator
+    gamma sqrt(pi/2) / sqrt(D) <S y, sign(S r)> of <y, r> (unbiased over the sketch's
+    signs for large D)."""
+    d = np.asarray(z).shape[-1]
+    zpm = 2.0 * np.asarray(z, dtype=np.float64) - 1.0
+    return (np.asarray(gamma, dtype=np.float64)[..., None] * QJL_CONST / math.sqrt(d)
+            * rht_inverse(zpm, qjl_signs))
+
+
+def quantize_keys_qjl(x: np.ndarray, rot, table: CodebookTable, qjl_signs: np.ndarray):
+    """Keys with the QJL residual: the MSE quantizer of ``quantize_rows``, then the 1-bit
+    sketch of the rotated-domain residual r = u - c[idx].  Returns (idx, norm float32,
+    z, gamma float32, u, nonfinite); a non-finite row stores z = 0 and gamma = 0."""
+    idx, n32, u, bad = quantize_rows(x, rot, table)
+    c = np.asarray(table.centroids, dtype=np.float64)[idx]
+    r = np.where(bad[..., None], 0.0, u - c)
+    z, gamma = qjl_sketch(r, qjl_signs)
+    z = np.where(bad[..., None], 0, z)
+    return idx, n32, z, gamma.astype(np.float32), u, bad
+
+
+def encode_k_region_qjl(idx, norm32, z, gamma32, bits: int) -> np.ndarray:
+    """K region with the sketch: packed codes, fp32 norm, D sign bits (LSB-first, bit j
+    = z_j), fp32 residual norm gamma (little endian)."""
+    head = encode_region(idx, norm32, bits)
+    zb = pack_bits(z, 1)
+    g = np.asarray(gamma32, dtype="<f4").reshape(*zb.shape[:-1], 1).view(np.uint8)
+    return np.concatenate([head, zb, g.reshape(*zb.shape[:-1], 4)], axis=-1)
+
+
+def decode_k_region_qjl(region: np.ndarray, dim: int, bits: int):
+    """(idx, norm float32, z, gamma float32) of a K region written by encode_k_region_qjl."""
+    region = np.asarray(region, dtype=np.uint8)
+    rb = region_bytes(dim, bits)
+    idx, norm = decode_region(region[..., :rb], dim, bits)
+    z = unpack_bits(region[..., rb:rb + dim // 8], dim, 1)
+    g = np.ascontiguousarray(region[..., rb + dim // 8:rb + dim // 8 + 4]).view("<f4")[..., 0]
+    return idx, norm, z, g.astype(np.float32)
+
+
+def dequantize_keys_qjl(idx, norm32, z, gamma32, table: CodebookTable, rot,
+                        qjl_signs: np.ndarray) -> np.ndarray:
+    """k_hat = norm R^T (c[idx] + qjl_correction): the key whose inner product with any q
+    is the QJL-corrected score norm (<R q, c> + gamma sqrt(pi/2)/sqrt(D) <S R q, 2z-1>)."""
+    c = np.asarray(table.centroids, dtype=np.float64)[np.asarray(idx)]
+    w = c + qjl_correction(z, gamma32, qjl_signs)
+    return np.asarray(norm32, dtype=np.float64)[..., None] * rotate_inverse(w, rot)
+
+
+def quantize_append_qjl(pages: np.ndarray, slot_mapping: np.ndarray, k: np.ndarray,
+                        v: np.ndarray, k_table: CodebookTable, v_table: CodebookTable,
+                        sign_seed: int, qjl_seed: int) -> np.ndarray:
+    """quantize_append with the QJL sketch in the K region: slot = [K codes | K norm |
+    sketch bits | gamma][V codes | V norm] (the V region as before)."""
+    pages = np.array(pages, dtype=np.uint8, copy=True)
+    num_blocks, block_size, h_kv, stride = pages.shape
+    t, hk, d = k.shape
+    kb = k_region_bytes(d, k_table.bits, True)
+    vb = region_bytes(d, v_table.bits)
+    assert hk == h_kv and kb + vb <= stride
+    signs = rht_signs(d, sign_seed)
+    ki, kn, kz, kg, _, _ = quantize_keys_qjl(np.asarray(k, dtype=np.float64), signs, k_table,
+                                             rht_signs(d, qjl_seed))
+    vi, vn, _, _ = quantize_rows(np.asarray(v, dtype=np.float64), signs, v_table)
+    kreg = encode_k_region_qjl(ki, kn, kz, kg, k_table.bits)
+    vreg = encode_region(vi, vn, v_table.bits)
+    for tok in range(t):
+        slot = int(slot_mapping[tok])
+        if slot < 0:
+            continue
+        blk, row = slot_position(slot, block_size)
+        pages[blk, row, :, :kb] = kreg[tok]
+        pages[blk, row, :, kb:kb + vb] = vreg[tok]
+    return pages
+
+
+def paged_decode_qjl(q: np.ndarray, pages: np.ndarray, block_table: np.ndarray,
+                     seq_lens: np.ndarray, k_table: CodebookTable, v_table: CodebookTable,
+                     sign_seed: int, qjl_seed: int, scale: float) -> np.ndarray:
+    """paged_decode over slots written by quantize_append_qjl: the keys dequantized with
+    their QJL correction, then plain softmax attention."""
+    q = np.asarray(q, dtype=np.float64)
+    bsz, h_q, d = q.shape
+    h_kv = pages.shape[2]
+    g = h_q // h_kv
+    kb = k_region_bytes(d, k_table.bits, True)
+    vb = region_bytes(d, v_table.bits)
+    signs = rht_signs(d, sign_seed)
+    qs = rht_signs(d, qjl_seed)
+    out = np.zeros((bsz, h_q, d), dtype=np.float64)
+    for b in range(bsz):
+        n = int(seq_lens[b])
+        if n == 0:
+            continue
+        slots = gather_sequence(pages, block_table[b], n)
+        ki, kn, kz, kg = decode_k_region_qjl(slots[..., :kb], d, k_table.bits)
+        vi, vn = decode_region(slots[..., kb:kb + vb], d, v_table.bits)
+        khat = dequantize_keys_qjl(ki, kn, kz, kg, k_table, signs, qs)
+        vhat = dequantize_rows(vi, vn, v_table, signs)
+        for h in range(h_q):
+            kv = h // g
+            s = scale * (khat[:, kv, :] @ q[b, h])
+            p = np.exp(s - np.max(s))
+            out[b, h] = (p / np.sum(p)) @ vhat[:, kv, :]
+    return out

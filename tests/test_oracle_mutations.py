@@ -169,3 +169,10 @@ def test_mutation_haar_without_sign_fix(monkeypatch):
         return np.linalg.qr(np.random.default_rng(seed).standard_normal((dim, dim)))[0]
     monkeypatch.setattr(O, "haar_orthogonal", bad)
     _fails(TR.test_haar_matrix_is_orthogonal_and_the_positive_diagonal_qr, 16)
+
+
+def test_mutation_qjl_constant(monkeypatch):
+    # sqrt(2/pi) in place of sqrt(pi/2): the estimator is biased by 2/pi
+    monkeypatch.setattr(O, "QJL_CONST", math.sqrt(2.0 / math.pi))
+    from tests import test_oracle_qjl as TQ
+    _fails(TQ.test_qjl_estimator_is_unbiased_over_sketch_signs)
