@@ -158,6 +158,12 @@ __host__ __device__ __forceinline__ int64_t cta_begin(int64_t c, int64_t S, int6
 __host__ __device__ __forceinline__ int64_t cta_of(int64_t x, int64_t S, int64_t C) {
   return ((x + 1) * C - 1) / S;
 }
+// Whether CTA c has steps.  Every CTA does when S >= C; callers test that first, and
+// the divisions stay out of line so that they are not executed (predicated off) on
+// that path.
+static __device__ __noinline__ bool cta_has_steps(int64_t c, int64_t S, int64_t C) {
+  return cta_begin(c, S, C) < cta_begin(c + 1, S, C);
+}
 
 template <int D>
 __host__ __device__ constexpr float inv_sqrt_dim() {
@@ -968,9 +974,8 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     }
   };
 
-  auto nonempty = [&](int64_t c) {
-    return S >= Cn || cta_begin(c, S, Cn) < cta_begin(c + 1, S, Cn);
-  };
+  const bool every_cta_busy = S >= Cn;
+  auto nonempty = [&](int64_t c) { return every_cta_busy || cta_has_steps(c, S, Cn); };
   unsigned int* arrived = p.counters;                // records of sequence b written
   unsigned int* merged = p.counters + B;             // covering CTAs done merging b
 
@@ -980,7 +985,7 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   // in batches (contiguous loads) and folded in with an online rescale.
   auto merge_part = [&](int b, int h, int64_t c_lo, int R, int i_first, int i_step, float& M,
                         float& l, float (&o)[E]) {
-    constexpr int NB = 4;                             // records per batch
+    constexpr int NB = E <= 4 ? 8 : 4;                // records per batch
     const int64_t rstride = (int64_t)p.h_q * (D + 2);
     const float* hb = p.part + (int64_t)h * (D + 2);
     M = -INFINITY;
@@ -1041,6 +1046,11 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   // Covering CTAs of sequence b that have records (n) and this CTA's rank among them.
   auto cover = [&](int b, int& n, int& rank) {
     const int64_t c_lo = cta_of(prefix[b], S, Cn), c_hi = cta_of(prefix[b + 1] - 1, S, Cn);
+    if (every_cta_busy) {
+      n = (int)(c_hi - c_lo + 1);
+      rank = (int)((int64_t)blockIdx.x - c_lo);
+      return;
+    }
     n = 0;
     rank = 0;
     for (int64_t c = c_lo; c <= c_hi; ++c)
