@@ -208,7 +208,7 @@ tq_status plan_decode(int batch, int h_q, int h_kv, int dim, int kb, int vb, int
       for (int nst = kMaxStages; nst >= min_st; --nst) {
         const int64_t misc = 16 * nst + 2LL * h_q * dim + 4LL * h_q + 4LL * (batch + 1) +
                              4LL * ids_cap + 4 * 36 + (int64_t)plan->maxw * (dim + 2) * 4 +
-                             4LL * dim + 32 +
+                             4LL * dim + 4LL * batch + 32 +
                              (qjl ? ((int64_t)h_q * qjl_qz_stride(dim) + 15) / 16 * 16 : 0);
         for (int at_top = 0; at_top < 2; ++at_top) {
           const int64_t below = at_top ? low : low - misc;   // room for stages below
@@ -250,9 +250,16 @@ tq_status plan_decode(int batch, int h_q, int h_kv, int dim, int kb, int vb, int
   }
   if (!found) return TQ_ERR_UNSUPPORTED;
   // workspace: merge counters (at the start, so that they can be cleared without
-  // knowing a call's geometry), then the partial records (sized for the widest step)
+  // knowing a call's geometry: per sequence, covering CTAs that published and heads
+  // finished; per (sequence, head), parts finished), the second-level records (a head
+  // split into P = C / (B H_q) parts when there are more CTAs than heads), then the
+  // partial records (sized for the widest step)
+  const int64_t bh = (int64_t)batch * h_q;
+  const int64_t parts = std::max<int64_t>(1, plan->max_ctas / bh);
   plan->counters_off = 0;
-  plan->part_off = align256((size_t)batch * 2 * sizeof(unsigned int));
+  plan->part2_off = align256((size_t)(2 * batch + bh) * sizeof(unsigned int));
+  plan->part_off = plan->part2_off +
+                   align256(parts > 1 ? (size_t)(bh * parts) * (dim + 2) * sizeof(float) : 0);
   plan->ws_bytes = plan->part_off + (size_t)(plan->max_ctas + batch) * wph_max * h_q * (dim + 2) *
                                         sizeof(float);
   return TQ_OK;
@@ -462,6 +469,7 @@ tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tens
   p.misc_off = plan.misc_off;
   p.smem_end = (int32_t)plan.smem;
   p.part = (float*)(ws + plan.part_off);
+  p.part2 = (float*)(ws + plan.part2_off);
   p.counters = (unsigned int*)(ws + plan.counters_off);
   p.wait_ms = kWaitMs;
   p.withhold_cta = -1;
@@ -484,7 +492,7 @@ tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tens
   }
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    ds->counter_bytes = std::max(ds->counter_bytes, plan.part_off);
+    ds->counter_bytes = std::max(ds->counter_bytes, plan.part2_off);
     if (ds->inject_wait_ms > 0) {
       p.wait_ms = ds->inject_wait_ms;
       p.withhold_cta = ds->inject_withhold;

@@ -107,8 +107,10 @@ struct DecodeParams {
   int32_t misc_off;             // barriers, q', prefix sums, block ids, merge scratch
   int32_t smem_end;             // bytes of dynamic shared memory the layout spans
   float* part;                  // records [(C + B) * wph][H_q][D + 2]
-  unsigned int* counters;       // [2][B]: records written, merges done (per sequence);
-                                // zero between calls (the last user of a counter clears it)
+  float* part2;                 // second-level records [B][H_q][P][D + 2] (P > 1 only)
+  unsigned int* counters;       // [B] covering CTAs that published, [B] heads finished,
+                                // [B][H_q] parts finished; zero between calls (the last
+                                // user of a counter clears it)
   unsigned int* err;
   uint32_t wait_ms;             // limit of every bounded wait (milliseconds)
   int32_t withhold_cta;         // test hook: this CTA never announces its records (-1: none)
@@ -341,6 +343,43 @@ __device__ __forceinline__ uint32_t lut_pair2(const uint32_t (&w0)[NW], const ui
     const uint32_t ex = lut_ld(lut_addr<POS, BITS>(w0, off));
     const uint32_t ey = lut_ld(lut_addr<POS, BITS>(w1, off));
     return __byte_perm(ex, ey, 0x5410);              // fp16(c[x]), fp16(c[y])
+  }
+}
+
+// Online fold of `count` partial records into (M, l, o) (one warp; each lane holds E
+// values): load(j, m, l, v) fills record j's reference, sum and this lane's values, or
+// leaves them empty (m = -inf).  Records are read in batches of NB with all loads of a
+// batch in flight together, and folded in with one rescale per batch.
+template <int E, class Load>
+__device__ __forceinline__ void fold_records(int count, const Load& load, float& M, float& l,
+                                             float (&o)[E]) {
+  constexpr int NB = E <= 4 ? 8 : 4;
+  for (int j0 = 0; j0 < count; j0 += NB) {
+    float mj[NB], lj[NB], vj[NB][E];
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      mj[j] = -INFINITY;
+      lj[j] = 0.f;
+#pragma unroll
+      for (int k = 0; k < E; ++k) vj[j][k] = 0.f;
+      if (j0 + j < count) load(j0 + j, mj[j], lj[j], vj[j]);
+    }
+    float mx = M;
+#pragma unroll
+    for (int j = 0; j < NB; ++j) mx = fmaxf(mx, mj[j]);
+    if (mx == -INFINITY) continue;
+    const float f = M == -INFINITY ? 0.f : exp2f(M - mx);
+    l *= f;
+#pragma unroll
+    for (int k = 0; k < E; ++k) o[k] *= f;
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      const float w = mj[j] == -INFINITY ? 0.f : exp2f(mj[j] - mx);
+      l = fmaf(w, lj[j], l);
+#pragma unroll
+      for (int k = 0; k < E; ++k) o[k] = fmaf(w, vj[j][k], o[k]);
+    }
+    M = mx;
   }
 }
 
@@ -633,11 +672,15 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   int32_t* ids = (int32_t*)(prefix + p.batch + 1);     // block ids of the range
   int* wsum = (int*)(ids + p.ids_cap);                 // [32] per-warp sums of the scan
   int* timed_out = wsum + 32;                          // a stage wait of this CTA gave up
-  int* merge_gave_up = timed_out + 1;                  // the current merge wait gave up
+  int* merge_gave_up = timed_out + 1;                  // a merge wait of this CTA gave up
   float* scratch = (float*)(timed_out + 4);            // [warps][D + 2] merge partials
   int* rpos = (int*)(scratch + blockDim.x / 32 * (D + 2));  // [D] coordinate at a record position
+  int32_t* lens = (int32_t*)(rpos + D);                // [B] sequence lengths (0 if rejected)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the first copies need the tensor map: fetch it while the prefix sums run
+  if (tid == 0 && p.copy_mode)
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
   const int gid = lane >> 2, tig = lane & 3;
   auto hot_args = [&]() {
     HotArgs a;
@@ -674,8 +717,10 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
       int steps = 0;
       if (len < 0 || len > p.max_blocks * kBlockSize) {
         if (blockIdx.x == 0) report_error(p.err, TQ_DEVERR_SEQLEN_RANGE);
+        lens[b] = 0;
       } else {
         steps = ((len + kBlockSize - 1) / kBlockSize + wph - 1) / wph;
+        lens[b] = len;
       }
       prefix[b + 1] = steps;
       sum += steps;
@@ -684,7 +729,10 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
       mbar_init(&full[tid], 1);
       released[tid] = 0;
     }
-    if (tid == 0) *timed_out = 0;
+    if (tid == 0) {
+      *timed_out = 0;
+      *merge_gave_up = 0;
+    }
     fence_mbar_init();
     // exclusive scan of the per-thread sums: in each warp, then over the warp totals
     int inc = sum;
@@ -771,7 +819,7 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   auto block_id = [&](int64_t s, int k) -> int32_t {
     const int b = locate(s);
     const int bi = (int)(s - prefix[b]) * wph + k;
-    const int nblk = (p.seq_lens[b] + kBlockSize - 1) / kBlockSize;
+    const int nblk = (lens[b] + kBlockSize - 1) / kBlockSize;
     if (bi >= nblk) return -1;
     const int32_t blk = p.block_table[(int64_t)b * p.bt_stride + bi];
     if (blk < 0 || blk >= p.num_blocks) {
@@ -976,145 +1024,172 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
 
   const bool every_cta_busy = S >= Cn;
   auto nonempty = [&](int64_t c) { return every_cta_busy || cta_has_steps(c, S, Cn); };
-  unsigned int* arrived = p.counters;                // records of sequence b written
-  unsigned int* merged = p.counters + B;             // covering CTAs done merging b
+  unsigned int* arrived = p.counters;                // covering CTAs that published b's records
+  unsigned int* merged = p.counters + B;             // query heads of b finished
+  unsigned int* parts_done = p.counters + 2 * B;     // [B][h_q]: parts of (b, h) finished
+  // Covering CTAs of sequence b (those with records of it) and the first of them.
+  auto covering = [&](int b, int64_t& c_lo) -> int {
+    c_lo = cta_of(prefix[b], S, Cn);
+    const int64_t c_hi = cta_of(prefix[b + 1] - 1, S, Cn);
+    if (every_cta_busy) return (int)(c_hi - c_lo + 1);
+    int n = 0;
+    for (int64_t c = c_lo; c <= c_hi; ++c) n += nonempty(c) ? 1 : 0;
+    return n;
+  };
 
-  // Merge of query head h of sequence b over records i = i_first, i_first + i_step, ...
-  // (record i: CTA c_lo + i / wph, sub-stream i % wph) into this warp's partial
-  // (M, l, and o[k] = O' at record position 2 + lane E + k).  One pass: records are read
-  // in batches (contiguous loads) and folded in with an online rescale.
-  auto merge_part = [&](int b, int h, int64_t c_lo, int R, int i_first, int i_step, float& M,
-                        float& l, float (&o)[E]) {
-    constexpr int NB = E <= 4 ? 8 : 4;                // records per batch
-    const int64_t rstride = (int64_t)p.h_q * (D + 2);
-    const float* hb = p.part + (int64_t)h * (D + 2);
-    M = -INFINITY;
-    l = 0.f;
+  // (M, l) and this lane's E values of a record whose values start at rec + 2 + lane E
+  auto load_record = [&](const float* rec, float& m, float& ll, float (&v)[E]) {
+    const float2 ml = __ldcg((const float2*)rec);
+    m = ml.x;
+    ll = ml.y;
 #pragma unroll
-    for (int k = 0; k < E; ++k) o[k] = 0.f;
-    for (int i0 = i_first; i0 < R; i0 += NB * i_step) {
-      float mj[NB], lj[NB], vj[NB][E];
-#pragma unroll
-      for (int j = 0; j < NB; ++j) {
-        const int i = i0 + j * i_step;
-        const int64_t c = c_lo + i / wph;
-        mj[j] = -INFINITY;
-        lj[j] = 0.f;
-#pragma unroll
-        for (int k = 0; k < E; ++k) vj[j][k] = 0.f;
-        if (i < R && nonempty(c)) {
-          const float* rec = hb + ((c + b) * wph + i % wph) * rstride;
-          const float2 ml = __ldcg((const float2*)rec);
-          mj[j] = ml.x;
-          lj[j] = ml.y;
-#pragma unroll
-          for (int k = 0; k < E / 2; ++k) {
-            const float2 t = __ldcg((const float2*)(rec + 2 + lane * E) + k);
-            vj[j][2 * k] = t.x;
-            vj[j][2 * k + 1] = t.y;
-          }
-        }
-      }
-      float mx = M;
-#pragma unroll
-      for (int j = 0; j < NB; ++j) mx = fmaxf(mx, mj[j]);
-      if (mx == -INFINITY) continue;
-      const float f = M == -INFINITY ? 0.f : exp2f(M - mx);
-      l *= f;
-#pragma unroll
-      for (int k = 0; k < E; ++k) o[k] *= f;
-#pragma unroll
-      for (int j = 0; j < NB; ++j) {
-        const float w = mj[j] == -INFINITY ? 0.f : exp2f(mj[j] - mx);
-        l = fmaf(w, lj[j], l);
-#pragma unroll
-        for (int k = 0; k < E; ++k) o[k] = fmaf(w, vj[j][k], o[k]);
-      }
-      M = mx;
+    for (int k = 0; k < E / 2; ++k) {
+      const float2 t = __ldcg((const float2*)(rec + 2 + lane * E) + k);
+      v[2 * k] = t.x;
+      v[2 * k + 1] = t.y;
     }
   };
 
-  // This CTA is done with sequence b (merged its share, or gave up): the last of the n
-  // covering CTAs to get here clears both of b's counters (ready for the next call).
-  // Every covering CTA has passed its wait by then, so none still reads them.
-  auto release_counters = [&](int b, int n) {
-    if (tid == 0 && atomicAdd(&merged[b], 1u) == (unsigned)n - 1) {
-      atomicExch(&arrived[b], 0u);
-      atomicExch(&merged[b], 0u);
-    }
-  };
-  // Covering CTAs of sequence b that have records (n) and this CTA's rank among them.
-  auto cover = [&](int b, int& n, int& rank) {
-    const int64_t c_lo = cta_of(prefix[b], S, Cn), c_hi = cta_of(prefix[b + 1] - 1, S, Cn);
-    if (every_cta_busy) {
-      n = (int)(c_hi - c_lo + 1);
-      rank = (int)((int64_t)blockIdx.x - c_lo);
-      return;
-    }
-    n = 0;
-    rank = 0;
-    for (int64_t c = c_lo; c <= c_hi; ++c)
-      if (nonempty(c)) {
-        if (c < (int64_t)blockIdx.x) ++rank;
-        ++n;
-      }
-  };
-
-  // End phase for sequence b: once every CTA covering b has written its records, this
-  // CTA (rank k of the n covering CTAs) merges query heads k, k + n, ...: groups of g
-  // warps take one head each, split its records, and the group's first warp combines
-  // the g partials, divides by l and applies o = R^T O' (FWHT, 1/sqrt(D), sign flips).
-  auto coop_merge = [&](int b) {
-    const int64_t c_lo = cta_of(prefix[b], S, Cn), c_hi = cta_of(prefix[b + 1] - 1, S, Cn);
-    int n, rank;
-    cover(b, n, rank);
-    const int R = (int)(c_hi - c_lo + 1) * wph;
-    if (tid == 0) {
-      // wait until all n covering CTAs have arrived (bounded)
+  // Wait (lane 0, bounded) until all n covering CTAs have published sequence b's
+  // records.  After one wait of this CTA has given up, later ones give up at once.
+  auto wait_arrived = [&](int b, int n) -> bool {
+    int ok = 1;
+    if (lane == 0) {
       const uint64_t t0 = globaltimer_ns();
-      int gave_up = 0;
       while (*(volatile unsigned int*)&arrived[b] < (unsigned)n) {
-        if (globaltimer_ns() - t0 > (uint64_t)p.wait_ms * 1000000ull) {
+        if (*(volatile int*)merge_gave_up ||
+            globaltimer_ns() - t0 > (uint64_t)p.wait_ms * 1000000ull) {
           report_error(p.err, TQ_DEVERR_TIMEOUT);
-          gave_up = 1;
+          *(volatile int*)merge_gave_up = 1;
+          ok = 0;
           break;
         }
         __nanosleep(256);
       }
       __threadfence();
-      *merge_gave_up = gave_up;
     }
-    __syncthreads();
-    if (*merge_gave_up) {
-      // some records never arrived: merge nothing, but still count this CTA as done with
-      // the sequence, so that the counters return to zero
-      release_counters(b, n);
-      __syncthreads();
-      return;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  };
+
+  // Output of query head h of sequence b from its merged partial (Mx, L, a), a in
+  // natural coordinate order (lane E + i): o = R^T a / L (the dense rotation, or the
+  // FWHT, 1/sqrt(D) and the sign flips), joined with the hot window's partial when
+  // there is one.  One warp.
+  auto finalize = [&](int b, int h, float Mx, float L, float (&acc_o)[E]) {
+    const int64_t ob = (int64_t)b * p.o_bstride + (int64_t)h * p.o_hstride + lane * E;
+    uint32_t sg[E];                      // sign flips of this lane's output coordinates
+#pragma unroll
+    for (int i = 0; i < E; ++i) sg[i] = sign_mask_at(p.sign_seed, lane * E + i);
+    auto inverse_rotate = [&](float (&a)[E]) {
+      if (EXT && p.rot_hi != nullptr) {
+        float* sc = scratch + warp * (D + 2);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < E; ++i) sc[lane * E + i] = a[i];
+        dense_inverse<E>(p.rot_hi, p.rot_lo, sc, lane);
+#pragma unroll
+        for (int i = 0; i < E; ++i) a[i] = sc[lane * E + i];
+        __syncwarp();
+      } else {
+        warp_fwht<E>(a, lane);
+#pragma unroll
+        for (int i = 0; i < E; ++i)
+          a[i] = __uint_as_float(__float_as_uint(a[i] * inv_sqrt_dim<D>()) ^ sg[i]);
+      }
+    };
+    if (!EXT || p.hot_k == nullptr) {
+      const float inv = L > 0.f ? 1.0f / L : 0.f;
+#pragma unroll
+      for (int i = 0; i < E; ++i) acc_o[i] *= inv;
+      inverse_rotate(acc_o);
+#pragma unroll
+      for (int i = 0; i < E; ++i) store_from_f32(p.out, ob + i, p.out_dtype, acc_o[i]);
+    } else {
+      // R^T O' of the packed tokens (not yet divided by L), then one softmax with the hot
+      // window's partial: rescale both to the larger reference and divide by the joint sum
+      inverse_rotate(acc_o);
+      float* sc = scratch + warp * (D + 2);
+      hot_partial<D>(hot_args(), b, h, lane, sc);
+      const float Mh = sc[0], Lh = sc[1];
+      float oh[E];
+#pragma unroll
+      for (int i = 0; i < E; ++i) oh[i] = sc[2 + lane * E + i];
+      __syncwarp();
+      const float Mt = fmaxf(Mx, Mh);
+      const float f1 = Mx == -INFINITY ? 0.f : exp2f(Mx - Mt);
+      const float f2 = Mh == -INFINITY ? 0.f : exp2f(Mh - Mt);
+      const float Lt = f1 * L + f2 * Lh;
+      const float inv = Lt > 0.f ? 1.0f / Lt : 0.f;
+#pragma unroll
+      for (int i = 0; i < E; ++i)
+        store_from_f32(p.out, ob + i, p.out_dtype, (f1 * acc_o[i] + f2 * oh[i]) * inv);
     }
-    const int nh = rank < p.h_q ? (p.h_q - rank + n - 1) / n : 0;   // heads of this CTA
+  };
+
+  // End phase.  The merge work is dealt out as items (b, h, part): the R = n_b wph
+  // records of query head h of sequence b (n_b covering CTAs) are split into P parts, P
+  // as large as the grid allows (P > 1 only when there are fewer heads than CTAs), and
+  // item i goes to the CTA of rank i mod C' among the C' CTAs with steps, so the merge
+  // spreads over the whole grid instead of the CTAs that happen to cover a sequence.
+  // A CTA's items are taken by groups of g warps (g as large as its item count allows);
+  // each warp folds its share of the item's records, the group's first warp combines
+  // the g partials.  With P = 1 that is the head's output.  With P > 1 the part goes
+  // to a second-level record, and the last part of (b, h) to finish (a counter) folds
+  // the P parts and writes the output, so no part waits for another.  The last head of
+  // b to finish clears b's counters.  `dead`: this CTA gave up a stage wait; its items
+  // are counted (so that the counters return to zero) but not merged.
+  auto end_phase = [&](bool dead) {
+    const int64_t Ce = every_cta_busy ? Cn : S;               // CTAs with steps
+    const int64_t my = every_cta_busy ? (int64_t)blockIdx.x : s0;  // rank among them
+    const int64_t bh = (int64_t)B * p.h_q;
+    const int P = (int)(Ce / bh > 1 ? Ce / bh : 1);
+    const int64_t NI = bh * P;
+    const int m = my < NI ? (int)((NI - my + Ce - 1) / Ce) : 0;
+    if (m == 0) return;
     int g = 1;
-    while (nh > 0 && 2 * g * min(nh, nwarps) <= nwarps) g *= 2;
+    while (2 * g * min(m, nwarps) <= nwarps) g *= 2;
     const int groups = nwarps / g, gi = warp / g, mi = warp % g;
     int nat[E];                          // coordinate at record position 2 + lane E + k
 #pragma unroll
     for (int k = 0; k < E; ++k) nat[k] = rpos[lane * E + k];
-    uint32_t sg[E];
-#pragma unroll
-    for (int i = 0; i < E; ++i) sg[i] = sign_mask_at(p.sign_seed, lane * E + i);
-    for (int j0 = 0; j0 < nh; j0 += groups) {
-      const int j = j0 + gi;
-      const int h = rank + j * n;
-      float M, l, o[E];
-      if (j < nh) {
-        merge_part(b, h, c_lo, R, mi, g, M, l, o);
-        float* sc = scratch + warp * (D + 2);    // natural coordinate order
-        if (lane == 0) { sc[0] = M; sc[1] = l; }
-#pragma unroll
-        for (int i = 0; i < E; ++i) sc[2 + nat[i]] = o[i];
+    const int64_t rstride = (int64_t)p.h_q * (D + 2);
+    const int lw = __ffs(wph) - 1;                   // wph is a power of two
+    for (int k0 = 0; k0 < m; k0 += groups) {
+      const int k = k0 + gi;
+      int b = -1, h = 0, part = 0;
+      if (k < m) {
+        const int64_t i = my + (int64_t)k * Ce;
+        b = (int)(i / ((int64_t)p.h_q * P));
+        h = (int)((i / P) % p.h_q);
+        part = (int)(i % P);
+        if (prefix[b + 1] == prefix[b]) b = -1;        // no steps: output written already
       }
+      float M = -INFINITY, l = 0.f, o[E];
+#pragma unroll
+      for (int i = 0; i < E; ++i) o[i] = 0.f;
+      bool ok = false;
+      if (b >= 0) {
+        int64_t c_lo;
+        const int n = covering(b, c_lo);
+        ok = !dead && wait_arrived(b, n);
+        if (ok) {
+          const int R = (int)((cta_of(prefix[b + 1] - 1, S, Cn) - c_lo + 1) << lw);
+          const int r_lo = (int)((int64_t)R * part / P), r_hi = (int)((int64_t)R * (part + 1) / P);
+          const int cnt = r_hi - r_lo > mi ? (r_hi - r_lo - mi + g - 1) / g : 0;
+          const float* hb = p.part + (int64_t)h * (D + 2);
+          fold_records<E>(cnt, [&](int j, float& mm, float& ll, float (&v)[E]) {
+            const int r = r_lo + mi + j * g;
+            const int64_t c = c_lo + (r >> lw);
+            if (nonempty(c)) load_record(hb + ((c + b) * wph + (r & (wph - 1))) * rstride, mm, ll, v);
+          }, M, l, o);
+        }
+      }
+      float* sc = scratch + warp * (D + 2);              // natural coordinate order
+      if (lane == 0) { sc[0] = M; sc[1] = l; }
+#pragma unroll
+      for (int i = 0; i < E; ++i) sc[2 + nat[i]] = o[i];
       __syncthreads();
-      if (j < nh && mi == 0) {
+      if (b >= 0 && mi == 0) {
         float Mx = -INFINITY;
         for (int w = 0; w < g; ++w) Mx = fmaxf(Mx, scratch[(warp + w) * (D + 2)]);
         float L = 0.f, acc_o[E];
@@ -1122,65 +1197,55 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
         for (int i = 0; i < E; ++i) acc_o[i] = 0.f;
         if (Mx != -INFINITY) {
           for (int w = 0; w < g; ++w) {
-            const float* sc = scratch + (warp + w) * (D + 2);
-            const float mw = sc[0];
+            const float* s2 = scratch + (warp + w) * (D + 2);
+            const float mw = s2[0];
             const float f = mw == -INFINITY ? 0.f : exp2f(mw - Mx);
-            L += f * sc[1];
+            L += f * s2[1];
 #pragma unroll
-            for (int i = 0; i < E; ++i) acc_o[i] = fmaf(f, sc[2 + lane * E + i], acc_o[i]);
+            for (int i = 0; i < E; ++i) acc_o[i] = fmaf(f, s2[2 + lane * E + i], acc_o[i]);
           }
         }
-        const int64_t ob = (int64_t)b * p.o_bstride + (int64_t)h * p.o_hstride + lane * E;
-        // o = R^T a: the dense rotation, or the FWHT, 1/sqrt(D) and the sign flips
-        auto inverse_rotate = [&](float (&a)[E]) {
-          if (EXT && p.rot_hi != nullptr) {
-            float* sc = scratch + warp * (D + 2);
-            __syncwarp();
+        bool last = true;
+        if (P > 1) {
+          // publish this part; the last part of (b, h) to finish folds all P of them
+          float* rec2 = p.part2 + ((int64_t)b * p.h_q + h) * P * (D + 2);
+          float* mine = rec2 + (int64_t)part * (D + 2);
+          if (lane == 0) __stcg((float2*)mine, make_float2(Mx, L));
 #pragma unroll
-            for (int i = 0; i < E; ++i) sc[lane * E + i] = a[i];
-            dense_inverse<E>(p.rot_hi, p.rot_lo, sc, lane);
-#pragma unroll
-            for (int i = 0; i < E; ++i) a[i] = sc[lane * E + i];
-            __syncwarp();
-          } else {
-            warp_fwht<E>(a, lane);
-#pragma unroll
-            for (int i = 0; i < E; ++i)
-              a[i] = __uint_as_float(__float_as_uint(a[i] * inv_sqrt_dim<D>()) ^ sg[i]);
-          }
-        };
-        if (!EXT || p.hot_k == nullptr) {
-          const float inv = L > 0.f ? 1.0f / L : 0.f;
-#pragma unroll
-          for (int i = 0; i < E; ++i) acc_o[i] *= inv;
-          inverse_rotate(acc_o);
-#pragma unroll
-          for (int i = 0; i < E; ++i) store_from_f32(p.out, ob + i, p.out_dtype, acc_o[i]);
-        } else {
-          // R^T O' of the packed tokens (not yet divided by L), then one softmax with
-          // the hot window's partial: rescale both to the larger reference and divide
-          // by the joint sum
-          inverse_rotate(acc_o);
-          float* sc = scratch + warp * (D + 2);
-          hot_partial<D>(hot_args(), b, h, lane, sc);
-          const float Mh = sc[0], Lh = sc[1];
-          float oh[E];
-#pragma unroll
-          for (int i = 0; i < E; ++i) oh[i] = sc[2 + lane * E + i];
+          for (int i = 0; i < E; ++i) __stcg(mine + 2 + lane * E + i, acc_o[i]);
           __syncwarp();
-          const float Mt = fmaxf(Mx, Mh);
-          const float f1 = Mx == -INFINITY ? 0.f : exp2f(Mx - Mt);
-          const float f2 = Mh == -INFINITY ? 0.f : exp2f(Mh - Mt);
-          const float Lt = f1 * L + f2 * Lh;
-          const float inv = Lt > 0.f ? 1.0f / Lt : 0.f;
+          int lst = 0;
+          if (lane == 0) {
+            __threadfence();
+            unsigned int* pc = parts_done + (int64_t)b * p.h_q + h;
+            lst = atomicAdd(pc, 1u) == (unsigned)P - 1;
+            if (lst) {
+              atomicExch(pc, 0u);
+              __threadfence();
+            }
+          }
+          last = __shfl_sync(0xffffffffu, lst, 0) != 0;
+          if (last) {
+            Mx = -INFINITY;
+            L = 0.f;
 #pragma unroll
-          for (int i = 0; i < E; ++i)
-            store_from_f32(p.out, ob + i, p.out_dtype, (f1 * acc_o[i] + f2 * oh[i]) * inv);
+            for (int i = 0; i < E; ++i) acc_o[i] = 0.f;
+            fold_records<E>(P, [&](int j, float& mm, float& ll, float (&v)[E]) {
+              load_record(rec2 + (int64_t)j * (D + 2), mm, ll, v);
+            }, Mx, L, acc_o);
+          }
+        }
+        if (last) {
+          if (ok) finalize(b, h, Mx, L, acc_o);
+          // the last head of b to finish clears b's counters; every wait on them is over
+          if (lane == 0 && atomicAdd(&merged[b], 1u) == (unsigned)p.h_q - 1) {
+            atomicExch(&arrived[b], 0u);
+            atomicExch(&merged[b], 0u);
+          }
         }
       }
       __syncthreads();
     }
-    release_counters(b, n);
   };
 
   // Outer loop: the segments (one per sequence) of this CTA's step range; inner loop:
@@ -1196,7 +1261,7 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   for (int r = 0;;) {
     const int seg_end = (int)(imin64(s1, prefix[cur_b + 1]) - s0);
     // tokens of this warp's block still to come in the sequence
-    int rem = p.seq_lens[cur_b] - ((int)(s0 + r - prefix[cur_b]) * wph + sub) * kBlockSize;
+    int rem = lens[cur_b] - ((int)(s0 + r - prefix[cur_b]) * wph + sub) * kBlockSize;
     start(cur_b, cur_b == b_first);
     for (; r < seg_end; ++r, rem -= wph * kBlockSize) {
       if (!dead && !mbar_wait(&full[x], phase, p.wait_ms)) {
@@ -1430,8 +1495,8 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     if (r >= nsteps) break;
     do ++cur_b; while (prefix[cur_b + 1] == prefix[cur_b]);   // next sequence with steps
   }
-  // end phase: publish the records of every sequence of the range, then merge each
-  // of them together with the other CTAs that cover it
+  // end phase: publish the records of every sequence of the range, then take this
+  // CTA's share of the merge work
   __syncthreads();
   if (tid == 0) {
     __threadfence();
@@ -1439,24 +1504,17 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
       for (int b = b_first; b <= cur_b; ++b)
         if (prefix[b + 1] > prefix[b]) atomicAdd(&arrived[b], 1u);
   }
-  if (*timed_out) {
-    // copies may still be landing in the stages: give them time (bounded), skip the
-    // merge, and count this CTA as done with its sequences (counters back to zero)
+  const bool dead_cta = *(volatile int*)timed_out != 0;
+  if (dead_cta) {
+    // copies may still be landing in the stages: give them time (bounded); this CTA's
+    // merge items are only counted
     if (tid == 0) {
       const uint64_t t0 = globaltimer_ns();
       while (globaltimer_ns() - t0 < 100000000ull) __nanosleep(1000);
     }
     __syncthreads();
-    for (int b = b_first; b <= cur_b; ++b)
-      if (prefix[b + 1] > prefix[b]) {
-        int n, rank;
-        cover(b, n, rank);
-        release_counters(b, n);
-      }
-    return;
   }
-  for (int b = b_first; b <= cur_b; ++b)
-    if (prefix[b + 1] > prefix[b]) coop_merge(b);
+  end_phase(dead_cta);
 }
 
 }  // namespace tq
