@@ -191,15 +191,16 @@ TQ_API tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_
  *   scale        softmax scale (typically 1/sqrt(D)).
  * K and V code widths (cb->k.bits, cb->v.bits): each of 2, 3, 4 and 8, in any pair
  * (TQ_ERR_UNSUPPORTED otherwise; tq_quantize_append takes 1..8).
- * H_q must be a multiple of H_kv with H_q / H_kv <= 16; block_size must be 16.
- * H_kv is at most 16 (8 when D = 256 or H_q / H_kv > 8), and a staged block of all
+ * H_q must be a multiple of H_kv with H_q / H_kv <= 16; block_size must be 16;
+ * B * H_q < 2^31.  H_kv is at most 16 (8 when D = 256 or H_q / H_kv > 8), and a staged block of all
  * KV heads plus the code tables must fit in shared memory: with 8-bit tables that
  * excludes 16 KV heads at D = 128 and 8 at D = 256 (TQ_ERR_UNSUPPORTED;
  * tq_decode_plan_probe tells in advance).
- * One cooperative kernel launch: the CTAs that share a sequence wait for one another
- * (bounded, about 2 s) before merging its partial results.  A wait that gives up raises
- * TQ_DEVERR_TIMEOUT, leaves that sequence's output unwritten, and still returns the
- * merge counters to zero, so the next call runs normally.
+ * One cooperative kernel launch: the merge of a sequence's partial results waits
+ * (bounded, about 2 s) until every CTA that covers the sequence has published its
+ * part; the merge work is spread over all CTAs.  A wait that gives up raises
+ * TQ_DEVERR_TIMEOUT, leaves the affected query heads' output unwritten, and still
+ * returns the merge counters to zero, so the next call runs normally.
  * Uses the per-device workspace (tq_set_workspace, or allocated by the library on
  * the first call that needs more, and kept until process exit).
  * Errors: TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED / TQ_ERR_WORKSPACE (nothing

@@ -338,6 +338,8 @@ tq_status decode_prepare(const tq_tensor& out, const tq_tensor& q, const tq_tens
     return TQ_ERR_INVALID_ARG;
   if (!valid_tensor(seq_lens, 1) || seq_lens.dtype != TQ_I32 || seq_lens.stride[0] != 1)
     return TQ_ERR_INVALID_ARG;
+  // (sequence, query head) pairs are counted in 32 bits
+  if (q.shape[0] * q.shape[1] >= (int64_t)1 << 31) return TQ_ERR_UNSUPPORTED;
   const int B = (int)q.shape[0], h_q = (int)q.shape[1], D = (int)q.shape[2];
   const int h_kv = (int)pages.shape[2];
   for (int i = 0; i < 3; ++i)

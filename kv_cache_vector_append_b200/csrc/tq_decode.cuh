@@ -1027,16 +1027,6 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   unsigned int* arrived = p.counters;                // covering CTAs that published b's records
   unsigned int* merged = p.counters + B;             // query heads of b finished
   unsigned int* parts_done = p.counters + 2 * B;     // [B][h_q]: parts of (b, h) finished
-  // Covering CTAs of sequence b (those with records of it) and the first of them.
-  auto covering = [&](int b, int64_t& c_lo) -> int {
-    c_lo = cta_of(prefix[b], S, Cn);
-    const int64_t c_hi = cta_of(prefix[b + 1] - 1, S, Cn);
-    if (every_cta_busy) return (int)(c_hi - c_lo + 1);
-    int n = 0;
-    for (int64_t c = c_lo; c <= c_hi; ++c) n += nonempty(c) ? 1 : 0;
-    return n;
-  };
-
   // (M, l) and this lane's E values of a record whose values start at rec + 2 + lane E
   auto load_record = [&](const float* rec, float& m, float& ll, float (&v)[E]) {
     const float2 ml = __ldcg((const float2*)rec);
@@ -1055,19 +1045,21 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   auto wait_arrived = [&](int b, int n) -> bool {
     int ok = 1;
     if (lane == 0) {
-      const uint64_t t0 = globaltimer_ns();
-      while (*(volatile unsigned int*)&arrived[b] < (unsigned)n) {
-        if (*(volatile int*)merge_gave_up ||
-            globaltimer_ns() - t0 > (uint64_t)p.wait_ms * 1000000ull) {
-          report_error(p.err, TQ_DEVERR_TIMEOUT);
-          *(volatile int*)merge_gave_up = 1;
-          ok = 0;
-          break;
+      if (ld_acquire(&arrived[b]) < (unsigned)n) {
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire(&arrived[b]) < (unsigned)n) {
+          if (*(volatile int*)merge_gave_up ||
+              globaltimer_ns() - t0 > (uint64_t)p.wait_ms * 1000000ull) {
+            report_error(p.err, TQ_DEVERR_TIMEOUT);
+            *(volatile int*)merge_gave_up = 1;
+            ok = 0;
+            break;
+          }
+          __nanosleep(128);
         }
-        __nanosleep(256);
       }
-      __threadfence();
     }
+    __syncwarp();
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
   };
 
@@ -1139,12 +1131,12 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   // b to finish clears b's counters.  `dead`: this CTA gave up a stage wait; its items
   // are counted (so that the counters return to zero) but not merged.
   auto end_phase = [&](bool dead) {
-    const int64_t Ce = every_cta_busy ? Cn : S;               // CTAs with steps
-    const int64_t my = every_cta_busy ? (int64_t)blockIdx.x : s0;  // rank among them
-    const int64_t bh = (int64_t)B * p.h_q;
-    const int P = (int)(Ce / bh > 1 ? Ce / bh : 1);
-    const int64_t NI = bh * P;
-    const int m = my < NI ? (int)((NI - my + Ce - 1) / Ce) : 0;
+    const int Ce = every_cta_busy ? (int)Cn : (int)S;         // CTAs with steps
+    const int my = every_cta_busy ? (int)blockIdx.x : (int)s0;  // rank among them
+    const int bh = B * p.h_q;                                   // < 2^31 (host check)
+    const int P = Ce / bh > 1 ? Ce / bh : 1;
+    const int NI = bh * P;                                      // <= max(bh, Ce)
+    const int m = my < NI ? (NI - my + Ce - 1) / Ce : 0;
     if (m == 0) return;
     int g = 1;
     while (2 * g * min(m, nwarps) <= nwarps) g *= 2;
@@ -1154,14 +1146,20 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     for (int k = 0; k < E; ++k) nat[k] = rpos[lane * E + k];
     const int64_t rstride = (int64_t)p.h_q * (D + 2);
     const int lw = __ffs(wph) - 1;                   // wph is a power of two
+    // the CTA of step x: 32-bit arithmetic when (x + 1) C fits
+    const bool small = (uint64_t)S * (uint64_t)Cn < (1ull << 32);
+    auto cta_of_step = [&](int64_t x) -> int64_t {
+      return small ? (int64_t)((uint32_t)((x + 1) * Cn - 1) / (uint32_t)S) : cta_of(x, S, Cn);
+    };
     for (int k0 = 0; k0 < m; k0 += groups) {
       const int k = k0 + gi;
       int b = -1, h = 0, part = 0;
       if (k < m) {
-        const int64_t i = my + (int64_t)k * Ce;
-        b = (int)(i / ((int64_t)p.h_q * P));
-        h = (int)((i / P) % p.h_q);
-        part = (int)(i % P);
+        const int i = my + k * Ce;
+        const int hp = i / P;
+        b = hp / p.h_q;
+        h = hp - b * p.h_q;
+        part = i - hp * P;
         if (prefix[b + 1] == prefix[b]) b = -1;        // no steps: output written already
       }
       float M = -INFINITY, l = 0.f, o[E];
@@ -1169,12 +1167,17 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
       for (int i = 0; i < E; ++i) o[i] = 0.f;
       bool ok = false;
       if (b >= 0) {
-        int64_t c_lo;
-        const int n = covering(b, c_lo);
+        const int64_t c_lo = cta_of_step(prefix[b]);
+        const int64_t c_hi = cta_of_step(prefix[b + 1] - 1);
+        int n = (int)(c_hi - c_lo + 1);
+        if (!every_cta_busy) {
+          n = 0;
+          for (int64_t c = c_lo; c <= c_hi; ++c) n += nonempty(c) ? 1 : 0;
+        }
         ok = !dead && wait_arrived(b, n);
         if (ok) {
-          const int R = (int)((cta_of(prefix[b + 1] - 1, S, Cn) - c_lo + 1) << lw);
-          const int r_lo = (int)((int64_t)R * part / P), r_hi = (int)((int64_t)R * (part + 1) / P);
+          const int R = (int)(c_hi - c_lo + 1) << lw;
+          const int r_lo = R * part / P, r_hi = R * (part + 1) / P;
           const int cnt = r_hi - r_lo > mi ? (r_hi - r_lo - mi + g - 1) / g : 0;
           const float* hb = p.part + (int64_t)h * (D + 2);
           fold_records<E>(cnt, [&](int j, float& mm, float& ll, float (&v)[E]) {
@@ -1190,21 +1193,28 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
       for (int i = 0; i < E; ++i) sc[2 + nat[i]] = o[i];
       __syncthreads();
       if (b >= 0 && mi == 0) {
-        float Mx = -INFINITY;
-        for (int w = 0; w < g; ++w) Mx = fmaxf(Mx, scratch[(warp + w) * (D + 2)]);
-        float L = 0.f, acc_o[E];
+        // combine the g partials of the group: lane w < g takes partial w's reference
+        // and sum, the rescale factors go round by shuffles
+        const float* s0w = scratch + (warp + (lane < g ? lane : 0)) * (D + 2);
+        const float mw = lane < g ? s0w[0] : -INFINITY;
+        const float lwv = lane < g ? s0w[1] : 0.f;
+        float Mx = mw;
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) Mx = fmaxf(Mx, __shfl_xor_sync(0xffffffffu, Mx, o2));
+        const float fw = (lane < g && mw != -INFINITY) ? exp2f(mw - Mx) : 0.f;
+        float L = fw * lwv;
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o2);
+        float acc_o[E];
 #pragma unroll
         for (int i = 0; i < E; ++i) acc_o[i] = 0.f;
-        if (Mx != -INFINITY) {
-          for (int w = 0; w < g; ++w) {
-            const float* s2 = scratch + (warp + w) * (D + 2);
-            const float mw = s2[0];
-            const float f = mw == -INFINITY ? 0.f : exp2f(mw - Mx);
-            L += f * s2[1];
+        for (int w = 0; w < g; ++w) {
+          const float f = __shfl_sync(0xffffffffu, fw, w);
+          const float* s2 = scratch + (warp + w) * (D + 2) + 2 + lane * E;
 #pragma unroll
-            for (int i = 0; i < E; ++i) acc_o[i] = fmaf(f, s2[2 + lane * E + i], acc_o[i]);
-          }
+          for (int i = 0; i < E; ++i) acc_o[i] = fmaf(f, s2[i], acc_o[i]);
         }
+        if (Mx == -INFINITY) L = 0.f;
         bool last = true;
         if (P > 1) {
           // publish this part; the last part of (b, h) to finish folds all P of them
@@ -1216,14 +1226,11 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
           __syncwarp();
           int lst = 0;
           if (lane == 0) {
-            __threadfence();
             unsigned int* pc = parts_done + (int64_t)b * p.h_q + h;
-            lst = atomicAdd(pc, 1u) == (unsigned)P - 1;
-            if (lst) {
-              atomicExch(pc, 0u);
-              __threadfence();
-            }
+            lst = atom_add_acq_rel(pc, 1u) == (unsigned)P - 1;
+            if (lst) atomicExch(pc, 0u);
           }
+          __syncwarp();
           last = __shfl_sync(0xffffffffu, lst, 0) != 0;
           if (last) {
             Mx = -INFINITY;
@@ -1236,9 +1243,12 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
           }
         }
         if (last) {
+          // count the head first (the counter's round trip overlaps the output); the
+          // last head of b clears b's counters, every wait on them being over
+          unsigned int done = 0;
+          if (lane == 0) done = atomicAdd(&merged[b], 1u);
           if (ok) finalize(b, h, Mx, L, acc_o);
-          // the last head of b to finish clears b's counters; every wait on them is over
-          if (lane == 0 && atomicAdd(&merged[b], 1u) == (unsigned)p.h_q - 1) {
+          if (lane == 0 && done == (unsigned)p.h_q - 1) {
             atomicExch(&arrived[b], 0u);
             atomicExch(&merged[b], 0u);
           }
@@ -1498,12 +1508,9 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   // end phase: publish the records of every sequence of the range, then take this
   // CTA's share of the merge work
   __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    if ((int)blockIdx.x != p.withhold_cta)
-      for (int b = b_first; b <= cur_b; ++b)
-        if (prefix[b + 1] > prefix[b]) atomicAdd(&arrived[b], 1u);
-  }
+  if (tid == 0 && (int)blockIdx.x != p.withhold_cta)
+    for (int b = b_first; b <= cur_b; ++b)
+      if (prefix[b + 1] > prefix[b]) red_add_release(&arrived[b], 1u);
   const bool dead_cta = *(volatile int*)timed_out != 0;
   if (dead_cta) {
     // copies may still be landing in the stages: give them time (bounded); this CTA's

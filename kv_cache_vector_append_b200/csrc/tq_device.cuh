@@ -208,6 +208,24 @@ __device__ __forceinline__ void report_error(unsigned int* err, unsigned int bit
   if (err) atomicOr(err, bits);
 }
 
+// GPU-scope counters with release / acquire ordering (no separate fence): a release add
+// after a CTA barrier publishes every write the CTA made before the barrier to a reader
+// whose acquire load observes the add.
+__device__ __forceinline__ void red_add_release(unsigned int* p, unsigned int v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned int ld_acquire(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ unsigned int atom_add_acq_rel(unsigned int* p, unsigned int v) {
+  unsigned int old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+
 __device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
 
 }  // namespace tq
