@@ -832,10 +832,6 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   // once (below); the other warps preload the rest of the range meanwhile.
   const int64_t nids = imin64((s1 - s0) * wph, p.ids_cap);
   const int64_t nfirst = imin64((int64_t)nst * wph, nids);
-  if (warp == 0) {
-    for (int64_t i = lane; i < nfirst; i += 32) ids[i] = block_id(s0 + i / wph, (int)(i % wph));
-    __syncwarp();
-  }
   {
     const int first_t = nwarps > 1 ? 32 : 0;          // a lone warp preloads the rest too
     if (tid >= first_t)
@@ -864,8 +860,31 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
       else bulk_g2s(d, p.pages + (int64_t)blk * p.blk_stride, blk_copy_bytes, &full[x]);
     }
   };
-  if (warp == 0)
-    for (int i = 0; i < nst && s0 + i < s1; ++i) refill(s0 + i, i);
+  // The first nst steps: one lane per (stage, block) resolves its block id and issues
+  // its copy, all in one pass (a stage's lanes lie in one 32-lane round: wph divides 32).
+  if (warp == 0) {
+    const int nfs = (int)imin64(nst, s1 - s0);
+    const int lwp = __ffs(wph) - 1;
+    const uint32_t stage_mask = wph >= 32 ? 0xffffffffu : (1u << wph) - 1u;
+    for (int j0 = 0; j0 < nfs * wph; j0 += 32) {
+      const int j = j0 + lane;
+      const int x = j >> lwp, k = j & (wph - 1);
+      const bool in = j < nfs * wph;
+      const int32_t blk = in ? block_id(s0 + x, k) : -1;
+      const uint32_t bits = __ballot_sync(0xffffffffu, blk >= 0);
+      if (in && k == 0) {
+        const uint32_t mask = (bits >> lane) & stage_mask;
+        present[x] = mask;               // published by the arrive (release) below
+        mbar_arrive_expect_tx(&full[x], __popc(mask) * blk_copy_bytes);
+      }
+      __syncwarp();
+      if (blk >= 0) {
+        uint8_t* d = stage_ptr(x) + k * blk_smem;
+        if (p.copy_mode) tensor_g2s_2d(d, &tmap, 0, blk * kBlockSize, &full[x]);
+        else bulk_g2s(d, p.pages + (int64_t)blk * p.blk_stride, blk_copy_bytes, &full[x]);
+      }
+    }
+  }
 
   // tables (they depend on nothing but the centroids) while the copies and the query
   // loads are in flight
@@ -1193,28 +1212,33 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
       for (int i = 0; i < E; ++i) sc[2 + nat[i]] = o[i];
       __syncthreads();
       if (b >= 0 && mi == 0) {
-        // combine the g partials of the group: lane w < g takes partial w's reference
-        // and sum, the rescale factors go round by shuffles
-        const float* s0w = scratch + (warp + (lane < g ? lane : 0)) * (D + 2);
-        const float mw = lane < g ? s0w[0] : -INFINITY;
-        const float lwv = lane < g ? s0w[1] : 0.f;
-        float Mx = mw;
+        float Mx = M, L = l, acc_o[E];
+        if (g == 1) {
 #pragma unroll
-        for (int o2 = 16; o2 > 0; o2 >>= 1) Mx = fmaxf(Mx, __shfl_xor_sync(0xffffffffu, Mx, o2));
-        const float fw = (lane < g && mw != -INFINITY) ? exp2f(mw - Mx) : 0.f;
-        float L = fw * lwv;
+          for (int i = 0; i < E; ++i) acc_o[i] = sc[2 + lane * E + i];
+        } else {
+          // combine the g partials of the group: lane w < g takes partial w's reference
+          // and sum, the rescale factors go round by shuffles
+          const float* s0w = scratch + (warp + (lane < g ? lane : 0)) * (D + 2);
+          const float mw = lane < g ? s0w[0] : -INFINITY;
+          const float lwv = lane < g ? s0w[1] : 0.f;
+          Mx = mw;
 #pragma unroll
-        for (int o2 = 16; o2 > 0; o2 >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o2);
-        float acc_o[E];
+          for (int o2 = 16; o2 > 0; o2 >>= 1) Mx = fmaxf(Mx, __shfl_xor_sync(0xffffffffu, Mx, o2));
+          const float fw = (lane < g && mw != -INFINITY) ? exp2f(mw - Mx) : 0.f;
+          L = fw * lwv;
 #pragma unroll
-        for (int i = 0; i < E; ++i) acc_o[i] = 0.f;
-        for (int w = 0; w < g; ++w) {
-          const float f = __shfl_sync(0xffffffffu, fw, w);
-          const float* s2 = scratch + (warp + w) * (D + 2) + 2 + lane * E;
+          for (int o2 = 16; o2 > 0; o2 >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o2);
 #pragma unroll
-          for (int i = 0; i < E; ++i) acc_o[i] = fmaf(f, s2[i], acc_o[i]);
+          for (int i = 0; i < E; ++i) acc_o[i] = 0.f;
+          for (int w = 0; w < g; ++w) {
+            const float f = __shfl_sync(0xffffffffu, fw, w);
+            const float* s2 = scratch + (warp + w) * (D + 2) + 2 + lane * E;
+#pragma unroll
+            for (int i = 0; i < E; ++i) acc_o[i] = fmaf(f, s2[i], acc_o[i]);
+          }
+          if (Mx == -INFINITY) L = 0.f;
         }
-        if (Mx == -INFINITY) L = 0.f;
         bool last = true;
         if (P > 1) {
           // publish this part; the last part of (b, h) to finish folds all P of them
