@@ -36,7 +36,7 @@
 //   * S^T = K~ . Qhat^T on mma.sync m16n8k16 (M = 16 tokens, N = 8 query heads of the
 //     group, K = D; fp16 operands, fp32 accumulation); s = acc * nK * |q'| * scale * log2 e;
 //   * online softmax in base 2 against a running reference M >= max(s + e(nV)),
-//     e(x) = floor(log2 x) + 1 read from the exponent bits, raised only when a tile
+//     e(x) = log2 x + 1 from the hardware logarithm (an upper bound), raised only when a tile
 //     exceeds it by more than 2^8 (lazy rescale), so the fp16 weights
 //     P~ = 2^(s - M) nV stay below 2^9 whatever the V norms;
 //   * O'^T += V~^T . P~^T on mma.sync (M = coordinates, N = query heads, K = tokens);
@@ -408,12 +408,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// floor(log2 x) + 1 for x > 0 (exponent bits; an upper bound of log2 x within 1),
-// -126 for zero or subnormal x, NaN for NaN.
-__device__ __forceinline__ float log2_ceilish(float x) {
-  const uint32_t e = (__float_as_uint(x) >> 23) & 0xFFu;
-  const float f = __uint_as_float(0x4B000000u | e) - 8388608.0f;   // exact small integer
-  return x != x ? x : f - 126.0f;
+// An upper bound of log2 x within about 1 for x > 0: the hardware base-2 logarithm
+// (absolute error far below 1) plus 1; -inf for zero or subnormal x (flushed), NaN for
+// NaN.
+__device__ __forceinline__ float log2_bound(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y + 1.0f;
 }
 
 // In-warp FWHT of D = 32 E values, lane l holding coordinates l E .. l E + E - 1
@@ -1395,7 +1396,7 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
           // masked tokens may hold stale norms (even NaN): their V norm is taken as 0
           nV[r] = ok[r] ? *(const float*)(sl + p.k_region + C::VPACK) : 0.f;
           // floor at 2^-100 keeps 2^(s - M) finite for rows of (near) zero V norm
-          eV[r] = fmaxf(log2_ceilish(nV[r]), -100.0f);
+          eV[r] = fmaxf(log2_bound(nV[r]), -100.0f);
         }
         uint32_t pb[NH][2];   // [head group][b0b1 | b2b3]
   #pragma unroll
