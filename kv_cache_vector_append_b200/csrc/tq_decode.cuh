@@ -283,6 +283,21 @@ __device__ __forceinline__ void lut_build(uint8_t* lut, const float* c, int tid,
   }
 }
 
+// Table of 2-bit V codes taken four at a time (used where the V codes are read
+// interleaved): entry q = a | a' << 2 | b << 4 | b' << 6, the codes of two coordinates
+// (a, a' of token A; b, b' of token B), holds {half2(c[a], c[b]), half2(c[a'], c[b'])},
+// the A-fragment registers of one m-tile's rows g and g + 8.  The V half of row q holds
+// 16 copies of the 8-byte entry; lane l reads copy l % 16 (an 8-byte load is served in
+// two 16-lane phases, so a warp's lookups never conflict).
+__device__ __forceinline__ void lut_build_vquad(uint8_t* lut, const float* c, int tid, int nt) {
+  for (int i = tid; i < 256 * 16; i += nt) {
+    const int e = i >> 4, cp = i & 15;
+    const uint32_t lo = pack_half2(c[e & 3], c[(e >> 4) & 3]);
+    const uint32_t hi = pack_half2(c[(e >> 2) & 3], c[e >> 6]);
+    *(uint2*)(lut + e * kLutRow + 128 + 8 * cp) = make_uint2(lo, hi);
+  }
+}
+
 // Shared-window address (e << 8) | off of the entry e held in the field of LEN bits at
 // bit POS of the word array; `off` is lut_win | the lane's column (4 lane, + 128 for
 // the V table).
@@ -314,6 +329,12 @@ __device__ __forceinline__ uint32_t lut_addr1(uint32_t w, uint32_t off) {
 __device__ __forceinline__ uint32_t lut_ld(uint32_t addr) {
   uint32_t v;
   asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+// Two table words (an 8-byte entry) at shared-window address addr.
+__device__ __forceinline__ uint2 lut_ld2(uint32_t addr) {
+  uint2 v;
+  asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
 }
 
@@ -646,6 +667,8 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   using KS = typename C::KS;
   using VS = typename C::VS;
   constexpr int E = D / 32;
+  // 2-bit V codes read interleaved are looked up four at a time (lut_build_vquad)
+  constexpr bool VQUAD = VS::kInterleaved && VB == 2;
   extern __shared__ __align__(16) uint8_t smem[];
   {
     // the layout planned on the host must match this launch: tables at lut_win and
@@ -890,7 +913,8 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   // tables (they depend on nothing but the centroids) while the copies and the query
   // loads are in flight
   lut_build<KB, 0>(smem + p.lut_off, p.kc, tid, nthreads);
-  lut_build<VB, 1>(smem + p.lut_off, p.vc, tid, nthreads);
+  if constexpr (VQUAD) lut_build_vquad(smem + p.lut_off, p.vc, tid, nthreads);
+  else lut_build<VB, 1>(smem + p.lut_off, p.vc, tid, nthreads);
   // coordinate held at each record position 2 + i (the fragment order; see flush)
   for (int i = tid; i < D; i += nthreads) {
     const int g = i & 7, m = i >> 3;
@@ -901,7 +925,8 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   const int kvh = warp % p.h_kv;
   const int sub = warp / p.h_kv;
   const int G = p.group;
-  const uint32_t lk_off = p.lut_win | (4u * lane), lv_off = p.lut_win | (128u + 4u * lane);
+  const uint32_t lk_off = p.lut_win | (4u * lane);
+  const uint32_t lv_off = p.lut_win | (VQUAD ? 128u + 8u * (lane & 15) : 128u + 4u * lane);
 
   // per warp: q fragments (B operand of the score product), softmax state, O'^T
   uint32_t qb[C::KSTEPS][NH][2];
@@ -1471,7 +1496,28 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
             const int t = 2 * tig + (i & 1) + 8 * (i >> 1);
             VS::load(vw[i], base + t * pitch + p.k_region, gid);
           }
-          if constexpr (VS::kInterleaved && (VB == 4 || VB == 2)) {
+          if constexpr (VQUAD) {
+            // regroup the 2-bit codes of tokens A/B and C/D by nibble: byte n of lo
+            // holds nibble 2n of the first token's word and of the second's, byte n of hi
+            // nibble 2n + 1; nibble k (codes 2k, 2k + 1) is m-tile k of the word, one
+            // quad lookup giving its rows g and g + 8
+            static_for<VS::NW>([&](auto JI) {
+              constexpr int j = decltype(JI)::value;
+              const uint32_t loAB = (vw[0][j] & 0x0F0F0F0Fu) | ((vw[1][j] << 4) & 0xF0F0F0F0u);
+              const uint32_t hiAB = ((vw[0][j] >> 4) & 0x0F0F0F0Fu) | (vw[1][j] & 0xF0F0F0F0u);
+              const uint32_t loCD = (vw[2][j] & 0x0F0F0F0Fu) | ((vw[3][j] << 4) & 0xF0F0F0F0u);
+              const uint32_t hiCD = ((vw[2][j] >> 4) & 0x0F0F0F0Fu) | (vw[3][j] & 0xF0F0F0F0u);
+              static_for<8>([&](auto KI) {
+                constexpr int k = decltype(KI)::value;
+                constexpr int mt = j * 8 + k;
+                const uint2 ab = lut_ld2(lut_addr1<8 * (k >> 1), 8>((k & 1) ? hiAB : loAB, lv_off));
+                const uint2 cd = lut_ld2(lut_addr1<8 * (k >> 1), 8>((k & 1) ? hiCD : loCD, lv_off));
+  #pragma unroll
+                for (int hh = 0; hh < NH; ++hh)
+                  mma_16816(acc[hh][mt], ab.x, ab.y, cd.x, cd.y, pb[hh][0], pb[hh][1]);
+              });
+            });
+          } else if constexpr (VS::kInterleaved && (VB == 4 || VB == 2)) {
             // transpose the code nibbles (or crumbs) of tokens A/B and C/D into pair
             // indices: lo holds the even codes of a word, hi the odd ones
             constexpr uint32_t M1 = VB == 4 ? 0x0F0F0F0Fu : 0x33333333u;

@@ -142,7 +142,9 @@ inline tq_status launch_decode_any(int dim, int kb, int vb, const DecodeParams& 
 
 // Bytes of the lookup tables of the decode kernel (one 256-byte row per entry).
 inline size_t decode_lut_bytes(int kb, int vb) {
-  return (size_t)std::max(lut_entries(kb), lut_entries(vb)) * kLutRow;
+  // 2-bit V codes are looked up four at a time (256 entries) where they are read
+  // interleaved; the table is sized for that whatever the head dimension
+  return (size_t)std::max(lut_entries(kb), vb == 2 ? 256 : lut_entries(vb)) * kLutRow;
 }
 
 }  // namespace tq
