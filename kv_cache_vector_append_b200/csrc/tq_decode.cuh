@@ -579,24 +579,35 @@ __device__ __forceinline__ void hot_partial_t(const HotArgs& a, int b, int h, in
   const T* hv = (const T*)a.hot_v;
   const int64_t base = (int64_t)b * a.hot_bstride + (int64_t)(h / a.group) * a.hot_hstride +
                        lane * E;
-  for (int t0 = 0; t0 < n; t0 += 4) {          // four tokens: independent reductions
-    float dot[4];
+  // TPI tokens an iteration, their K and V rows all loaded at its top (one round trip
+  // to memory per iteration); independent reductions
+  constexpr int TPI = E <= 4 ? 8 : 4;
+  for (int t0 = 0; t0 < n; t0 += TPI) {
+    float kx[TPI][E], vx[TPI][E];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      dot[j] = 0.f;
-      if (t0 + j < n) {
-        const int64_t off = base + (int64_t)(t0 + j) * a.hot_tstride;
+    for (int j = 0; j < TPI; ++j) {
+      const bool in = t0 + j < n;
+      const int64_t off = base + (int64_t)(in ? t0 + j : 0) * a.hot_tstride;
 #pragma unroll
-        for (int i = 0; i < E; ++i) dot[j] = fmaf(qv[i], as_f32(hk[off + i]), dot[j]);
+      for (int i = 0; i < E; ++i) {
+        kx[j][i] = in ? as_f32(hk[off + i]) : 0.f;
+        vx[j][i] = in ? as_f32(hv[off + i]) : 0.f;
       }
+    }
+    float dot[TPI];
+#pragma unroll
+    for (int j = 0; j < TPI; ++j) {
+      dot[j] = 0.f;
+#pragma unroll
+      for (int i = 0; i < E; ++i) dot[j] = fmaf(qv[i], kx[j][i], dot[j]);
     }
 #pragma unroll
     for (int m = 16; m > 0; m >>= 1)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) dot[j] += __shfl_xor_sync(0xffffffffu, dot[j], m);
+      for (int j = 0; j < TPI; ++j) dot[j] += __shfl_xor_sync(0xffffffffu, dot[j], m);
     float mx = M;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < TPI; ++j) {
       dot[j] = t0 + j < n ? dot[j] * a.scale_log2 : -INFINITY;
       mx = fmaxf(mx, dot[j]);
     }
@@ -608,13 +619,12 @@ __device__ __forceinline__ void hot_partial_t(const HotArgs& a, int b, int h, in
       M = mx;
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < TPI; ++j) {
       if (t0 + j < n) {
         const float w = exp2f(dot[j] - M);
-        const int64_t off = base + (int64_t)(t0 + j) * a.hot_tstride;
         L += w;
 #pragma unroll
-        for (int i = 0; i < E; ++i) o[i] = fmaf(w, as_f32(hv[off + i]), o[i]);
+        for (int i = 0; i < E; ++i) o[i] = fmaf(w, vx[j][i], o[i]);
       }
     }
   }
