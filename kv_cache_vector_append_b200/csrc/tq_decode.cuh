@@ -485,35 +485,43 @@ __device__ __forceinline__ void rot_row_part(const uint16_t* hi, const uint16_t*
   }
 }
 
-// sc[0 .. D) <- R sc[0 .. D) for one warp (sc: this warp's shared scratch).  Output c is
-// the warp sum of the lanes' partial dot products with row c of R (fp32).  Out of line,
-// so that it leaves the register allocation of the caller's step loop alone.
+// sc[0 .. D) <- R sc[0 .. D) for one warp (sc: this warp's shared scratch).  Rounds of
+// 16 outputs: every lane loads its E columns of the 16 rows (all loads of a round in
+// flight together) and forms its 16 partial dot products; a reduce-scatter over the lane
+// bits 3..0 (lane l keeps output l mod 16, 15 shuffles) and one more over bit 4 sum
+// them over the warp in fp32.  Out of line, so that it leaves the register allocation of
+// the caller's step loop alone.
 template <int E>
 __device__ __noinline__ void dense_forward(const uint16_t* hi, const uint16_t* lo, float* sc,
                                            int lane) {
   constexpr int D = 32 * E;
+  constexpr int CH = 16;
   float x[E];
 #pragma unroll
   for (int i = 0; i < E; ++i) x[i] = sc[lane * E + i];
   __syncwarp();
-  for (int c = 0; c < D; c += 4) {            // four independent reductions at a time
-    float part[4];
+  for (int c0 = 0; c0 < D; c0 += CH) {
+    float p[CH];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < CH; ++j) {
       float r[E];
-      rot_row_part<E>(hi, lo, c + j, lane, r);
-      part[j] = 0.f;
+      rot_row_part<E>(hi, lo, c0 + j, lane, r);
+      p[j] = 0.f;
 #pragma unroll
-      for (int i = 0; i < E; ++i) part[j] = fmaf(r[i], x[i], part[j]);
+      for (int i = 0; i < E; ++i) p[j] = fmaf(r[i], x[i], p[j]);
     }
 #pragma unroll
-    for (int m = 16; m > 0; m >>= 1)
+    for (int m = CH / 2; m > 0; m >>= 1) {
+      const bool up = (lane & m) != 0;      // keep outputs [m, 2m) of the current set
 #pragma unroll
-      for (int j = 0; j < 4; ++j) part[j] += __shfl_xor_sync(0xffffffffu, part[j], m);
-    if (lane == 0) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) sc[c + j] = part[j];
+      for (int j = 0; j < m; ++j) {
+        const float keep = up ? p[j + m] : p[j];
+        const float send = up ? p[j] : p[j + m];
+        p[j] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+      }
     }
+    const float out = p[0] + __shfl_xor_sync(0xffffffffu, p[0], 16);
+    if (lane < CH) sc[c0 + lane] = out;
   }
   __syncwarp();
 }
@@ -528,6 +536,7 @@ __device__ __noinline__ void dense_inverse(const uint16_t* hi, const uint16_t* l
 #pragma unroll
   for (int i = 0; i < E; ++i) a[i] = 0.f;
   __syncwarp();
+#pragma unroll 16
   for (int j = 0; j < D; ++j) {
     float r[E];
     rot_row_part<E>(hi, lo, j, lane, r);
