@@ -59,7 +59,7 @@ struct DenseAppendMaps {
 };
 
 constexpr int kDenseRows = 128;      // pairs per tile (the MMA's M)
-constexpr int kDenseThreads = 256;   // 8 warps
+constexpr int kDenseThreads = 512;   // 16 warps: (row quarter, kind, column half)
 
 // ---------------------------------------------------------------------------
 // tcgen05 / tensor memory wrappers (cta_group::1, no multicast)
@@ -230,9 +230,16 @@ struct DenseSmem {
   static __host__ __device__ constexpr int slot_words(int kbits, int vbits) {
     return (D * kbits / 8 + 4 + D * vbits / 8 + 4) / 4;
   }
+  // words of the slot area: the tile's slots, and at least the norm pass's half-row
+  // exchange ([2][2][128] u32 pairs)
+  static __host__ __device__ constexpr int slot_area_words(int kbits, int vbits) {
+    return kDenseRows * slot_words(kbits, vbits) > 2 * 2 * kDenseRows * 2
+               ? kDenseRows * slot_words(kbits, vbits)
+               : 2 * 2 * kDenseRows * 2;
+  }
   // [R hi | R lo | nst stages] (1024-aligned), tables, slots, slot offsets, misc
   static __host__ __device__ constexpr int bytes(int kbits, int vbits, int nst) {
-    return 1024 + 2 * ROT + nst * STAGE + TABLES + kDenseRows * slot_words(kbits, vbits) * 4 +
+    return 1024 + 2 * ROT + nst * STAGE + TABLES + slot_area_words(kbits, vbits) * 4 +
            kDenseRows * 8 + 64;
   }
 };
@@ -249,17 +256,25 @@ append_dense_kernel(DenseAppendParams p, const __grid_constant__ DenseAppendMaps
   EncodeTables* tabs = (EncodeTables*)(stage_s + p.nst * SM::STAGE);
   const int swords = SM::slot_words(p.bits[0], p.bits[1]);
   uint32_t* slots_s = (uint32_t*)((uint8_t*)tabs + SM::TABLES);   // [128][swords]
-  int64_t* dst_s = (int64_t*)(slots_s + kDenseRows * swords);
-  uint64_t* bars = (uint64_t*)(dst_s + kDenseRows);        // full[2], mma_done
-  uint32_t* tmem_slot = (uint32_t*)(bars + 3);
+  int64_t* dst_s = (int64_t*)(slots_s + SM::slot_area_words(p.export_mode ? 1 : p.bits[0],
+                                                              p.export_mode ? 1 : p.bits[1]));
+  uint64_t* bars = (uint64_t*)(dst_s + kDenseRows);        // full[2], mma_done[2]
+  uint32_t* tmem_slot = (uint32_t*)(bars + 4);
   int* flags = (int*)(tmem_slot + 1);                       // fast[2], dead
+  // half-row sums of squares and maxima [kind][half][row] (ss, max |x| bits), in the slot
+  // area while it is free (the norm pass, before the epilogue writes the slots)
+  uint2* half_norm = (uint2*)slots_s;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int kind = warp >> 2;                               // epilogue kind of this warp
+  const int kind = (warp >> 2) & 1;                        // epilogue kind of this warp
+  const int half = warp >> 3;                               // its half of the columns
   const int row = ((warp & 3) << 5) | lane;                 // epilogue row (TMEM lane)
   const int kwords = (D * p.bits[0] + 7) / 8 / 4 + 1;
   const int64_t npairs = p.num_tokens * p.h_kv;
   const int64_t ntiles = (npairs + kDenseRows - 1) / kDenseRows;
-  const uint32_t ncols = 2 * D;                             // K and V accumulators
+  // Two input stages and, where tensor memory holds two sets of accumulators (4 D <= 512
+  // columns), a pipelined loop: the next tile's MMAs run while this tile's epilogue does.
+  const bool pipe = p.nst == 2 && 4 * D <= 512;
+  const uint32_t ncols = pipe ? 4 * D : 2 * D;              // K and V accumulators (x2)
 
   // rotation into shared memory (16-byte pieces: 8 consecutive k of one row j)
   for (int i = tid; i < 2 * D * D / 8; i += blockDim.x) {
@@ -276,6 +291,7 @@ append_dense_kernel(DenseAppendParams p, const __grid_constant__ DenseAppendMaps
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
     mbar_init(&bars[2], 1);
+    mbar_init(&bars[3], 1);
     flags[2] = 0;
     fence_mbar_init();
   }
@@ -302,60 +318,29 @@ append_dense_kernel(DenseAppendParams p, const __grid_constant__ DenseAppendMaps
         tensor_g2s_3d(stage_s + b * SM::STAGE + k * SM::KIND + blk * kDenseRows * 128,
                       k ? &maps.v : &maps.k, 64 * blk, h0, t0, &bars[b]);
   };
-  const int64_t first = blockIdx.x;
-  const int nst = p.nst;
-  // copies issued but not yet consumed (thread 0): their stage and completion parity
-  int pend_b = -1;
-  uint32_t pend_par = 0;
-  if (tid == 0 && first < ntiles) {
-    load_tile(first, 0);
-    pend_b = 0;
-    pend_par = 0;
-  }
-  __syncthreads();
-
-  uint32_t it = 0;
-  for (int64_t tile = first; tile < ntiles; tile += gridDim.x, ++it) {
-    const int b = nst == 2 ? (int)(it & 1) : 0;
-    const uint32_t full_parity = nst == 2 ? (it >> 1) & 1u : it & 1u;
-    const int64_t r0 = tile * kDenseRows;
-    const int nr = (int)imin64(kDenseRows, npairs - r0);
-    uint8_t* st = stage_s + b * SM::STAGE;
-    if (tid == 0) {
-      // the MMAs of this tile once its rows have landed
-      if (!mbar_wait(&bars[b], full_parity, p.wait_ms)) {
-        report_error(p.err, TQ_DEVERR_TIMEOUT);
-        flags[2] = 1;
-      } else {
-        pend_b = -1;
-        tc_fence_after();
-        const uint32_t idesc = dense_idesc(D);
+  // the MMAs of the tile staged in stage b into accumulator set a (tensor memory columns
+  // [a 2D, a 2D + 2D)), committed to mma_done[a] (thread 0)
+  auto issue_mma = [&](int b, int a) {
+    const uint8_t* st = stage_s + b * SM::STAGE;
+    const uint32_t idesc = dense_idesc(D);
 #pragma unroll 1
-        for (int k = 0; k < (p.export_mode ? 1 : 2); ++k) {
-          const uint32_t a0 = smem_u32(st + k * SM::KIND);
+    for (int k = 0; k < (p.export_mode ? 1 : 2); ++k) {
+      const uint32_t a0 = smem_u32(st + k * SM::KIND);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t aoff = (ks >> 2) * (kDenseRows * 128) + (ks & 3) * 32;
-            const uint32_t boff = (ks >> 2) * (D * 128) + (ks & 3) * 32;
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t aoff = (ks >> 2) * (kDenseRows * 128) + (ks & 3) * 32;
+        const uint32_t boff = (ks >> 2) * (D * 128) + (ks & 3) * 32;
 #pragma unroll
-            for (int part = 0; part < 2; ++part)
-              umma_bf16(tmem + k * D, sw128_desc(a0 + aoff),
-                        sw128_desc(smem_u32(rot_s + part * SM::ROT) + boff), idesc,
-                        (ks > 0 || part > 0) ? 1u : 0u);
-          }
-        }
-        umma_commit(&bars[2]);
-        // with two stages the next tile's rows come in meanwhile (its stage was freed at
-        // the end of the previous tile)
-        if (nst == 2 && tile + gridDim.x < ntiles) {
-          load_tile(tile + gridDim.x, b ^ 1);
-          pend_b = b ^ 1;
-          pend_par = ((it + 1) >> 1) & 1u;
-        }
+        for (int part = 0; part < 2; ++part)
+          umma_bf16(tmem + (uint32_t)(a * 2 * D + k * D), sw128_desc(a0 + aoff),
+                    sw128_desc(smem_u32(rot_s + part * SM::ROT) + boff), idesc,
+                    (ks > 0 || part > 0) ? 1u : 0u);
       }
     }
-    __syncwarp();
-    // slot offsets of the tile's pairs
+    umma_commit(&bars[2 + a]);
+  };
+  // slot offsets of the tile's pairs (threads 0 .. 127)
+  auto slot_offsets = [&](int64_t r0, int nr) {
     if (tid < kDenseRows) {
       int64_t off = -1;
       if (tid < nr && !p.export_mode) {
@@ -374,39 +359,49 @@ append_dense_kernel(DenseAppendParams p, const __grid_constant__ DenseAppendMaps
       }
       dst_s[tid] = off;
     }
-    // the staged rows are read below: every thread waits for the tile's copies (thread 0
-    // has already waited for them before issuing the MMAs)
-    if (tid != 0 && !mbar_wait(&bars[b], full_parity, p.wait_ms)) {
-      report_error(p.err, TQ_DEVERR_TIMEOUT);
-      flags[2] = 1;
-    }
-    // the row's norm from the staged input (plain fp32 sum of squares in k order)
-    const bool active = !(p.export_mode && kind == 1);
-    const uint8_t* xblk = st + kind * SM::KIND;
-    float ss = 0.f;
-    uint32_t mx = 0u;
+  };
+  // Per-thread row state of the tile's norm pass.
+  struct RowNorm {
+    float ss, n, r, norm;
+    uint32_t mx;
+    int e;
+    bool bad, in_range;
+  };
+  const bool active = !(p.export_mode && kind == 1);
+  // the row's norm from the staged input (plain fp32 sum of squares in k order)
+  auto norm_pass = [&](const uint8_t* xblk) -> RowNorm {
+    RowNorm q;
+    q.ss = 0.f;
+    q.mx = 0u;
     if (active) {
 #pragma unroll 4
-      for (int c = 0; c < D / 8; ++c) {
-        const uint4 q = *(const uint4*)(xblk + sw128_offset(row, 8 * c, kDenseRows));
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+      for (int c = half * (D / 16); c < (half + 1) * (D / 16); ++c) {
+        const uint4 v = *(const uint4*)(xblk + sw128_offset(row, 8 * c, kDenseRows));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float lo = bf16_bits_to_f32(w[i] & 0xffffu), hi = __uint_as_float(w[i] & 0xffff0000u);
-          ss = fmaf(lo, lo, ss);
-          ss = fmaf(hi, hi, ss);
-          mx = max(mx, max((w[i] << 16) & 0x7fffffffu, w[i] & 0x7fff0000u));
+          q.ss = fmaf(lo, lo, q.ss);
+          q.ss = fmaf(hi, hi, q.ss);
+          q.mx = max(q.mx, max((w[i] << 16) & 0x7fffffffu, w[i] & 0x7fff0000u));
         }
       }
     }
-    const bool bad = mx >= 0x7f800000u;
-    const bool in_range = ss >= 0x1p-60f && ss <= 0x1p100f;
-    int e = 0;
-    float n = sqrtf(ss);
-    if (active && !in_range && !bad && mx != 0u) {
+    // the row's two halves (this thread's and the one of warp ^ 8): half 0's sum comes first
+    half_norm[(kind * 2 + half) * kDenseRows + row] = make_uint2(__float_as_uint(q.ss), q.mx);
+    __syncthreads();
+    const uint2 o = half_norm[(kind * 2 + (half ^ 1)) * kDenseRows + row];
+    __syncthreads();                    // the slot area is written by the epilogue next
+    q.ss = half ? __fadd_rn(__uint_as_float(o.x), q.ss) : __fadd_rn(q.ss, __uint_as_float(o.x));
+    q.mx = max(q.mx, o.y);
+    q.bad = q.mx >= 0x7f800000u;
+    q.in_range = q.ss >= 0x1p-60f && q.ss <= 0x1p100f;
+    q.e = 0;
+    q.n = sqrtf(q.ss);
+    if (active && !q.in_range && !q.bad && q.mx != 0u) {
       // scaled sum of squares: the largest magnitude brought into [1, 2) (exact)
-      e = exponent_of(mx);
-      const float s1 = pow2f(-e / 2), s2 = pow2f(-e - (-e / 2));
+      q.e = exponent_of(q.mx);
+      const float s1 = pow2f(-q.e / 2), s2 = pow2f(-q.e - (-q.e / 2));
       float ss2 = 0.f;
       for (int k = 0; k < D; ++k) {
         const float x = __fmul_rn(
@@ -415,56 +410,53 @@ append_dense_kernel(DenseAppendParams p, const __grid_constant__ DenseAppendMaps
             s2);
         ss2 = fmaf(x, x, ss2);
       }
-      n = sqrtf(ss2);
+      q.n = sqrtf(ss2);
     }
-    const float r = n > 0.f ? __frcp_rn(n) : 0.f;
-    const float norm = e == 0 ? n : __fmul_rn(__fmul_rn(n, pow2f(e / 2)), pow2f(e - e / 2));
-    // the accumulators (every thread waits; a launch that stopped never completes them)
-    const bool acc_ok = mbar_wait(&bars[2], it & 1u, p.wait_ms);
-    if (!acc_ok) {
-      if (tid == 0) report_error(p.err, TQ_DEVERR_TIMEOUT);
-      flags[2] = 1;
-    }
-    __syncwarp();
-    tc_fence_after();
+    q.r = q.n > 0.f ? __frcp_rn(q.n) : 0.f;
+    q.norm = q.e == 0 ? q.n : __fmul_rn(__fmul_rn(q.n, pow2f(q.e / 2)), pow2f(q.e - q.e / 2));
+    return q;
+  };
+  // epilogue of the tile (staged rows xblk, accumulator set a): u = y r, encode and pack
+  // into the slots in shared memory (or, in export mode, write u and n)
+  auto epilogue = [&](const uint8_t* xblk, int a, int64_t r0, int nr, const RowNorm& q) {
     const int bits = p.bits[kind];
     const int rwords = kind ? swords - kwords : kwords;
     uint32_t* orow = slots_s + row * swords + (kind ? kwords : 0);
-    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(kind * D);
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(a * 2 * D + kind * D);
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
       float y[32];
       tmem_ld32(tl + 32 * c, y);             // every thread of the warp takes part
-      if (active && !in_range && !bad && mx != 0u) {
-        const float s1 = pow2f(-e / 2), s2 = pow2f(-e - (-e / 2));
+      if (active && !q.in_range && !q.bad && q.mx != 0u) {
+        const float s1 = pow2f(-q.e / 2), s2 = pow2f(-q.e - (-q.e / 2));
         dense_row_fallback<D>(p, xblk, row, s1, s2, c, y);
       }
 #pragma unroll
-      for (int i = 0; i < 32; ++i) y[i] = __fmul_rn(y[i], r);
+      for (int i = 0; i < 32; ++i) y[i] = __fmul_rn(y[i], q.r);
       if (!active) continue;
       if (p.export_mode) {
         if (row < nr) {
           float* u = p.u_out + (r0 + row) * p.u_stride + 32 * c;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) u[i] = bad ? 0.f : y[i];
+          for (int i = 0; i < 32; ++i) u[i] = q.bad ? 0.f : y[i];
         }
-      } else if (!bad) {
+      } else if (!q.bad) {
         encode32_bits(bits, y, &tabs[kind], flags[kind], orow + c * bits);
       } else {
         for (int w = 0; w < bits; ++w) orow[c * bits + w] = 0u;
       }
     }
-    if (active) {
+    if (active && half == 0) {
       if (p.export_mode) {
-        if (row < nr) p.n_out[r0 + row] = bad ? __uint_as_float(0x7FC00000u) : norm;
+        if (row < nr) p.n_out[r0 + row] = q.bad ? __uint_as_float(0x7FC00000u) : q.norm;
       } else {
-        orow[rwords - 1] = bad ? 0x7FC00000u : __float_as_uint(norm);
-        if (bad && row < nr) report_error(p.err, TQ_DEVERR_NONFINITE);
+        orow[rwords - 1] = q.bad ? 0x7FC00000u : __float_as_uint(q.norm);
+        if (q.bad && row < nr) report_error(p.err, TQ_DEVERR_NONFINITE);
       }
     }
-    // tensor memory, the stage and the slots are complete
-    tc_fence_before();
-    __syncthreads();
+  };
+  // the tile's slots to the page pool (lanes over (slot, word))
+  auto store_slots = [&](int nr) {
     if (!p.export_mode) {
       for (int i = tid; i < nr * swords; i += blockDim.x) {
         const int rr = i / swords, w = i - rr * swords;
@@ -472,17 +464,150 @@ append_dense_kernel(DenseAppendParams p, const __grid_constant__ DenseAppendMaps
         if (off >= 0) ((uint32_t*)(p.pages + off))[w] = slots_s[rr * swords + w];
       }
     }
+  };
+  auto fail = [&]() {
+    report_error(p.err, TQ_DEVERR_TIMEOUT);
+    flags[2] = 1;
+  };
+  const int64_t first = blockIdx.x;
+  const int nst = p.nst;
+  // operations issued by thread 0 and not yet waited for: copies into stage b (pend_full[b]
+  // = completion parity, or -1) and MMAs into accumulator set a (pend_mma[a])
+  int pend_full[2] = {-1, -1}, pend_mma[2] = {-1, -1};
+
+  if (pipe) {
+    // prologue: copies of the first two tiles, the MMAs of the first
+    if (tid == 0 && first < ntiles) {
+      load_tile(first, 0);
+      pend_full[0] = 0;
+      if (first + gridDim.x < ntiles) {
+        load_tile(first + gridDim.x, 1);
+        pend_full[1] = 0;
+      }
+      if (!mbar_wait(&bars[0], 0, p.wait_ms)) {
+        fail();
+      } else {
+        pend_full[0] = -1;
+        tc_fence_after();
+        issue_mma(0, 0);
+        pend_mma[0] = 0;
+      }
+    }
     __syncthreads();
-    if (flags[2]) break;
-    // with one stage the next tile's rows come in now that the stage is free
-    if (nst == 1 && tid == 0 && tile + gridDim.x < ntiles) {
-      load_tile(tile + gridDim.x, 0);
-      pend_b = 0;
-      pend_par = (it + 1) & 1u;
+    uint32_t it = 0;
+    for (int64_t tile = first; tile < ntiles && !flags[2]; tile += gridDim.x, ++it) {
+      const int b = (int)(it & 1u);                 // stage and accumulator set of the tile
+      const uint32_t ph = (it >> 1) & 1u;           // their completion parity
+      const int64_t r0 = tile * kDenseRows;
+      const int nr = (int)imin64(kDenseRows, npairs - r0);
+      const uint8_t* xblk = stage_s + b * SM::STAGE + kind * SM::KIND;
+      slot_offsets(r0, nr);
+      // the staged rows (thread 0 waited for them before the MMAs)
+      if (tid != 0 && !mbar_wait(&bars[b], ph, p.wait_ms)) fail();
+      const RowNorm q = norm_pass(xblk);
+      // the next tile's MMAs into the other accumulator set, overlapping this epilogue
+      // (its rows were requested one tile ago; the set was released at the last barrier)
+      if (tid == 0 && tile + gridDim.x < ntiles && !flags[2]) {
+        const uint32_t nph = ((it + 1) >> 1) & 1u;
+        if (!mbar_wait(&bars[b ^ 1], nph, p.wait_ms)) {
+          fail();
+        } else {
+          pend_full[b ^ 1] = -1;
+          tc_fence_after();
+          issue_mma(b ^ 1, b ^ 1);
+          pend_mma[b ^ 1] = (int)nph;
+        }
+      }
+      __syncwarp();
+      // this tile's accumulators (every thread waits; a launch that stopped never
+      // completes them)
+      if (!mbar_wait(&bars[2 + b], ph, p.wait_ms)) {
+        if (tid == 0) report_error(p.err, TQ_DEVERR_TIMEOUT);
+        flags[2] = 1;
+      } else if (tid == 0) {
+        pend_mma[b] = -1;
+      }
+      __syncwarp();
+      tc_fence_after();
+      epilogue(xblk, b, r0, nr, q);
+      // tensor memory set b, stage b and the slots are complete
+      tc_fence_before();
+      __syncthreads();
+      store_slots(nr);
+      __syncthreads();
+      // stage b is free: the rows of the tile after next come in
+      if (tid == 0 && !flags[2] && tile + 2 * (int64_t)gridDim.x < ntiles) {
+        load_tile(tile + 2 * (int64_t)gridDim.x, b);
+        pend_full[b] = (int)(((it + 2) >> 1) & 1u);
+      }
+    }
+  } else {
+    if (tid == 0 && first < ntiles) {
+      load_tile(first, 0);
+      pend_full[0] = 0;
+    }
+    __syncthreads();
+    uint32_t it = 0;
+    for (int64_t tile = first; tile < ntiles; tile += gridDim.x, ++it) {
+      const int b = nst == 2 ? (int)(it & 1) : 0;
+      const uint32_t full_parity = nst == 2 ? (it >> 1) & 1u : it & 1u;
+      const int64_t r0 = tile * kDenseRows;
+      const int nr = (int)imin64(kDenseRows, npairs - r0);
+      if (tid == 0) {
+        // the MMAs of this tile once its rows have landed
+        if (!mbar_wait(&bars[b], full_parity, p.wait_ms)) {
+          fail();
+        } else {
+          pend_full[b] = -1;
+          tc_fence_after();
+          issue_mma(b, 0);
+          pend_mma[0] = (int)(it & 1u);
+          // with two stages the next tile's rows come in meanwhile (its stage was freed at
+          // the end of the previous tile)
+          if (nst == 2 && tile + gridDim.x < ntiles) {
+            load_tile(tile + gridDim.x, b ^ 1);
+            pend_full[b ^ 1] = (int)(((it + 1) >> 1) & 1u);
+          }
+        }
+      }
+      __syncwarp();
+      slot_offsets(r0, nr);
+      // the staged rows are read below: every thread waits for the tile's copies (thread 0
+      // has already waited for them before issuing the MMAs)
+      if (tid != 0 && !mbar_wait(&bars[b], full_parity, p.wait_ms)) fail();
+      const uint8_t* xblk = stage_s + b * SM::STAGE + kind * SM::KIND;
+      const RowNorm q = norm_pass(xblk);
+      // the accumulators (every thread waits; a launch that stopped never completes them)
+      if (!mbar_wait(&bars[2], it & 1u, p.wait_ms)) {
+        if (tid == 0) report_error(p.err, TQ_DEVERR_TIMEOUT);
+        flags[2] = 1;
+      } else if (tid == 0) {
+        pend_mma[0] = -1;
+      }
+      __syncwarp();
+      tc_fence_after();
+      epilogue(xblk, 0, r0, nr, q);
+      // tensor memory, the stage and the slots are complete
+      tc_fence_before();
+      __syncthreads();
+      store_slots(nr);
+      __syncthreads();
+      if (flags[2]) break;
+      // with one stage the next tile's rows come in now that the stage is free
+      if (nst == 1 && tid == 0 && tile + gridDim.x < ntiles) {
+        load_tile(tile + gridDim.x, 0);
+        pend_full[0] = (int)((it + 1) & 1u);
+      }
     }
   }
-  // copies still in flight (a launch that stopped early) land before the CTA ends
-  if (tid == 0 && pend_b >= 0) mbar_wait(&bars[pend_b], pend_par, p.wait_ms);
+  // copies and MMAs still in flight (a launch that stopped early) complete before the
+  // tensor memory is released and the CTA ends (bounded waits)
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b) {
+      if (pend_full[b] >= 0) mbar_wait(&bars[b], (uint32_t)pend_full[b], p.wait_ms);
+      if (pend_mma[b] >= 0) mbar_wait(&bars[2 + b], (uint32_t)pend_mma[b], p.wait_ms);
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
