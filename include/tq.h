@@ -287,9 +287,9 @@ TQ_API tq_status tq_paged_decode_noalloc(tq_tensor out, tq_tensor q, tq_tensor p
                                          void* stream);
 
 /* Workspace bytes tq_paged_decode needs for this geometry (host only).  The
- * workspace holds (2 + num_q_heads) * batch u32 merge counters at its start (zero
- * between calls: each call clears the ones it raised) and the split-KV partial
- * results (m, l, O') in fp32. */
+ * workspace holds 2 * batch u32 merge counters at its start (zero between calls:
+ * each call clears the ones it raised) and the split-KV partial results (m, l, O')
+ * in fp32. */
 TQ_API tq_status tq_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                                    int32_t head_dim, int32_t max_blocks, int32_t block_size,
                                    size_t* bytes);

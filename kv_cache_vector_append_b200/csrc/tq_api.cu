@@ -251,15 +251,9 @@ tq_status plan_decode(int batch, int h_q, int h_kv, int dim, int kb, int vb, int
   if (!found) return TQ_ERR_UNSUPPORTED;
   // workspace: merge counters (at the start, so that they can be cleared without
   // knowing a call's geometry: per sequence, covering CTAs that published and heads
-  // finished; per (sequence, head), parts finished), the second-level records (a head
-  // split into P = C / (B H_q) parts when there are more CTAs than heads), then the
-  // partial records (sized for the widest step)
-  const int64_t bh = (int64_t)batch * h_q;
-  const int64_t parts = std::max<int64_t>(1, plan->max_ctas / bh);
+  // finished), then the partial records (sized for the widest step)
   plan->counters_off = 0;
-  plan->part2_off = align256((size_t)(2 * batch + bh) * sizeof(unsigned int));
-  plan->part_off = plan->part2_off +
-                   align256(parts > 1 ? (size_t)(bh * parts) * (dim + 2) * sizeof(float) : 0);
+  plan->part_off = align256((size_t)batch * 2 * sizeof(unsigned int));
   plan->ws_bytes = plan->part_off + (size_t)(plan->max_ctas + batch) * wph_max * h_q * (dim + 2) *
                                         sizeof(float);
   return TQ_OK;
@@ -471,7 +465,6 @@ tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tens
   p.misc_off = plan.misc_off;
   p.smem_end = (int32_t)plan.smem;
   p.part = (float*)(ws + plan.part_off);
-  p.part2 = (float*)(ws + plan.part2_off);
   p.counters = (unsigned int*)(ws + plan.counters_off);
   p.wait_ms = kWaitMs;
   p.withhold_cta = -1;
@@ -494,7 +487,7 @@ tq_status decode_run(const DecodeCall& call, const tq_tensor& out, const tq_tens
   }
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    ds->counter_bytes = std::max(ds->counter_bytes, plan.part2_off);
+    ds->counter_bytes = std::max(ds->counter_bytes, plan.part_off);
     if (ds->inject_wait_ms > 0) {
       p.wait_ms = ds->inject_wait_ms;
       p.withhold_cta = ds->inject_withhold;

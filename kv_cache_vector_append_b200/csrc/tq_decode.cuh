@@ -107,10 +107,8 @@ struct DecodeParams {
   int32_t misc_off;             // barriers, q', prefix sums, block ids, merge scratch
   int32_t smem_end;             // bytes of dynamic shared memory the layout spans
   float* part;                  // records [(C + B) * wph][H_q][D + 2]
-  float* part2;                 // second-level records [B][H_q][P][D + 2] (P > 1 only)
-  unsigned int* counters;       // [B] covering CTAs that published, [B] heads finished,
-                                // [B][H_q] parts finished; zero between calls (the last
-                                // user of a counter clears it)
+  unsigned int* counters;       // [B] covering CTAs that published, [B] heads finished;
+                                // zero between calls (the last user of a counter clears it)
   unsigned int* err;
   uint32_t wait_ms;             // limit of every bounded wait (milliseconds)
   int32_t withhold_cta;         // test hook: this CTA never announces its records (-1: none)
@@ -1090,7 +1088,6 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   auto nonempty = [&](int64_t c) { return every_cta_busy || cta_has_steps(c, S, Cn); };
   unsigned int* arrived = p.counters;                // covering CTAs that published b's records
   unsigned int* merged = p.counters + B;             // query heads of b finished
-  unsigned int* parts_done = p.counters + 2 * B;     // [B][h_q]: parts of (b, h) finished
   // (M, l) and this lane's E values of a record whose values start at rec + 2 + lane E
   auto load_record = [&](const float* rec, float& m, float& ll, float (&v)[E]) {
     const float2 ml = __ldcg((const float2*)rec);
@@ -1182,24 +1179,19 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     }
   };
 
-  // End phase.  The merge work is dealt out as items (b, h, part): the R = n_b wph
-  // records of query head h of sequence b (n_b covering CTAs) are split into P parts, P
-  // as large as the grid allows (P > 1 only when there are fewer heads than CTAs), and
-  // item i goes to the CTA of rank i mod C' among the C' CTAs with steps, so the merge
-  // spreads over the whole grid instead of the CTAs that happen to cover a sequence.
-  // A CTA's items are taken by groups of g warps (g as large as its item count allows);
-  // each warp folds its share of the item's records, the group's first warp combines
-  // the g partials.  With P = 1 that is the head's output.  With P > 1 the part goes
-  // to a second-level record, and the last part of (b, h) to finish (a counter) folds
-  // the P parts and writes the output, so no part waits for another.  The last head of
-  // b to finish clears b's counters.  `dead`: this CTA gave up a stage wait; its items
-  // are counted (so that the counters return to zero) but not merged.
+  // End phase.  The merge work is dealt out as items (b, h): the R = n_b wph records of
+  // query head h of sequence b (n_b covering CTAs); item i = b H_q + h goes to the CTA of
+  // rank i mod C' among the C' CTAs with steps, so the merge spreads over the whole grid
+  // instead of the CTAs that happen to cover a sequence.  A CTA's items are taken by
+  // groups of g warps (g as large as its item count allows); each warp folds its share
+  // of the item's records, the group's first warp combines the g partials and writes
+  // the head's output.  The last head of b to finish clears b's counters.  `dead`: this
+  // CTA gave up a stage wait; its items are counted (so that the counters return to
+  // zero) but not merged.
   auto end_phase = [&](bool dead) {
     const int Ce = every_cta_busy ? (int)Cn : (int)S;         // CTAs with steps
     const int my = every_cta_busy ? (int)blockIdx.x : (int)s0;  // rank among them
-    const int bh = B * p.h_q;                                   // < 2^31 (host check)
-    const int P = Ce / bh > 1 ? Ce / bh : 1;
-    const int NI = bh * P;                                      // <= max(bh, Ce)
+    const int NI = B * p.h_q;                                   // < 2^31 (host check)
     const int m = my < NI ? (NI - my + Ce - 1) / Ce : 0;
     if (m == 0) return;
     int g = 1;
@@ -1217,13 +1209,11 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     };
     for (int k0 = 0; k0 < m; k0 += groups) {
       const int k = k0 + gi;
-      int b = -1, h = 0, part = 0;
+      int b = -1, h = 0;
       if (k < m) {
         const int i = my + k * Ce;
-        const int hp = i / P;
-        b = hp / p.h_q;
-        h = hp - b * p.h_q;
-        part = i - hp * P;
+        b = i / p.h_q;
+        h = i - b * p.h_q;
         if (prefix[b + 1] == prefix[b]) b = -1;        // no steps: output written already
       }
       float M = -INFINITY, l = 0.f, o[E];
@@ -1241,11 +1231,10 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
         ok = !dead && wait_arrived(b, n);
         if (ok) {
           const int R = (int)(c_hi - c_lo + 1) << lw;
-          const int r_lo = R * part / P, r_hi = R * (part + 1) / P;
-          const int cnt = r_hi - r_lo > mi ? (r_hi - r_lo - mi + g - 1) / g : 0;
+          const int cnt = R > mi ? (R - mi + g - 1) / g : 0;
           const float* hb = p.part + (int64_t)h * (D + 2);
           fold_records<E>(cnt, [&](int j, float& mm, float& ll, float (&v)[E]) {
-            const int r = r_lo + mi + j * g;
+            const int r = mi + j * g;
             const int64_t c = c_lo + (r >> lw);
             if (nonempty(c)) load_record(hb + ((c + b) * wph + (r & (wph - 1))) * rstride, mm, ll, v);
           }, M, l, o);
@@ -1284,43 +1273,14 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
           }
           if (Mx == -INFINITY) L = 0.f;
         }
-        bool last = true;
-        if (P > 1) {
-          // publish this part; the last part of (b, h) to finish folds all P of them
-          float* rec2 = p.part2 + ((int64_t)b * p.h_q + h) * P * (D + 2);
-          float* mine = rec2 + (int64_t)part * (D + 2);
-          if (lane == 0) __stcg((float2*)mine, make_float2(Mx, L));
-#pragma unroll
-          for (int i = 0; i < E; ++i) __stcg(mine + 2 + lane * E + i, acc_o[i]);
-          __syncwarp();
-          int lst = 0;
-          if (lane == 0) {
-            unsigned int* pc = parts_done + (int64_t)b * p.h_q + h;
-            lst = atom_add_acq_rel(pc, 1u) == (unsigned)P - 1;
-            if (lst) atomicExch(pc, 0u);
-          }
-          __syncwarp();
-          last = __shfl_sync(0xffffffffu, lst, 0) != 0;
-          if (last) {
-            Mx = -INFINITY;
-            L = 0.f;
-#pragma unroll
-            for (int i = 0; i < E; ++i) acc_o[i] = 0.f;
-            fold_records<E>(P, [&](int j, float& mm, float& ll, float (&v)[E]) {
-              load_record(rec2 + (int64_t)j * (D + 2), mm, ll, v);
-            }, Mx, L, acc_o);
-          }
-        }
-        if (last) {
-          // count the head first (the counter's round trip overlaps the output); the
-          // last head of b clears b's counters, every wait on them being over
-          unsigned int done = 0;
-          if (lane == 0) done = atomicAdd(&merged[b], 1u);
-          if (ok) finalize(b, h, Mx, L, acc_o);
-          if (lane == 0 && done == (unsigned)p.h_q - 1) {
-            atomicExch(&arrived[b], 0u);
-            atomicExch(&merged[b], 0u);
-          }
+        // count the head first (the counter's round trip overlaps the output); the last
+        // head of b clears b's counters, every wait on them being over
+        unsigned int done = 0;
+        if (lane == 0) done = atomicAdd(&merged[b], 1u);
+        if (ok) finalize(b, h, Mx, L, acc_o);
+        if (lane == 0 && done == (unsigned)p.h_q - 1) {
+          atomicExch(&arrived[b], 0u);
+          atomicExch(&merged[b], 0u);
         }
       }
       __syncthreads();

@@ -33,7 +33,7 @@ struct DecodePlan {
   int lut_bytes = 0;      // lookup tables at the start of shared memory
   size_t smem = 0;        // dynamic shared memory of the decode kernel
   int max_ctas = 0;       // upper bound of the persistent grid (one CTA per SM)
-  size_t part_off = 0, part2_off = 0, counters_off = 0;
+  size_t part_off = 0, counters_off = 0;
   size_t ws_bytes = 0;
 };
 
