@@ -128,18 +128,27 @@ __device__ __forceinline__ void build_tables(EncodeTables* t, const float* b, in
 // Phase 2: 4 k0 of each bucket (binary search over the boundaries already in shared
 // memory).  The lowest float of bucket g is g << 20 for a positive bucket and
 // -((g & 0x7ff) << 20 | 0xfffff) for a negative one.  Only used for bits <= 4.
+// Coordinates of a unit vector have |u| <= 1 (up to rounding), so only the buckets of
+// |u| < 2 are searched; the others hold their exact counts directly: every boundary
+// (|b| < 1) lies below u >= 2, none below u <= -2, and NaN patterns get a valid entry.
 __device__ __forceinline__ void build_bucket_table(EncodeTables* t, int bits, int tid,
                                                    int nthreads) {
   if (bits > 4) return;
   const int n = (1 << bits) - 1;
   for (int g = tid; g < kBuckets; g += nthreads) {
-    const uint32_t lowbits = (g & 0x800) ? ((uint32_t)g << kBucketShift) | 0xFFFFFu
-                                         : (uint32_t)g << kBucketShift;
-    const float lo = __uint_as_float(lowbits);
-    int a = 0, c = n;                   // count of boundaries < lo lies in [a, c]
-    while (a < c) {
-      const int m = (a + c) >> 1;
-      if (t->bnd[m] < lo) a = m + 1; else c = m;
+    int a;
+    if ((g & 0x7ff) >= 0x400) {         // |u| >= 2 (or inf / NaN patterns)
+      a = (g & 0x800) ? 0 : n;
+    } else {
+      const uint32_t lowbits = (g & 0x800) ? ((uint32_t)g << kBucketShift) | 0xFFFFFu
+                                           : (uint32_t)g << kBucketShift;
+      const float lo = __uint_as_float(lowbits);
+      a = 0;
+      int c = n;                        // count of boundaries < lo lies in [a, c]
+      while (a < c) {
+        const int m = (a + c) >> 1;
+        if (t->bnd[m] < lo) a = m + 1; else c = m;
+      }
     }
     t->k4[g] = (uint8_t)(4 * a);
   }
