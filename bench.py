@@ -89,11 +89,23 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def code_text(src):
+    """Kernel source without its // comments and blank lines: what the counters depend on."""
+    lines = []
+    for line in src.splitlines():
+        code = line.split("//", 1)[0].rstrip()
+        if code.strip():
+            lines.append(code)
+    return "\n".join(lines)
+
+
 def kernel_hash():
+    """Hash of the kernel sources' code (comments and blank lines ignored), keying the
+    committed ncu traffic figures to the kernels they were taken on."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            h.update(code_text(f.read()).encode())
     return h.hexdigest()[:16]
 
 

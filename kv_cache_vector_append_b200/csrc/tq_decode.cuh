@@ -45,10 +45,12 @@
 //   * at the end of a segment every warp writes its partial (M, l, O') to record
 //     ((CTA + sequence) * wph + sub-stream), an index no other (CTA, sequence) pair
 //     shares because the ranges are monotone;
-//   * end phase: the CTA counts its records on each sequence's counter, waits (bounded)
-//     until every CTA covering the sequence has done so, and merges a share of the
-//     sequence's query heads: divide by l, then o = R^T O' (FWHT, 1/sqrt(D), sign
-//     flips).  The launch is cooperative, so the CTAs that wait are co-resident.
+//   * end phase: the CTA publishes its records on each covered sequence's counter
+//     (release), then takes its share of the merge items (sequence, query head), dealt
+//     round-robin over all CTAs: wait (bounded, acquire) until every CTA covering the
+//     sequence has published, fold the head's records, divide by l, then o = R^T O'
+//     (FWHT, 1/sqrt(D), sign flips).  The launch is cooperative, so the CTAs that wait
+//     are co-resident.
 // The coordinate order inside each mma tile is free (a permutation applied to both
 // operands of a contraction leaves it unchanged); it is chosen so that every thread
 // reads whole 32-bit words of codes, and undone when O' is written to its record.
