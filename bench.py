@@ -58,21 +58,24 @@ def parse_args(argv=None):
 # bytes and units
 # ---------------------------------------------------------------------------
 
-def append_bytes(spec, n_tokens):
+def append_bytes(spec, n_tokens, sb=None):
     """Algorithmic bytes of quantize-append: per (token, KV head) read 2 rows of D
-    inputs, write slot_bytes; plus 8 bytes of slot_mapping per token."""
+    inputs, write slot_bytes (``sb``, default the plain slot); plus 8 bytes of
+    slot_mapping per token."""
     d = spec.head_dim
     es = 4 if spec.dtype == "float32" else 2
-    sb = (d * spec.k_bits + 7) // 8 + 4 + (d * spec.v_bits + 7) // 8 + 4
+    if sb is None:
+        sb = (d * spec.k_bits + 7) // 8 + 4 + (d * spec.v_bits + 7) // 8 + 4
     return n_tokens * spec.num_kv_heads * (2 * d * es + sb) + 8 * n_tokens
 
 
-def decode_bytes(spec, seq_lens):
-    """Algorithmic bytes of paged decode: slot_bytes per (token, KV head), 4 bytes
-    of block table per 16 tokens, q read and out written."""
+def decode_bytes(spec, seq_lens, sb=None):
+    """Algorithmic bytes of paged decode: slot_bytes (``sb``, default the plain slot)
+    per (token, KV head), 4 bytes of block table per 16 tokens, q read and out written."""
     d = spec.head_dim
     es = 4 if spec.dtype == "float32" else 2
-    sb = (d * spec.k_bits + 7) // 8 + 4 + (d * spec.v_bits + 7) // 8 + 4
+    if sb is None:
+        sb = (d * spec.k_bits + 7) // 8 + 4 + (d * spec.v_bits + 7) // 8 + 4
     lens = np.asarray(seq_lens, dtype=np.int64)
     packed = int(lens.sum()) * spec.num_kv_heads * sb
     bt = int(((lens + 15) // 16).sum()) * 4
@@ -446,11 +449,11 @@ def time_legs(spec, x, steps, stream, flush=None):
             float(np.mean([e[2].elapsed_time(e[3]) for e in ev])))
 
 
-def leg_summary(wl, app_ms, dec_ms, peak):
+def leg_summary(wl, app_ms, dec_ms, peak, sb=None):
     spec = wl.spec
     n_step = len(wl.step_tokens)
-    a_bytes = append_bytes(spec, n_step)
-    d_bytes, d_packed = decode_bytes(spec, wl.seq_lens)
+    a_bytes = append_bytes(spec, n_step, sb)
+    d_bytes, d_packed = decode_bytes(spec, wl.seq_lens, sb)
     rows = 2 * n_step * spec.num_kv_heads
     return {"append": {"ms": app_ms, "mrows_per_s": rows / (app_ms * 1e-3) / 1e6,
                        "gbs": a_bytes / (app_ms * 1e-3) / 1e9,
@@ -505,8 +508,9 @@ def extra_config_legs(configs, dev, steps, warmup, peak):
 
 def variant_legs(wl, x, dev, steps, warmup, peak):
     """The survey's next rows on the main workload, each in its own timed region:
-    quantize-append and decode with the dense (QR) rotation (tcgen05 GEMM), and the
-    decode with a 64-token uncompressed hot window per sequence (bf16)."""
+    quantize-append and decode with the dense (QR) rotation (tcgen05 GEMM), the decode
+    with a 64-token uncompressed hot window per sequence (bf16), and quantize-append and
+    decode of keys that carry the QJL residual sketch."""
     import torch
     import kv_cache_vector_append_b200 as tq
     spec = wl.spec
@@ -564,6 +568,33 @@ def variant_legs(wl, x, dev, steps, warmup, peak):
     res["hot_window"] = {"window_tokens": w, "ms": dec,
                          "gbs": (d_bytes + hot_bytes) / (dec * 1e-3) / 1e9,
                          "frac_of_peak": (d_bytes + hot_bytes) / (dec * 1e-3) / 1e9 / peak}
+    # keys that also carry the QJL sketch of their residual: their own page pool (the slot
+    # is larger, its stride a multiple of 8)
+    if spec.head_dim >= 128 and spec.k_bits <= 4:
+        from kv_cache_vector_append_b200 import workloads as W
+        sbq = tq.slot_bytes_qjl(spec.head_dim, spec.k_bits, spec.v_bits)
+        qpages = W.empty_pages(wl, device=dev, slot_stride=(sbq + 7) // 8 * 8)
+        qseed = spec.sign_seed + 1
+        for _ in range(max(warmup, 3)):
+            tq.quantize_append_qjl(qpages, x["sm"], x["k"], x["v"], x["cb"], spec.sign_seed,
+                                   qseed, stream)
+            tq.paged_decode_qjl(x["out"], x["q"], qpages, x["bt"], x["sl"], x["cb"],
+                                spec.sign_seed, qseed, spec.scale, stream)
+        torch.cuda.synchronize(dev)
+        e = [[ev() for _ in range(3)] for _ in range(steps)]
+        for i in range(steps):
+            e[i][0].record(stream)
+            tq.quantize_append_qjl(qpages, x["sm"], x["k"], x["v"], x["cb"], spec.sign_seed,
+                                   qseed, stream)
+            e[i][1].record(stream)
+            tq.paged_decode_qjl(x["out"], x["q"], qpages, x["bt"], x["sl"], x["cb"],
+                                spec.sign_seed, qseed, spec.scale, stream)
+            e[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+        app = float(np.mean([a.elapsed_time(b) for a, b, _ in e]))
+        dec = float(np.mean([b.elapsed_time(c) for _, b, c in e]))
+        res["qjl"] = dict(leg_summary(wl, app, dec, peak, sb=sbq), slot_bytes=sbq)
+        del qpages
     if tq.get_device_error(stream):
         raise RuntimeError("device error during the variant legs")
     return res
