@@ -660,6 +660,11 @@ tq_status append_impl(tq_tensor pages, tq_tensor slot_mapping, tq_tensor k, tq_t
   p.bulk_out = p.run_heads > 0 && pages.shape[3] == slot && pages.stride[2] == slot &&
                (uintptr_t)pages.data % 16 == 0 && pages.stride[0] % 16 == 0 &&
                pages.stride[1] % 16 == 0 && ((int64_t)p.run_heads * slot) % 16 == 0;
+  // a padded slot stride: slots stored one by one, the 16-byte body by a bulk copy
+  p.slot_body = 0;
+  if (!p.bulk_out && slot >= 16 && (uintptr_t)pages.data % 16 == 0 &&
+      pages.stride[0] % 16 == 0 && pages.stride[1] % 16 == 0 && pages.stride[2] % 16 == 0)
+    p.slot_body = slot & ~15;
   AppendMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   p.tma_in = 0;

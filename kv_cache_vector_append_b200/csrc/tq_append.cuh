@@ -56,6 +56,9 @@ struct AppendParams {
   int32_t run_heads;        // heads of one token in a tile (tiles token-aligned), else 0
   int32_t tma_in;           // 1: input rows staged by tensor copies (maps K, V)
   int32_t bulk_out;         // 1: slots stored by one bulk copy per token run
+  int32_t slot_body;        // > 0 (padded slot stride): slots stored one by one, the first
+                            // slot_body bytes (a multiple of 16) by a bulk copy, the rest
+                            // by 4-byte stores
   unsigned int* redo;       // [2]: a row left the fast path's range; CTAs of the redo done
   // QJL residual sketch of the keys (append_kernel<..., QJL = true>): K centroids and the
   // seed of the sketch's signs
@@ -568,8 +571,9 @@ struct AppendSmem {
   static __host__ __device__ constexpr int slot_words(int kbits, int vbits) {
     return (D * kbits / 8 + 4 + D * vbits / 8 + 4) / 4 + D / 32 + 1;   // room for a sketch
   }
+  // the staged slots' rows are (swords rounded up to 4) words apart at most
   static __host__ __device__ constexpr int misc_per_warp(int swords) {
-    return 16 + 2 * G::ROWS * 8 + 2 * 2 * G::ROWS * 8 + (G::ROWS * swords * 4 + 15) / 16 * 16;
+    return 16 + 2 * G::ROWS * 8 + 2 * 2 * G::ROWS * 8 + G::ROWS * ((swords + 3) / 4) * 16;
   }
   static __host__ __device__ constexpr int bytes(int kbits, int vbits) {
     return TABLES + 1024 + kAppendWarps * (2 * KIND + misc_per_warp(slot_words(kbits, vbits)));
@@ -613,7 +617,9 @@ append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
   uint64_t* bars = (uint64_t*)misc;                                // [2 kinds]
   int64_t* dst_s = (int64_t*)(misc + 16);                          // [2 tiles][ROWS] slots
   const uint8_t** src_s = (const uint8_t**)(dst_s + 2 * G::ROWS);  // [2 tiles][2 kinds][ROWS]
-  uint32_t* out_s = (uint32_t*)(src_s + 2 * 2 * G::ROWS);          // [ROWS][swords]
+  uint32_t* out_s = (uint32_t*)(src_s + 2 * 2 * G::ROWS);          // [ROWS][srow]
+  // words between the staged slots: 16-byte rows when slots are stored one by one
+  const int srow = p.slot_body > 0 ? (swords + 3) & ~3 : swords;
 
   const int64_t npairs = p.num_tokens * p.h_kv;                    // < 2^31 (host check)
   const int64_t ntiles = (npairs + G::ROWS - 1) / G::ROWS;
@@ -746,11 +752,11 @@ append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
       const float r = rotate_row<D, Tin, SAFE>(xp, row0 + (uint32_t)(kind * SM::KIND),
                                                smask + part * 64, part, &n, &bad, &oor);
       if constexpr (!SAFE) redo_needed |= oor && rl < nr;
-      if (kind == 0 && p.bulk_out) {    // the previous tile's slots have been read out
+      if (kind == 0 && (p.bulk_out || p.slot_body > 0)) {   // previous slots read out
         bulk_wait_read_all();
         __syncwarp();
       }
-      uint32_t* orow = out_s + rl * swords + (kind ? kwords : 0);
+      uint32_t* orow = out_s + rl * srow + (kind ? kwords : 0);
       const EncodeTables* t = &tabs[kind];
       const int cw = D * bits / 32;                        // code words of the region
       const int wpl = cw / G::TPR;                         // code words per lane
@@ -792,6 +798,23 @@ append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
           bulk_s2g(p.pages + off, out_s + lane * hr * swords, (uint32_t)(hr * swords * 4));
         bulk_commit();
       }
+    } else if (p.slot_body > 0) {
+      // slots one by one (a padded slot stride): each row's 16-byte body by a bulk copy,
+      // its tail words by plain stores; the padding is never written
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane < nr) {
+        const int64_t off = dst_s[tb * G::ROWS + lane];
+        if (off >= 0) bulk_s2g(p.pages + off, out_s + lane * srow, (uint32_t)p.slot_body);
+        bulk_commit();
+      }
+      const int bw = p.slot_body >> 2, tw = swords - bw;   // body and tail words
+      for (int i = lane; i < nr * tw; i += 32) {
+        const int rr = i / tw, w = bw + (i - rr * tw);
+        const int64_t off = dst_s[tb * G::ROWS + rr];
+        if (off >= 0) ((uint32_t*)(p.pages + off))[w] = out_s[rr * srow + w];
+      }
+      __syncwarp();
     } else {
       // write back the tile's full slots: lanes run over (pair, word)
       int rr = 0, w = lane;

@@ -31,9 +31,9 @@ def _regions(pages_np, wl, tokens, kind):
     return rows[..., :kb] if kind == 0 else rows[..., kb:kb + vb]
 
 
-def _bit_exact_case(tq, wl, tokens=None, kind="beta"):
+def _bit_exact_case(tq, wl, tokens=None, kind="beta", slot_stride=None, fill=0):
     """Packed bytes equal the oracle's packing of the GPU's own fp32 unit coords."""
-    pages, cb = gpu_append(tq, wl, tokens, kind=kind)
+    pages, cb = gpu_append(tq, wl, tokens, kind=kind, slot_stride=slot_stride, fill=fill)
     pages_np = pages.cpu().numpy()
     toks = np.arange(wl.k.shape[0]) if tokens is None else np.asarray(tokens)
     d = wl.spec.head_dim
@@ -201,6 +201,19 @@ def test_full_size_configs_sampled(cfg):
             b = table.boundaries.astype(np.float64)
             assert np.all(np.min(np.abs(ref_u[bad][:, None] - b[None, :]), axis=1) < 1e-5)
     assert mism <= 1e-4 * total
+
+
+# A padded slot stride stores the slots one by one: with a stride that is a multiple of
+# 16 bytes (pads 8 and 24 here), each slot's 16-byte body by a bulk copy and its tail by
+# words; otherwise (pad 16) word by word.  Both write the oracle's bytes and leave the
+# padding alone.
+@pytest.mark.parametrize("pad", [8, 16, 24])
+@pytest.mark.parametrize("d,kb,vb", [(128, 4, 2), (128, 4, 4), (64, 3, 3)])
+def test_bit_exact_padded_slot_stride(d, kb, vb, pad):
+    tq = _tq()
+    wl = W.generate(_mini(d, kb, vb, h_kv=4, batch=3, seq=45, seed=pad + kb))
+    pages_np = _bit_exact_case(tq, wl, slot_stride=wl.slot_bytes + pad, fill=0xA5)
+    assert np.all(pages_np[..., wl.slot_bytes:] == 0xA5)
 
 
 def test_padding_and_unmapped_slots_untouched():
