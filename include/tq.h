@@ -165,7 +165,11 @@ TQ_API tq_status tq_slot_bytes(int32_t dim, int32_t k_bits, int32_t v_bits, int3
  *   - each token's slots are stored with one bulk copy when, in addition to that H_kv
  *     rule, slot_stride == tq_slot_bytes(...), pages is 16-byte aligned with block and
  *     row strides that are multiples of 16, and the token's run of slots is a
- *     multiple of 16 bytes.
+ *     multiple of 16 bytes;
+ *   - otherwise, when pages is 16-byte aligned with block, row and head strides that
+ *     are multiples of 16 (a padded slot_stride), each slot's first
+ *     (slot_bytes & ~15) bytes are stored by one bulk copy and the rest by 4-byte
+ *     stores; the padding is not written.
  *   Other layouts take lane-wise copies.
  * Errors: TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED (nothing enqueued), TQ_ERR_CUDA. */
 TQ_API tq_status tq_quantize_append(tq_tensor pages, tq_tensor slot_mapping, tq_tensor k,
