@@ -1062,9 +1062,12 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   // This warp's partial of sequence b -> its record.  Record of query head h:
   // [M, l, O'] with O' in fragment order: coordinate VS::coord(g, 2 mt + c) at
   // 2 + 2 (8 mt + g) + c, so that each store (one mt, one head column per thread) writes
-  // eight contiguous pairs per head.
+  // eight contiguous pairs per head.  Records sit at [h][slot][sub] with slot = CTA + b
+  // (unique, as a CTA's sequences follow the previous CTA's), so the records of one
+  // (b, h), those of the covering CTAs, are contiguous.
+  const int64_t nslots = (int64_t)gridDim.x + B;
   auto flush = [&](int b) {
-    float* base = p.part + ((int64_t)(blockIdx.x + b) * wph + sub) * (int64_t)p.h_q * (D + 2);
+    float* base = p.part + ((int64_t)(blockIdx.x + b) * wph + sub) * (D + 2);
 #pragma unroll
     for (int hh = 0; hh < NH; ++hh) {
 #pragma unroll
@@ -1075,7 +1078,7 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
         l += __shfl_xor_sync(0xffffffffu, l, 16);
         const int g = 8 * hh + 2 * tig + e;
         if (g < G) {
-          float* rec = base + (int64_t)(kvh * G + g) * (D + 2);
+          float* rec = base + (int64_t)(kvh * G + g) * nslots * wph * (D + 2);
           if (gid == 0) *(float2*)rec = make_float2(Mrun[hh][e], l);
 #pragma unroll
           for (int mt = 0; mt < C::MT; ++mt)
@@ -1202,7 +1205,6 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     int nat[E];                          // coordinate at record position 2 + lane E + k
 #pragma unroll
     for (int k = 0; k < E; ++k) nat[k] = rpos[lane * E + k];
-    const int64_t rstride = (int64_t)p.h_q * (D + 2);
     const int lw = __ffs(wph) - 1;                   // wph is a power of two
     // the CTA of step x: 32-bit arithmetic when (x + 1) C fits
     const bool small = (uint64_t)S * (uint64_t)Cn < (1ull << 32);
@@ -1234,11 +1236,11 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
         if (ok) {
           const int R = (int)(c_hi - c_lo + 1) << lw;
           const int cnt = R > mi ? (R - mi + g - 1) / g : 0;
-          const float* hb = p.part + (int64_t)h * (D + 2);
+          const float* hb = p.part + ((int64_t)h * nslots + c_lo + b) * wph * (D + 2);
           fold_records<E>(cnt, [&](int j, float& mm, float& ll, float (&v)[E]) {
             const int r = mi + j * g;
             const int64_t c = c_lo + (r >> lw);
-            if (nonempty(c)) load_record(hb + ((c + b) * wph + (r & (wph - 1))) * rstride, mm, ll, v);
+            if (nonempty(c)) load_record(hb + (int64_t)r * (D + 2), mm, ll, v);
           }, M, l, o);
         }
       }
