@@ -254,7 +254,7 @@ tq_status plan_decode(int batch, int h_q, int h_kv, int dim, int kb, int vb, int
   // finished), then the partial records (sized for the widest step)
   plan->counters_off = 0;
   plan->part_off = align256((size_t)batch * 2 * sizeof(unsigned int));
-  plan->ws_bytes = plan->part_off + (size_t)(plan->max_ctas + batch) * wph_max * h_q * (dim + 2) *
+  plan->ws_bytes = plan->part_off + (size_t)(plan->max_ctas + batch) * wph_max * h_q * (dim + 4) *
                                         sizeof(float);
   return TQ_OK;
 }

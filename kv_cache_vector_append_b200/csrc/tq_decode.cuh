@@ -1059,15 +1059,16 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
     }
   };
 
-  // This warp's partial of sequence b -> its record.  Record of query head h:
-  // [M, l, O'] with O' in fragment order: coordinate VS::coord(g, 2 mt + c) at
-  // 2 + 2 (8 mt + g) + c, so that each store (one mt, one head column per thread) writes
-  // eight contiguous pairs per head.  Records sit at [h][slot][sub] with slot = CTA + b
+  // This warp's partial of sequence b -> its record.  Record of query head h (kRec
+  // floats, 16-byte aligned): [O', M, l, 2 unused] with O' in fragment order: coordinate
+  // VS::coord(g, 2 mt + c) at 2 (8 mt + g) + c, so that each store (one mt, one head
+  // column per thread) writes eight contiguous pairs per head.  Records sit at [h][slot][sub] with slot = CTA + b
   // (unique, as a CTA's sequences follow the previous CTA's), so the records of one
   // (b, h), those of the covering CTAs, are contiguous.
   const int64_t nslots = (int64_t)gridDim.x + B;
+  constexpr int64_t kRec = D + 4;                    // floats per record
   auto flush = [&](int b) {
-    float* base = p.part + ((int64_t)(blockIdx.x + b) * wph + sub) * (D + 2);
+    float* base = p.part + ((int64_t)(blockIdx.x + b) * wph + sub) * kRec;
 #pragma unroll
     for (int hh = 0; hh < NH; ++hh) {
 #pragma unroll
@@ -1078,11 +1079,11 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
         l += __shfl_xor_sync(0xffffffffu, l, 16);
         const int g = 8 * hh + 2 * tig + e;
         if (g < G) {
-          float* rec = base + (int64_t)(kvh * G + g) * nslots * wph * (D + 2);
-          if (gid == 0) *(float2*)rec = make_float2(Mrun[hh][e], l);
+          float* rec = base + (int64_t)(kvh * G + g) * nslots * wph * kRec;
+          if (gid == 0) *(float2*)(rec + D) = make_float2(Mrun[hh][e], l);
 #pragma unroll
           for (int mt = 0; mt < C::MT; ++mt)
-            *(float2*)(rec + 2 + 2 * (8 * mt + gid)) =
+            *(float2*)(rec + 2 * (8 * mt + gid)) =
                 make_float2(acc[hh][mt][e], acc[hh][mt][e + 2]);
         }
       }
@@ -1093,16 +1094,27 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   auto nonempty = [&](int64_t c) { return every_cta_busy || cta_has_steps(c, S, Cn); };
   unsigned int* arrived = p.counters;                // covering CTAs that published b's records
   unsigned int* merged = p.counters + B;             // query heads of b finished
-  // (M, l) and this lane's E values of a record whose values start at rec + 2 + lane E
+  // (M, l) and this lane's E values of a record (16-byte aligned): values at rec + lane E
   auto load_record = [&](const float* rec, float& m, float& ll, float (&v)[E]) {
-    const float2 ml = __ldcg((const float2*)rec);
+    const float2 ml = __ldcg((const float2*)(rec + D));
     m = ml.x;
     ll = ml.y;
+    if constexpr (E % 4 == 0) {
 #pragma unroll
-    for (int k = 0; k < E / 2; ++k) {
-      const float2 t = __ldcg((const float2*)(rec + 2 + lane * E) + k);
-      v[2 * k] = t.x;
-      v[2 * k + 1] = t.y;
+      for (int k = 0; k < E / 4; ++k) {
+        const float4 t = __ldcg((const float4*)(rec + lane * E) + k);
+        v[4 * k] = t.x;
+        v[4 * k + 1] = t.y;
+        v[4 * k + 2] = t.z;
+        v[4 * k + 3] = t.w;
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < E / 2; ++k) {
+        const float2 t = __ldcg((const float2*)(rec + lane * E) + k);
+        v[2 * k] = t.x;
+        v[2 * k + 1] = t.y;
+      }
     }
   };
 
@@ -1236,11 +1248,11 @@ decode_kernel(DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
         if (ok) {
           const int R = (int)(c_hi - c_lo + 1) << lw;
           const int cnt = R > mi ? (R - mi + g - 1) / g : 0;
-          const float* hb = p.part + ((int64_t)h * nslots + c_lo + b) * wph * (D + 2);
+          const float* hb = p.part + ((int64_t)h * nslots + c_lo + b) * wph * kRec;
           fold_records<E>(cnt, [&](int j, float& mm, float& ll, float (&v)[E]) {
             const int r = mi + j * g;
             const int64_t c = c_lo + (r >> lw);
-            if (nonempty(c)) load_record(hb + (int64_t)r * (D + 2), mm, ll, v);
+            if (nonempty(c)) load_record(hb + (int64_t)r * kRec, mm, ll, v);
           }, M, l, o);
         }
       }
