@@ -591,8 +591,9 @@ struct AppendSmem {
 // with the rescaling rotation (identical results for the other rows); the last CTA
 // clears redo.
 // QJL: the K rows also store the QJL sketch of their residual (K region: codes, norm,
-// D sign bits, residual norm).
-template <int D, typename Tin, bool SAFE, bool QJL>
+// D sign bits, residual norm).  FIXB > 0: both code widths are FIXB, fixed at compile
+// time (no dispatch on the width in the loop).
+template <int D, typename Tin, bool SAFE, bool QJL, int FIXB = 0>
 __global__ void __launch_bounds__(kAppendWarps * 32, 2)
 append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
   if constexpr (SAFE) {
@@ -771,6 +772,8 @@ append_kernel(AppendParams p, const __grid_constant__ AppendMaps maps) {
           orow[cw + 1 + 2 * part] = z0;
           orow[cw + 2 + 2 * part] = z1;
           if (part == G::TPR - 1) orow[cw + 1 + D / 32] = __float_as_uint(gamma);
+        } else if constexpr (FIXB > 0) {
+          encode_pack_any<FIXB, false>(xp, r, t, use_fast, mine, 0u);
         } else {
           encode_pack_bits<false>(bits, xp, r, t, use_fast, mine, 0u);
         }

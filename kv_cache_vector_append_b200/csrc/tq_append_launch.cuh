@@ -6,12 +6,14 @@
 
 namespace tq {
 
-template <int D, typename Tin, bool QJL>
+// FIXB > 0: the fast path's instantiation for K and V codes of FIXB bits (the redo
+// stays generic; both give the same bytes).
+template <int D, typename Tin, bool QJL, int FIXB = 0>
 tq_status launch_append_q(const AppendParams& p, const AppendMaps& maps, const DeviceInfo& di,
                           cudaStream_t st) {
   const size_t smem = AppendSmem<D, Tin>::bytes(p.bits[0], p.bits[1]);
   if ((int)smem > di.max_smem_optin) return TQ_ERR_UNSUPPORTED;
-  auto kern = append_kernel<D, Tin, false, QJL>;
+  auto kern = append_kernel<D, Tin, false, QJL, FIXB>;
   auto kern_safe = append_kernel<D, Tin, true, QJL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
           cudaSuccess ||
@@ -39,7 +41,10 @@ tq_status launch_append_q(const AppendParams& p, const AppendMaps& maps, const D
 template <int D, typename Tin>
 tq_status launch_append_t(const AppendParams& p, const AppendMaps& maps, const DeviceInfo& di,
                           cudaStream_t st) {
-  if (p.kcent == nullptr) return launch_append_q<D, Tin, false>(p, maps, di, st);
+  if (p.kcent == nullptr) {
+    if (p.bits[0] == 4 && p.bits[1] == 4) return launch_append_q<D, Tin, false, 4>(p, maps, di, st);
+    return launch_append_q<D, Tin, false>(p, maps, di, st);
+  }
   if constexpr (D >= 128) return launch_append_q<D, Tin, true>(p, maps, di, st);
   return TQ_ERR_UNSUPPORTED;
 }
